@@ -1,0 +1,232 @@
+"""CPU oracle for group-wise HQQ quantization -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It wraps ``hqq_oracle.c`` (plain scalar
+fp32, see the header comment of that file for the method, its source sections
+and the readings taken) through ctypes.  It shares no code with the CUDA path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hqq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libhqq_oracle.so")
+_CFLAGS = ["-O2", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+           "-shared", "-pthread"]
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle library in-tree (gcc, strict IEEE fp32)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            P = ctypes.c_void_p
+            I64, I, F = ctypes.c_int64, ctypes.c_int, ctypes.c_float
+            lib.hqq_oracle_quantize.argtypes = [P, I64, I, I, F, F, F, I, I, P, P, P, P, P, P]
+            lib.hqq_oracle_quantize.restype = I
+            lib.hqq_oracle_trace_group.argtypes = [P, I, I, F, F, F, I, P, P, P, P, P, P, P, P, P]
+            lib.hqq_oracle_trace_group.restype = I
+            lib.hqq_oracle_shrink.argtypes = [P, I64, F, F, P]
+            lib.hqq_oracle_shrink.restype = None
+            lib.hqq_oracle_z_update.argtypes = [P, P, P, I, F]
+            lib.hqq_oracle_z_update.restype = F
+            lib.hqq_oracle_powp.argtypes = [P, I64, F, P]
+            lib.hqq_oracle_powp.restype = None
+            lib.hqq_oracle_powp_table.argtypes = [F, P, P, P, P]
+            lib.hqq_oracle_powp_table.restype = None
+            lib.hqq_oracle_psum.argtypes = [P, I]
+            lib.hqq_oracle_psum.restype = F
+            lib.hqq_oracle_packed_bytes.argtypes = [I64, I]
+            lib.hqq_oracle_packed_bytes.restype = I64
+            lib.hqq_oracle_pack.argtypes = [P, I64, I, P]
+            lib.hqq_oracle_pack.restype = I
+            lib.hqq_oracle_unpack.argtypes = [P, I64, I, P]
+            lib.hqq_oracle_unpack.restype = I
+            lib.hqq_oracle_dequantize.argtypes = [P, P, P, I64, I, P]
+            lib.hqq_oracle_dequantize.restype = I
+            lib.hqq_oracle_f32_to_f16.argtypes = [P, I64, P]
+            lib.hqq_oracle_f32_to_f16.restype = None
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+DEFAULTS = dict(p=0.7, beta=1.0, kappa=1.01, iters=20)
+
+
+def quantize(W: np.ndarray, nbits: int, group: int, p: float = 0.7, beta: float = 1.0,
+             kappa: float = 1.01, iters: int = 20, threads: int | None = None) -> dict:
+    """HQQ-quantize an fp16 array (any shape, flat size a multiple of ``group``;
+    groups are contiguous runs of ``group`` elements of the flat row-major order).
+
+    Returns codes (uint8 per weight, flat), packed bytes, fp16 scale/zero per
+    group, the fp32 zero and scale, and the accepted-iteration count per group.
+    """
+    lib = _load()
+    W = np.ascontiguousarray(W, dtype=np.float16).reshape(-1)
+    n = W.size
+    if n % group:
+        raise ValueError("size must be a multiple of the group size")
+    ng = n // group
+    codes = np.empty(n, np.uint8)
+    scale = np.empty(ng, np.uint16)
+    zero = np.empty(ng, np.uint16)
+    zf = np.empty(ng, np.float32)
+    sf = np.empty(ng, np.float32)
+    it = np.empty(ng, np.uint8)
+    if threads is None:
+        threads = os.cpu_count() or 1
+    st = lib.hqq_oracle_quantize(_ptr(W.view(np.uint16)), ng, group, nbits, p, beta, kappa,
+                                 iters, threads, _ptr(codes), _ptr(scale), _ptr(zero),
+                                 _ptr(zf), _ptr(sf), _ptr(it))
+    if st:
+        raise ValueError(f"oracle rejected the arguments (status {st})")
+    return dict(codes=codes, packed=pack(codes, nbits), scale=scale.view(np.float16),
+                zero=zero.view(np.float16), zero_f32=zf, scale_f32=sf, iters=it)
+
+
+def trace_group(w, nbits: int, p: float = 0.7, beta: float = 1.0, kappa: float = 1.01,
+                iters: int = 20) -> dict:
+    """Solve one fp32 group and return its whole per-iteration record."""
+    lib = _load()
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    G = w.size
+    T = max(iters, 1)
+    codes = np.empty(G, np.uint8)
+    out6 = np.empty(6, np.float32)
+    counts = np.empty(2, np.int32)
+    z = np.full(T, np.nan, np.float32)
+    e = np.full(T, np.nan, np.float32)
+    bh = np.full(T, np.nan, np.float32)
+    q = np.full((T, G), np.nan, np.float32)
+    d = np.full((T, G), np.nan, np.float32)
+    we = np.full((T, G), np.nan, np.float32)
+    st = lib.hqq_oracle_trace_group(_ptr(w), G, nbits, p, beta, kappa, iters, _ptr(codes),
+                                    _ptr(out6), _ptr(counts), _ptr(z), _ptr(e), _ptr(bh),
+                                    _ptr(q), _ptr(d), _ptr(we))
+    if st:
+        raise ValueError(f"oracle rejected the arguments (status {st})")
+    ne = int(counts[1])
+    return dict(codes=codes, s=out6[0], inv=out6[1], z0=out6[2], z_best=out6[3],
+                e_best=out6[4], accepted=int(counts[0]), evaluations=ne,
+                z=z[:ne], e=e[:ne], beta=bh[:ne], q=q[:ne], d=d[:ne], we=we[:ne])
+
+
+def shrink(x, p: float, beta: float) -> np.ndarray:
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty_like(x)
+    lib.hqq_oracle_shrink(_ptr(x), x.size, p, beta, _ptr(out))
+    return out
+
+
+def z_update(w, q, we, inv: float) -> np.float32:
+    lib = _load()
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    we = np.ascontiguousarray(we, dtype=np.float32)
+    return np.float32(lib.hqq_oracle_z_update(_ptr(w), _ptr(q), _ptr(we), w.size, inv))
+
+
+def powp(x, p: float) -> np.ndarray:
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty_like(x)
+    lib.hqq_oracle_powp(_ptr(x), x.size, p, _ptr(out))
+    return out
+
+
+def powp_table(p: float) -> dict:
+    lib = _load()
+    a = np.empty(256, np.float32)
+    b = np.empty(32, np.float32)
+    c = np.empty(32, np.float32)
+    k = np.empty(3, np.float32)
+    lib.hqq_oracle_powp_table(p, _ptr(a), _ptr(b), _ptr(c), _ptr(k))
+    return dict(two_pk=a, cj_p=b, inv_cj=c, coef=k)
+
+
+def psum(x) -> np.float32:
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    return np.float32(lib.hqq_oracle_psum(_ptr(x), x.size))
+
+
+def packed_bytes(n: int, nbits: int) -> int:
+    return int(_load().hqq_oracle_packed_bytes(n, nbits))
+
+
+def pack(codes, nbits: int) -> np.ndarray:
+    lib = _load()
+    codes = np.ascontiguousarray(codes, dtype=np.uint8).reshape(-1)
+    out = np.empty(packed_bytes(codes.size, nbits), np.uint8)
+    st = lib.hqq_oracle_pack(_ptr(codes), codes.size, nbits, _ptr(out))
+    if st:
+        raise ValueError(f"pack failed (status {st})")
+    return out
+
+
+def unpack(packed, n: int, nbits: int) -> np.ndarray:
+    lib = _load()
+    packed = np.ascontiguousarray(packed, dtype=np.uint8).reshape(-1)
+    if packed.size < packed_bytes(n, nbits):
+        raise ValueError("packed buffer too small")
+    out = np.empty(n, np.uint8)
+    st = lib.hqq_oracle_unpack(_ptr(packed), n, nbits, _ptr(out))
+    if st:
+        raise ValueError(f"unpack failed (status {st})")
+    return out
+
+
+def dequantize(codes, scale, zero, group: int) -> np.ndarray:
+    """W_hat = fp16((c - z) * s) per element, s and z the stored fp16 values."""
+    lib = _load()
+    codes = np.ascontiguousarray(codes, dtype=np.uint8).reshape(-1)
+    scale = np.ascontiguousarray(scale, dtype=np.float16).reshape(-1)
+    zero = np.ascontiguousarray(zero, dtype=np.float16).reshape(-1)
+    out = np.empty(codes.size, np.uint16)
+    st = lib.hqq_oracle_dequantize(_ptr(codes), _ptr(scale.view(np.uint16)),
+                                   _ptr(zero.view(np.uint16)), codes.size, group, _ptr(out))
+    if st:
+        raise ValueError(f"dequantize failed (status {st})")
+    return out.view(np.float16)
+
+
+def f32_to_f16(x) -> np.ndarray:
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.size, np.uint16)
+    lib.hqq_oracle_f32_to_f16(_ptr(x), x.size, _ptr(out))
+    return out.view(np.float16).reshape(x.shape)
+
+
+def lp_error(W, W_hat, p: float = 0.7) -> float:
+    """Per-tensor sum |W - W_hat|^p in fp64 (the parity metric; plain numpy)."""
+    a = np.asarray(W, dtype=np.float64).reshape(-1)
+    b = np.asarray(W_hat, dtype=np.float64).reshape(-1)
+    return float(np.sum(np.abs(a - b) ** p))
