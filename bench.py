@@ -1,0 +1,535 @@
+#!/usr/bin/env python3
+"""Benchmark of the HQQ quantize + dequantize path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole path over the workload's weight set: HQQ
+quantize (fused solver + packing) of every matrix, then dequantize of every
+matrix.  Inputs are generated on the device before timing and stay resident in
+HBM (the default workload holds ~137 GB of fp16 weights, far above the 126 MB
+L2, so no L2 flush is needed between steps).  Under torchrun every rank
+quantizes its own full weight set (weak scaling, no collective on the data
+path); the step time is the max over ranks.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the plain CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Gparams/s quantized & achieved HBM GB/s vs B200 peak; Llama-2-70B-shaped wall time"
+
+# Algorithmic binary32 operations per weight of the canonical solver (see the
+# design notes): initialisation (convert, min, max), one error evaluation
+# (code: fma, 2 clamps, round; residual: sub, fma; |.|; table power: 4 bit-field
+# ops, sub, mul, 3 fma, 2 mul; accumulate), one accepted update with W_e == 0
+# (threshold test, fma, accumulate), final code and packing (fma, 2 clamps,
+# round, shift, or).
+OPS_INIT, OPS_EVAL, OPS_UPDATE, OPS_FINAL = 3, 19, 3, 6
+ALU_LANES_PER_SM = 128
+
+
+# ------------------------------------------------------------------ workloads
+def workload(name: str, rank: int = 0):
+    """List of (label, (rows, cols), nbits, group, seed, stream)."""
+    import synth
+    out = []
+    if name in ("llama2-70b", "llama2-7b"):
+        big = name == "llama2-70b"
+        shapes = synth.llama2_70b_shapes() if big else synth.llama2_7b_shapes()
+        n_layers, seed, nbits = (80, 5, 3) if big else (32, 2, 4)
+        for layer in range(rank * n_layers, (rank + 1) * n_layers):
+            for m in synth.MATRIX_ORDER:
+                out.append((f"L{layer}.{m}", shapes[m], nbits, 64, seed,
+                            synth.stream_id(layer, m)))
+    elif name == "matrix-4096":
+        out.append(("4096x4096 4b g64", (4096, 4096), 4, 64, 1, rank))
+        out.append(("4096x4096 2b g32", (4096, 4096), 2, 32, 1, rank))
+    elif name == "matrix-1024":
+        out.append(("1024x1024 4b g64", (1024, 1024), 4, 64, 0, rank))
+    elif name == "70b-pair":
+        for g in (32, 128):
+            out.append((f"8192x8192 2b g{g}", (8192, 8192), 2, g, 3, 2 * rank))
+            out.append((f"28672x8192 2b g{g}", (28672, 8192), 2, g, 3, 2 * rank + 1))
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    return out
+
+
+def meta_bytes(rows, cols, group):
+    return 2 * 2 * rows * (cols // group)
+
+
+def algorithmic_bytes(mats):
+    """One pass: read fp16 W, write packed codes + fp16 scale and zero."""
+    import weight_only_quantization_b200 as hqq
+    tot = 0
+    for _, (r, c), nb, g, _, _ in mats:
+        tot += 2 * r * c + hqq.hqq_packed_bytes(r, c, nb) + meta_bytes(r, c, g)
+    return tot
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------- helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(mats, W_source, target_s: float):
+    """Bounded sample of the workload for the CPU oracle: the first rows of every
+    distinct (shape, format) in the list, sized to ~target_s seconds of oracle
+    work on this host's cores.  W_source(label, shape, rows) -> fp16 numpy."""
+    import numpy as np
+    import oracle
+    seen, picks = set(), []
+    for lab, shape, nb, g, seed, stream in mats:
+        key = (shape, nb, g)
+        if key not in seen:
+            seen.add(key)
+            picks.append((lab, shape, nb, g, seed, stream))
+    cores = cpu_cores()
+    # probe the rate on 16 rows of the first pick
+    lab, shape, nb, g, seed, stream = picks[0]
+    probe = W_source(lab, shape, 16, seed, stream)
+    t0 = time.perf_counter()
+    oracle.quantize(probe, nb, g, threads=cores)
+    rate = probe.size / max(time.perf_counter() - t0, 1e-6)
+    budget = rate * target_s
+    total_cols = sum(s[1] for _, s, *_ in picks)
+    rows = max(8, min(min(s[0] for _, s, *_ in picks), int(budget / total_cols)))
+    sample = [(lab, W_source(lab, shape, rows, seed, stream), nb, g)
+              for lab, shape, nb, g, seed, stream in picks]
+    desc = ", ".join(f"first {rows} rows of {lab.split('.')[-1]} {shape[0]}x{shape[1]}"
+                     for lab, shape, *_ in picks)
+    return sample, desc, cores
+
+
+def run_oracle_sample(sample, cores):
+    import oracle
+    n = 0
+    t0 = time.perf_counter()
+    for _, W, nb, g in sample:
+        oracle.quantize(W, nb, g, threads=cores)
+        n += W.size
+    return n, time.perf_counter() - t0
+
+
+def config_dict(name, mats, n_gpus):
+    params = sum(r * c for _, (r, c), *_ in mats)
+    fmts = sorted({f"{m[2]}b g{m[3]}" for m in mats})
+    return {"workload": name, "matrices_per_gpu": len(mats), "params_per_gpu": params,
+            "formats": fmts, "solver": {"p": 0.7, "beta": 1.0, "kappa": 1.01, "iters": 20,
+                                        "early_stop": "per group"},
+            "step": "quantize + dequantize of every matrix",
+            "l2": "inputs larger than L2 (no flush needed)" if params * 2 > 4 * 126e6
+            else "L2 flushed between steps",
+            "parallelism": f"replicas x{n_gpus} (weak)"}
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np
+    import synth
+    mats = workload(args.workload, 0)
+
+    use_dev = False
+    try:
+        import torch
+        use_dev = torch.cuda.is_available()
+    except ImportError:
+        pass
+
+    def W_source(lab, shape, rows, seed, stream):
+        # input generation only (the device generator is much faster than numpy's)
+        if use_dev:
+            return synth.student_t_device((rows, shape[1]), seed=seed, stream=stream).cpu().numpy()
+        return synth.student_t_host((rows, shape[1]), seed=seed, stream=stream)
+
+    sample, desc, cores = oracle_sample(mats, W_source, target_s=args.ref_step_s)
+    for _ in range(args.warmup):
+        run_oracle_sample(sample, cores)
+    times, n = [], 0
+    for _ in range(args.steps):
+        n, dt = run_oracle_sample(sample, cores)
+        times.append(dt)
+    total = sum(times)
+    value = n * len(times) / total / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Gparam/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_dict(args.workload, mats, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "Gparam/s", "cores": cores,
+                             "kind": "oracle", "sample": desc + f"; {n} params per step"},
+            "e2e": {"value": value, "unit": "Gparam/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ main arm
+def run_gpu(args):
+    import numpy as np
+    import torch
+
+    import synth
+    import weight_only_quantization_b200 as hqq
+
+    ws, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+        pg = dist
+
+    mats = workload(args.workload, rank)
+    params = sum(r * c for _, (r, c), *_ in mats)
+
+    # ---- resident buffers: weights, packed codes, scale/zero, dequant output
+    offs_w, offs_p, offs_m = [], [], []
+    nw = npk = nm = 0
+    for _, (r, c), nb, g, _, _ in mats:
+        offs_w.append(nw); nw += r * c
+        offs_p.append(npk); npk += (hqq.hqq_packed_bytes(r, c, nb) + 15) // 16 * 16
+        offs_m.append(nm); nm += (r * (c // g) + 7) // 8 * 8
+    maxn = max(r * c for _, (r, c), *_ in mats)
+    need = 2 * nw + npk + 4 * nm + 2 * maxn * 3 + (1 << 30)
+    free_b, _ = torch.cuda.mem_get_info(dev)
+    if need > free_b:
+        raise SystemExit(f"workload {args.workload} needs {need / 1e9:.1f} GB of device memory, "
+                         f"{free_b / 1e9:.1f} GB free")
+    Wbuf = torch.empty(nw, dtype=torch.float16, device=dev)
+    Pbuf = torch.empty(npk, dtype=torch.uint8, device=dev)
+    Sbuf = torch.empty(nm, dtype=torch.float16, device=dev)
+    Zbuf = torch.empty(nm, dtype=torch.float16, device=dev)
+    Obuf = torch.empty(maxn, dtype=torch.float16, device=dev)
+
+    views = []
+    for k, (lab, (r, c), nb, g, seed, stream) in enumerate(mats):
+        W = Wbuf[offs_w[k]:offs_w[k] + r * c].view(r, c)
+        synth.fill_student_t_(W, seed=seed, stream=stream)
+        pb = hqq.hqq_packed_bytes(r, c, nb)
+        P = Pbuf[offs_p[k]:offs_p[k] + pb]
+        mg = r * (c // g)
+        S = Sbuf[offs_m[k]:offs_m[k] + mg].view(r, c // g)
+        Z = Zbuf[offs_m[k]:offs_m[k] + mg].view(r, c // g)
+        q = hqq.QuantizedMatrix(P, S, Z, r, c, nb, g)
+        views.append((W, q, Obuf[:r * c].view(r, c)))
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        for k, (W, q, O) in enumerate(views):
+            if ev is not None:
+                ev[k][0].record(stream)
+            hqq.hqq_quantize(W, q.nbits, q.group, packed=q.packed, scale=q.scale,
+                             zero=q.zero)
+            if ev is not None:
+                ev[k][1].record(stream)
+            hqq.hqq_dequantize(q, out=O)
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in views] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    q_ms = [evs[s][k][0].elapsed_time(evs[s][k][1]) for s in range(args.steps)
+            for k in range(len(views))]
+    ms_t = torch.tensor([ms, sum(q_ms)], dtype=torch.float64, device=dev)
+    if pg is not None:
+        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
+    ms_max, qsum_max = float(ms_t[0]), float(ms_t[1])
+    ms_step = ms_max / args.steps
+    value = ws * params * args.steps / (ms_max / 1e3) / 1e9
+
+    # ---- per-kernel figures (rank 0's launches)
+    q_launch_ms = sum(q_ms) / len(q_ms)
+    dq_ms_step = ms_step - sum(q_ms) / args.steps
+    hbm_peak, peak_kind = measured_peaks()
+    qbytes = algorithmic_bytes(mats)
+    q_step_s = sum(q_ms) / args.steps / 1e3
+    quant_gbs = qbytes / q_step_s / 1e9
+    dq_gbs = qbytes / max(dq_ms_step / 1e3, 1e-9) / 1e9
+
+    # ---- algorithmic ALU work of the solver from the per-group iteration counts
+    acc_hist = np.zeros(256, np.int64)
+    max_groups = max(q.scale.numel() for _, q, _ in views)
+    zf_buf = torch.empty(max_groups, dtype=torch.float32, device=dev)
+    it_buf = torch.empty(max_groups, dtype=torch.uint8, device=dev)
+    for W, q, _ in views:
+        ng = q.scale.numel()
+        qq = hqq.hqq_quantize_ex(W, q.nbits, q.group, packed=q.packed, scale=q.scale,
+                                 zero=q.zero, zero_f32=zf_buf[:ng].view(q.scale.shape),
+                                 iters_out=it_buf[:ng].view(q.scale.shape))
+        acc_hist += torch.bincount(qq.iters.view(-1).long(), minlength=256).cpu().numpy()[:256]
+    torch.cuda.synchronize()
+    del zf_buf, it_buf
+    acc = np.arange(256)
+    evals = np.where(acc < 20, acc + 1, acc)
+    n_groups_hist = acc_hist.sum()
+    mean_acc = float((acc_hist * acc).sum() / n_groups_hist)
+    mean_eval = float((acc_hist * evals).sum() / n_groups_hist)
+    ops_per_weight = OPS_INIT + OPS_FINAL + mean_eval * OPS_EVAL + mean_acc * OPS_UPDATE
+    ops_per_launch = ops_per_weight * params / len(views)
+    props = torch.cuda.get_device_properties(dev)
+    sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
+    alu_peak = props.multi_processor_count * ALU_LANES_PER_SM * sm_mhz * 1e6 / 1e12  # Tops/s
+    achieved = ops_per_launch / (q_launch_ms / 1e3) / 1e12
+
+    line = {"metric": METRIC, "value": value, "unit": "Gparam/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic (Philox Student-t(4), std 0.02, 0.1% x20 outliers, fp16)",
+            "config": config_dict(args.workload, mats, ws),
+            "wall_time_s_per_pass": ms_step / 1e3,
+            "quantize": {"gparam_s": params / q_step_s / 1e9, "gbs": quant_gbs,
+                         "hbm_frac": quant_gbs / hbm_peak, "ms_per_pass": q_step_s * 1e3,
+                         "mean_accepted_iters": mean_acc, "mean_evaluations": mean_eval},
+            "dequantize": {"gbs": dq_gbs, "hbm_frac": dq_gbs / hbm_peak,
+                           "ms_per_pass": dq_ms_step},
+            "roofline": {"kernel": "quantize_kernel", "bound": "alu", "achieved": achieved,
+                         "peak": alu_peak, "unit": "Tops/s", "frac": achieved / alu_peak,
+                         "traffic": None,
+                         "peak_source": f"{props.multi_processor_count} SMs x "
+                                        f"{ALU_LANES_PER_SM} fp32 lanes x {sm_mhz:.0f} MHz",
+                         "ops_per_weight": ops_per_weight,
+                         "hbm": {"achieved_gbs": quant_gbs, "peak_gbs": hbm_peak,
+                                 "frac": quant_gbs / hbm_peak, "peak_kind": peak_kind}},
+            "gpu_launches": 2 * len(views) * args.steps,
+            "clocks": clk}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    if ws == 1 and not args.no_cpu_baseline:
+        def W_source(lab, shape, rows, seed, stream_):
+            k = [m[0] for m in mats].index(lab)
+            return views[k][0][:rows].cpu().numpy()
+        sample, desc, cores = oracle_sample(mats, W_source, target_s=args.cpu_s)
+        n, dt = run_oracle_sample(sample, cores)
+        line["cpu_baseline"] = {"value": n / dt / 1e9, "unit": "Gparam/s", "cores": cores,
+                                "kind": "oracle", "sample": desc + f"; {n} params, {dt:.1f} s"}
+
+    # ---- end to end through the public API with host buffers
+    line["e2e"] = run_e2e(args, mats, views, hqq, dev, pg, ws)
+
+    del views, Wbuf, Pbuf, Sbuf, Zbuf, Obuf
+    if rank == 0:
+        print(json.dumps(line))
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, mats, views, hqq, dev, pg, ws):
+    """Same metric, through the API with pinned host buffers: every step copies
+    each matrix's fp16 weights host->device, quantizes + dequantizes it, and
+    copies the packed codes, scale and zero back.  Host data: one pinned buffer
+    per matrix kind (the first layer's values), reused by every layer."""
+    import torch
+    kinds = {}
+    for k, (lab, shape, nb, g, seed, stream) in enumerate(mats):
+        kind = lab.split(".")[-1]
+        if kind not in kinds:
+            kinds[kind] = views[k][0].cpu().pin_memory()
+    host_out = {}
+    for k, (lab, (r, c), nb, g, *_ ) in enumerate(mats):
+        kind = lab.split(".")[-1]
+        if kind not in host_out:
+            q = views[k][1]
+            host_out[kind] = (torch.empty(q.packed.numel(), dtype=torch.uint8, pin_memory=True),
+                              torch.empty(q.scale.shape, dtype=torch.float16, pin_memory=True),
+                              torch.empty(q.zero.shape, dtype=torch.float16, pin_memory=True))
+    maxn = max(r * c for _, (r, c), *_ in mats)
+    dW = [torch.empty(maxn, dtype=torch.float16, device=dev) for _ in range(2)]
+    s_copy = torch.cuda.Stream(dev)
+    s_comp = torch.cuda.current_stream(dev)
+    s_back = torch.cuda.Stream(dev)
+    h2d = d2h = 0
+
+    def one_step():
+        nonlocal h2d, d2h
+        h2d = d2h = 0
+        ready = [torch.cuda.Event() for _ in range(2)]
+        free = [torch.cuda.Event() for _ in range(2)]
+        done = []
+        for k, (lab, (r, c), nb, g, *_ ) in enumerate(mats):
+            kind = lab.split(".")[-1]
+            b = k % 2
+            with torch.cuda.stream(s_copy):
+                if k >= 2:
+                    s_copy.wait_event(free[b])
+                dst = dW[b][:r * c].view(r, c)
+                dst.copy_(kinds[kind], non_blocking=True)
+                ready[b].record(s_copy)
+            h2d += 2 * r * c
+            s_comp.wait_event(ready[b])
+            _, q, O = views[k]
+            hqq.hqq_quantize(dst, nb, g, packed=q.packed, scale=q.scale, zero=q.zero)
+            free[b].record(s_comp)
+            hqq.hqq_dequantize(q, out=O)
+            ev = torch.cuda.Event()
+            ev.record(s_comp)
+            with torch.cuda.stream(s_back):
+                s_back.wait_event(ev)
+                hp, hs, hz = host_out[kind]
+                hp.copy_(q.packed, non_blocking=True)
+                hs.copy_(q.scale, non_blocking=True)
+                hz.copy_(q.zero, non_blocking=True)
+            d2h += q.packed.numel() + 2 * q.scale.numel() + 2 * q.zero.numel()
+        s_comp.wait_stream(s_back)
+        s_comp.wait_stream(s_copy)
+
+    steps = max(1, min(args.steps, args.e2e_steps))
+    one_step()
+    torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_comp)
+    for _ in range(steps):
+        one_step()
+    t1.record(s_comp)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if pg is not None:
+        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
+    params = sum(r * c for _, (r, c), *_ in mats)
+    return {"value": ws * params * steps / (float(ms_t[0]) / 1e3) / 1e9, "unit": "Gparam/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "warmup": 1, "ms_per_step": float(ms_t[0]) / steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama2-70b",
+                    choices=["llama2-70b", "llama2-7b", "matrix-4096", "matrix-1024", "70b-pair"])
+    ap.add_argument("--impl", default="libhqq", choices=["libhqq", "reference"])
+    ap.add_argument("--cpu-s", type=float, default=10.0, help="oracle CPU-baseline budget (s)")
+    ap.add_argument("--ref-step-s", type=float, default=4.0, help="reference arm seconds per step")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl != "reference":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

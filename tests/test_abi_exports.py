@@ -1,0 +1,100 @@
+"""The C ABI library loads on a machine without a GPU, exports every entry point
+declared in include/hqq.h, and rejects bad arguments on the host before any
+CUDA call.  No compute call is made here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hqq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from weight_only_quantization_b200 import build
+    build.build()
+    import weight_only_quantization_b200 as hqq
+    return hqq
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hqq_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ["hqq_quantize", "hqq_quantize_ex", "hqq_dequantize", "hqq_packed_bytes",
+                 "hqq_status_string"]:
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (hqq_\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib._lib, name)
+
+
+def test_header_compiles_as_c():
+    src = '#include "hqq.h"\nint main(void){return (int)hqq_packed_bytes(1,16,4);}\n'
+    res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-x", "c",
+                          "-I", os.path.join(ROOT, "include"), "-"], input=src, text=True,
+                         capture_output=True)
+    assert res.returncode == 0, res.stderr
+
+
+def test_packed_bytes(lib):
+    assert lib.hqq_packed_bytes(4096, 4096, 4) == 4096 * 4096 // 2
+    assert lib.hqq_packed_bytes(4096, 4096, 2) == 4096 * 4096 // 4
+    assert lib.hqq_packed_bytes(4096, 4096, 3) == 4 * ((4096 * 4096 + 9) // 10)
+    assert lib.hqq_packed_bytes(1, 64, 3) == 28
+    assert lib._lib.hqq_packed_bytes(-1, 64, 4) == -1
+    assert lib._lib.hqq_packed_bytes(4, 64, 5) == -1
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.hqq_status_string(s).startswith("HQQ_")
+    assert "unknown" in lib.hqq_status_string(99)
+
+
+def test_host_validation_without_gpu(lib):
+    L = lib._lib
+    P = lambda v: ctypes.c_void_p(v)
+    a = dict(rows=64, cols=256, nbits=4, group=64, p=0.7, beta=1.0, kappa=1.01, iters=20)
+    cases = [
+        (dict(nbits=5), 3), (dict(nbits=1), 3), (dict(group=48), 3), (dict(group=8), 3),
+        (dict(group=512), 3), (dict(cols=250), 2), (dict(rows=-3), 2),
+        (dict(p=0.0), 4), (dict(p=1.0001), 4), (dict(p=float("nan")), 4),
+        (dict(beta=0.0), 4), (dict(beta=float("inf")), 4), (dict(kappa=0.0), 4),
+        (dict(kappa=float("nan")), 4), (dict(iters=-1), 4), (dict(iters=256), 4),
+    ]
+    for over, want in cases:
+        b = dict(a, **over)
+        st = L.hqq_quantize(P(256), b["rows"], b["cols"], b["nbits"], b["group"], b["p"],
+                            b["beta"], b["kappa"], b["iters"], P(256), P(256), P(256), None)
+        assert st == want, (over, st)
+    # null and misaligned pointers
+    assert L.hqq_quantize(None, 64, 256, 4, 64, 0.7, 1.0, 1.01, 20, P(256), P(256), P(256),
+                          None) == 1
+    assert L.hqq_quantize(P(258), 64, 256, 4, 64, 0.7, 1.0, 1.01, 20, P(256), P(256), P(256),
+                          None) == 5
+    assert L.hqq_quantize(P(256), 64, 256, 4, 64, 0.7, 1.0, 1.01, 20, P(258), P(256), P(256),
+                          None) == 5
+    assert L.hqq_quantize_ex(P(256), 64, 256, 4, 64, 0.7, 1.0, 1.01, 20, P(256), P(256),
+                             P(256), P(258), None, None) == 5
+    # empty matrices are valid no-ops (nothing launched, so no GPU needed)
+    assert L.hqq_quantize(None, 0, 256, 4, 64, 0.7, 1.0, 1.01, 20, None, None, None, None) == 0
+    assert L.hqq_dequantize(None, None, None, 16, 0, 3, 64, None, None) == 0
+    # dequantize validation
+    assert L.hqq_dequantize(P(256), P(256), P(256), 64, 256, 6, 64, P(256), None) == 3
+    assert L.hqq_dequantize(P(256), P(256), None, 64, 256, 4, 64, P(256), None) == 1
+    assert L.hqq_dequantize(P(256), P(256), P(256), 64, 256, 4, 64, P(264), None) == 5
+    assert L.hqq_dequantize(P(256), P(256), P(256), 64, 100, 4, 64, P(256), None) == 2

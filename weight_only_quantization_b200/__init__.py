@@ -1,0 +1,158 @@
+"""Python binding of libhqq (include/hqq.h): HQQ group-wise weight-only
+quantization of fp16 weight matrices on NVIDIA B200 (sm_100a).
+
+Argument marshalling only: every step of the quantization and dequantization
+runs in libhqq's CUDA kernels.  torch supplies device memory and the current
+stream.  There is no fallback: importing fails loudly when libhqq.so is absent,
+and every call raises ``HQQError`` on a non-zero status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+__all__ = ["HQQError", "hqq_quantize", "hqq_quantize_ex", "hqq_dequantize",
+           "hqq_packed_bytes", "hqq_status_string", "QuantizedMatrix", "LIB_PATH",
+           "DEFAULT_P", "DEFAULT_BETA", "DEFAULT_KAPPA", "DEFAULT_ITERS"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhqq.so")
+
+DEFAULT_P, DEFAULT_BETA, DEFAULT_KAPPA, DEFAULT_ITERS = 0.7, 1.0, 1.01, 20
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m weight_only_quantization_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P, _I64, _I, _F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+_lib.hqq_packed_bytes.argtypes = [_I64, _I64, _I]
+_lib.hqq_packed_bytes.restype = _I64
+_lib.hqq_status_string.argtypes = [_I]
+_lib.hqq_status_string.restype = ctypes.c_char_p
+_lib.hqq_quantize.argtypes = [_P, _I64, _I64, _I, _I, _F, _F, _F, _I, _P, _P, _P, _P]
+_lib.hqq_quantize.restype = _I
+_lib.hqq_quantize_ex.argtypes = [_P, _I64, _I64, _I, _I, _F, _F, _F, _I, _P, _P, _P, _P, _P, _P]
+_lib.hqq_quantize_ex.restype = _I
+_lib.hqq_dequantize.argtypes = [_P, _P, _P, _I64, _I64, _I, _I, _P, _P]
+_lib.hqq_dequantize.restype = _I
+
+
+class HQQError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        super().__init__(hqq_status_string(status))
+
+
+def hqq_status_string(status: int) -> str:
+    return _lib.hqq_status_string(status).decode()
+
+
+def hqq_packed_bytes(rows: int, cols: int, nbits: int) -> int:
+    n = _lib.hqq_packed_bytes(rows, cols, nbits)
+    if n < 0:
+        raise HQQError(2 if nbits in (2, 3, 4) else 3)
+    return int(n)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(st: int):
+    if st != 0:
+        raise HQQError(st)
+
+
+@dataclass
+class QuantizedMatrix:
+    """Packed codes + fp16 scale/zero of one [rows, cols] matrix."""
+    packed: "torch.Tensor"     # uint8 [hqq_packed_bytes]
+    scale: "torch.Tensor"      # fp16 [rows, cols/group]
+    zero: "torch.Tensor"       # fp16 [rows, cols/group]
+    rows: int
+    cols: int
+    nbits: int
+    group: int
+    zero_f32: "torch.Tensor | None" = None
+    iters: "torch.Tensor | None" = None
+
+
+def _outputs(W, nbits, group, packed, scale, zero):
+    import torch
+    rows, cols = W.shape
+    if packed is None:
+        packed = torch.empty(hqq_packed_bytes(rows, cols, nbits), dtype=torch.uint8,
+                             device=W.device)
+    meta = (rows, cols // group if group > 0 else 0)
+    if scale is None:
+        scale = torch.empty(meta, dtype=torch.float16, device=W.device)
+    if zero is None:
+        zero = torch.empty(meta, dtype=torch.float16, device=W.device)
+    return packed, scale, zero
+
+
+def _check_tensor(t, name):
+    if t is not None and not (t.is_cuda and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def hqq_quantize(W, nbits: int = 4, group: int = 64, p: float = DEFAULT_P,
+                 beta: float = DEFAULT_BETA, kappa: float = DEFAULT_KAPPA,
+                 iters: int = DEFAULT_ITERS, packed=None, scale=None, zero=None,
+                 stream=None) -> QuantizedMatrix:
+    """Quantize a contiguous fp16 CUDA matrix [rows, cols] (see include/hqq.h)."""
+    import torch
+    if W.dtype != torch.float16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float16 tensor")
+    for t, n in ((W, "W"), (packed, "packed"), (scale, "scale"), (zero, "zero")):
+        _check_tensor(t, n)
+    packed, scale, zero = _outputs(W, nbits, group, packed, scale, zero)
+    rows, cols = W.shape
+    _check(_lib.hqq_quantize(_ptr(W), rows, cols, nbits, group, p, beta, kappa, iters,
+                             _ptr(packed), _ptr(scale), _ptr(zero), _stream(stream)))
+    return QuantizedMatrix(packed, scale, zero, rows, cols, nbits, group)
+
+
+def hqq_quantize_ex(W, nbits: int = 4, group: int = 64, p: float = DEFAULT_P,
+                    beta: float = DEFAULT_BETA, kappa: float = DEFAULT_KAPPA,
+                    iters: int = DEFAULT_ITERS, packed=None, scale=None, zero=None,
+                    zero_f32=None, iters_out=None, stream=None) -> QuantizedMatrix:
+    """hqq_quantize plus the fp32 zero and accepted-iteration count per group."""
+    import torch
+    if W.dtype != torch.float16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float16 tensor")
+    for t, n in ((W, "W"), (packed, "packed"), (scale, "scale"), (zero, "zero"),
+                 (zero_f32, "zero_f32"), (iters_out, "iters_out")):
+        _check_tensor(t, n)
+    packed, scale, zero = _outputs(W, nbits, group, packed, scale, zero)
+    rows, cols = W.shape
+    meta = (rows, cols // group if group > 0 else 0)
+    if zero_f32 is None:
+        zero_f32 = torch.empty(meta, dtype=torch.float32, device=W.device)
+    if iters_out is None:
+        iters_out = torch.empty(meta, dtype=torch.uint8, device=W.device)
+    _check(_lib.hqq_quantize_ex(_ptr(W), rows, cols, nbits, group, p, beta, kappa, iters,
+                                _ptr(packed), _ptr(scale), _ptr(zero), _ptr(zero_f32),
+                                _ptr(iters_out), _stream(stream)))
+    return QuantizedMatrix(packed, scale, zero, rows, cols, nbits, group, zero_f32, iters_out)
+
+
+def hqq_dequantize(q: QuantizedMatrix, out=None, stream=None):
+    """fp16 [rows, cols] = (code - zero) * scale  (see include/hqq.h)."""
+    import torch
+    for t, n in ((q.packed, "packed"), (q.scale, "scale"), (q.zero, "zero"), (out, "out")):
+        _check_tensor(t, n)
+    if out is None:
+        out = torch.empty((q.rows, q.cols), dtype=torch.float16, device=q.packed.device)
+    _check(_lib.hqq_dequantize(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols,
+                               q.nbits, q.group, _ptr(out), _stream(stream)))
+    return out

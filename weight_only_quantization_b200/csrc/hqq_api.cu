@@ -1,0 +1,183 @@
+// hqq_api.cu -- the extern "C" boundary of libhqq (declared in include/hqq.h):
+// host-side validation, the per-call power tables and shrink thresholds, and
+// kernel dispatch.  Nothing is launched unless every check passes.
+#include <cmath>
+#include <cstring>
+
+#include "../../include/hqq.h"
+#include "hqq_common.cuh"
+
+namespace hqq {
+cudaError_t launch_quantize(const QuantParams& prm, int nbits, int group, cudaStream_t stream);
+cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_group,
+                              cudaStream_t stream);
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int log2_of_group(int group) {
+    switch (group) {
+        case 16: return 4;
+        case 32: return 5;
+        case 64: return 6;
+        case 128: return 7;
+        case 256: return 8;
+        default: return -1;
+    }
+}
+
+// Table of |x|^p for one exponent p (see PowTable).  Each entry is the double
+// library value rounded once to binary32.
+void build_pow_table(PowTable& t, float p) {
+    const double pd = (double)p;
+    for (int e = 0; e < 256; ++e) {
+        if (e == 0)
+            t.two_pk[e] = p > 0.0f ? 0.0f : (p < 0.0f ? INFINITY : 1.0f);
+        else if (e == 255)
+            t.two_pk[e] = p > 0.0f ? INFINITY : (p < 0.0f ? 0.0f : 1.0f);
+        else
+            t.two_pk[e] = (float)std::exp2(pd * (double)(e - 127));
+    }
+    for (int j = 0; j < 32; ++j) {
+        const double c = 1.0 + (double)(2 * j + 1) / 64.0;
+        t.cj_p[j] = (float)std::pow(c, pd);
+        const float cf = (float)c;
+        t.inv_cj[j] = 1.0f / cf;
+    }
+    t.a1 = p;
+    t.a2 = (float)(pd * (pd - 1.0) / 2.0);
+    t.a3 = (float)(pd * (pd - 1.0) * (pd - 2.0) / 6.0);
+}
+
+// Tables depend on p only; reuse them across calls made by the same host thread.
+struct TableCache {
+    bool valid = false;
+    uint32_t p_bits = 0;
+    PowTable tp, tq;
+};
+thread_local TableCache g_cache;
+
+int validate_common(int64_t rows, int64_t cols, int nbits, int group) {
+    if (rows < 0 || cols < 0) return HQQ_ERR_SHAPE;
+    if (nbits != 2 && nbits != 3 && nbits != 4) return HQQ_ERR_UNSUPPORTED;
+    if (log2_of_group(group) < 0) return HQQ_ERR_UNSUPPORTED;
+    if (cols % group != 0) return HQQ_ERR_SHAPE;
+    if (rows > 0 && cols > ((int64_t)1 << 46) / rows) return HQQ_ERR_SHAPE;
+    return HQQ_OK;
+}
+
+}  // namespace
+}  // namespace hqq
+
+using namespace hqq;
+
+extern "C" int64_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits) {
+    if (rows < 0 || cols < 0) return -1;
+    if (rows > 0 && cols > ((int64_t)1 << 46) / rows) return -1;
+    const int64_t n = rows * cols;
+    switch (nbits) {
+        case 4: return (n + 1) / 2;
+        case 2: return (n + 3) / 4;
+        case 3: return 4 * ((n + 9) / 10);
+        default: return -1;
+    }
+}
+
+extern "C" const char* hqq_status_string(int status) {
+    switch (status) {
+        case HQQ_OK: return "HQQ_OK";
+        case HQQ_ERR_NULL: return "HQQ_ERR_NULL: a required pointer is NULL";
+        case HQQ_ERR_SHAPE: return "HQQ_ERR_SHAPE: bad rows/cols or cols not a multiple of group";
+        case HQQ_ERR_UNSUPPORTED: return "HQQ_ERR_UNSUPPORTED: nbits must be 2/3/4, group 16..256 (power of two)";
+        case HQQ_ERR_PARAM: return "HQQ_ERR_PARAM: need 0<p<=1, beta>0, kappa>0 (finite), 0<=iters<=255";
+        case HQQ_ERR_ALIGN: return "HQQ_ERR_ALIGN: W/W_out need 16-byte, packed/zero_f32 4-byte, scale/zero 2-byte alignment";
+        case HQQ_ERR_CUDA: return "HQQ_ERR_CUDA: kernel launch failed (see cudaGetLastError)";
+        default: return "HQQ: unknown status";
+    }
+}
+
+extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nbits, int group,
+                               float p, float beta, float kappa, int iters, void* packed,
+                               void* scale, void* zero, float* zero_f32, uint8_t* iters_out,
+                               void* stream) {
+    int st = validate_common(rows, cols, nbits, group);
+    if (st != HQQ_OK) return st;
+    if (!(p > 0.0f && p <= 1.0f)) return HQQ_ERR_PARAM;
+    if (!(beta > 0.0f) || !std::isfinite(beta)) return HQQ_ERR_PARAM;
+    if (!(kappa > 0.0f) || !std::isfinite(kappa)) return HQQ_ERR_PARAM;
+    if (iters < 0 || iters > kMaxIters) return HQQ_ERR_PARAM;
+    const int64_t n = rows * cols;
+    if (n == 0) return HQQ_OK;
+    if (!W || !packed || !scale || !zero) return HQQ_ERR_NULL;
+    if (!aligned(W, 16) || !aligned(packed, 4) || !aligned(scale, 2) || !aligned(zero, 2) ||
+        (zero_f32 && !aligned(zero_f32, 4)))
+        return HQQ_ERR_ALIGN;
+
+    QuantParams prm;
+    std::memset(&prm, 0, sizeof prm);
+    prm.W = static_cast<const __half*>(W);
+    prm.packed = static_cast<uint8_t*>(packed);
+    prm.scale = static_cast<__half*>(scale);
+    prm.zero = static_cast<__half*>(zero);
+    prm.zero_f32 = zero_f32;
+    prm.iters_out = iters_out;
+    prm.n_groups = n / group;
+    prm.n_elems = n;
+    prm.iters = iters;
+    prm.beta = beta;
+    prm.kappa = kappa;
+
+    uint32_t pbits;
+    std::memcpy(&pbits, &p, 4);
+    if (!g_cache.valid || g_cache.p_bits != pbits) {
+        build_pow_table(g_cache.tp, p);
+        build_pow_table(g_cache.tq, p - 1.0f);
+        g_cache.p_bits = pbits;
+        g_cache.valid = true;
+    }
+    prm.tp = g_cache.tp;
+    prm.tq = g_cache.tq;
+
+    // Shrink shortcut: |r| - |r|^(p-1)/beta > 0  <=>  |r| > beta^(-1/(2-p)).  Below
+    // the threshold lowered by a 1e-4 relative margin (far above the rounding
+    // error of the table power), W_e is exactly zero, so the kernel may skip it.
+    float bt = beta;
+    for (int t = 0; t < iters; ++t) {
+        const double T = std::pow((double)bt, -1.0 / (2.0 - (double)p));
+        prm.shrink_thr[t] = (float)(T * (1.0 - 1e-4));
+        bt = bt * kappa;
+    }
+
+    const cudaError_t err = launch_quantize(prm, nbits, group, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
+extern "C" int hqq_quantize(const void* W, int64_t rows, int64_t cols, int nbits, int group,
+                            float p, float beta, float kappa, int iters, void* packed,
+                            void* scale, void* zero, void* stream) {
+    return hqq_quantize_ex(W, rows, cols, nbits, group, p, beta, kappa, iters, packed, scale,
+                           zero, nullptr, nullptr, stream);
+}
+
+extern "C" int hqq_dequantize(const void* packed, const void* scale, const void* zero,
+                              int64_t rows, int64_t cols, int nbits, int group, void* W_out,
+                              void* stream) {
+    int st = validate_common(rows, cols, nbits, group);
+    if (st != HQQ_OK) return st;
+    const int64_t n = rows * cols;
+    if (n == 0) return HQQ_OK;
+    if (!packed || !scale || !zero || !W_out) return HQQ_ERR_NULL;
+    if (!aligned(packed, 4) || !aligned(scale, 2) || !aligned(zero, 2) || !aligned(W_out, 16))
+        return HQQ_ERR_ALIGN;
+    DequantParams prm;
+    prm.packed = static_cast<const uint8_t*>(packed);
+    prm.scale = static_cast<const __half*>(scale);
+    prm.zero = static_cast<const __half*>(zero);
+    prm.out = static_cast<__half*>(W_out);
+    prm.n_units = n / 8;
+    prm.group = group;
+    const cudaError_t err = launch_dequantize(prm, nbits, log2_of_group(group),
+                                              static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
