@@ -38,10 +38,11 @@
  * |x|^p is the table-driven power "powp" (in the spirit of P. T. P. Tang,
  * "Table-driven implementation of the exponential function", ACM TOMS 15(2),
  * 1989): x = 2^k * m, m in [1,2); c_j = 1 + (2j+1)/64 is the centre of m's
- * 1/32-wide cell; m^p = c_j^p (1+r)^p with r = (m - c_j)/c_j, |r| <= 1/64, and
- * (1+r)^p is the binomial series to the cubic term.  The 2^(p k) and c_j^p
- * entries are the double-precision library values rounded once to binary32.
- * Zero and subnormal x give 0 (p > 0), +inf (p < 0), 1 (p == 0).
+ * 1/32-wide cell; m^p = c_j^p (1+r)^p with r = m/c_j - 1, |r| <= 1/64, formed
+ * as one fused multiply-add of m and fl(1/c_j), and (1+r)^p is the binomial
+ * series to the cubic term.  The 2^(p k) and c_j^p entries are the
+ * double-precision library values rounded once to binary32.  Zero and
+ * subnormal x give 0 (p > 0), +inf (p < 0), 1 (p == 0).
  */
 #include <math.h>
 #include <pthread.h>
@@ -105,8 +106,7 @@ static float powp(const powp_table *t, float x) {
     const uint32_t e = b >> 23;
     const uint32_t j = (b >> 18) & 31u;
     const float m = u2f((b & 0x007FFFFFu) | 0x3F800000u);   /* mantissa in [1,2) */
-    const float c = u2f((b & 0x007C0000u) | 0x3F820000u);   /* cell centre c_j   */
-    const float r = (m - c) * t->inv_cj[j];                  /* m - c is exact    */
+    const float r = fmaf(m, t->inv_cj[j], -1.0f);            /* m / c_j - 1       */
     const float poly = fmaf(fmaf(fmaf(r, t->a3, t->a2), r, t->a1), r, 1.0f);
     return (t->two_pk[e] * t->cj_p[j]) * poly;
 }
