@@ -43,7 +43,7 @@ ALU_LANES_PER_SM = 128
 
 
 # ------------------------------------------------------------------ workloads
-def workload(name: str, rank: int = 0):
+def workload(name: str, rank: int = 0, layers: int | None = None):
     """List of (label, (rows, cols), nbits, group, seed, stream)."""
     import synth
     out = []
@@ -51,6 +51,8 @@ def workload(name: str, rank: int = 0):
         big = name == "llama2-70b"
         shapes = synth.llama2_70b_shapes() if big else synth.llama2_7b_shapes()
         n_layers, seed, nbits = (80, 5, 3) if big else (32, 2, 4)
+        if layers is not None:
+            n_layers = min(n_layers, layers)
         for layer in range(rank * n_layers, (rank + 1) * n_layers):
             for m in synth.MATRIX_ORDER:
                 out.append((f"L{layer}.{m}", shapes[m], nbits, 64, seed,
@@ -58,6 +60,8 @@ def workload(name: str, rank: int = 0):
     elif name == "matrix-4096":
         out.append(("4096x4096 4b g64", (4096, 4096), 4, 64, 1, rank))
         out.append(("4096x4096 2b g32", (4096, 4096), 2, 32, 1, rank))
+    elif name == "gate-70b":
+        out.append(("L0.gate 28672x8192 3b g64", (28672, 8192), 3, 64, 5, rank * 7 + 4))
     elif name == "matrix-1024":
         out.append(("1024x1024 4b g64", (1024, 1024), 4, 64, 0, rank))
     elif name == "70b-pair":
@@ -216,7 +220,7 @@ def run_reference(args):
         return 0
     import numpy as np
     import synth
-    mats = workload(args.workload, 0)
+    mats = workload(args.workload, 0, args.layers)
 
     use_dev = False
     try:
@@ -274,7 +278,7 @@ def run_gpu(args):
                                 device_id=dev)
         pg = dist
 
-    mats = workload(args.workload, rank)
+    mats = workload(args.workload, rank, args.layers)
     params = sum(r * c for _, (r, c), *_ in mats)
 
     # ---- resident buffers: weights, packed codes, scale/zero, dequant output
@@ -415,12 +419,18 @@ def run_gpu(args):
             k = [m[0] for m in mats].index(lab)
             return views[k][0][:rows].cpu().numpy()
         sample, desc, cores = oracle_sample(mats, W_source, target_s=args.cpu_s)
-        n, dt = run_oracle_sample(sample, cores)
+        n = dt = 0.0
+        reps = 0
+        while dt < args.cpu_s and reps < 100:
+            n1, dt1 = run_oracle_sample(sample, cores)
+            n, dt, reps = n + n1, dt + dt1, reps + 1
+        desc += f"; repeated {reps}x"
         line["cpu_baseline"] = {"value": n / dt / 1e9, "unit": "Gparam/s", "cores": cores,
                                 "kind": "oracle", "sample": desc + f"; {n} params, {dt:.1f} s"}
 
     # ---- end to end through the public API with host buffers
-    line["e2e"] = run_e2e(args, mats, views, hqq, dev, pg, ws)
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, mats, views, hqq, dev, pg, ws)
 
     del views, Wbuf, Pbuf, Sbuf, Zbuf, Obuf
     if rank == 0:
@@ -517,7 +527,11 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="llama2-70b",
-                    choices=["llama2-70b", "llama2-7b", "matrix-4096", "matrix-1024", "70b-pair"])
+                    choices=["llama2-70b", "llama2-7b", "matrix-4096", "matrix-1024", "70b-pair",
+                             "gate-70b"])
+    ap.add_argument("--layers", type=int, default=None,
+                    help="first N layers only of a model-shaped set (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
     ap.add_argument("--impl", default="libhqq", choices=["libhqq", "reference"])
     ap.add_argument("--cpu-s", type=float, default=10.0, help="oracle CPU-baseline budget (s)")
     ap.add_argument("--ref-step-s", type=float, default=4.0, help="reference arm seconds per step")

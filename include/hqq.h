@@ -42,8 +42,8 @@ typedef enum hqq_status {
     HQQ_ERR_UNSUPPORTED = 3, /* nbits not in {2,3,4}, group not in {16..256, 2^k} */
     HQQ_ERR_PARAM = 4,       /* p not in (0,1], beta/kappa not > 0 and finite,
                                 iters not in [0,255]                             */
-    HQQ_ERR_ALIGN = 5,       /* W / W_out not 16-byte aligned, packed or
-                                zero_f32 not 4-byte, scale/zero not 2-byte       */
+    HQQ_ERR_ALIGN = 5,       /* W / W_out not 16-byte aligned; packed, zero_f32
+                                or err_out not 4-byte; scale/zero not 2-byte     */
     HQQ_ERR_CUDA = 6         /* the kernel launch failed                         */
 } hqq_status;
 
@@ -98,9 +98,12 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int nbits, int group
                  void* packed, void* scale, void* zero, void* stream);
 
 /*
- * hqq_quantize_ex -- hqq_quantize plus two optional per-group diagnostics
- * (either may be NULL):
+ * hqq_quantize_ex -- hqq_quantize plus three optional per-group diagnostics
+ * (any may be NULL; the float arrays must be 4-byte aligned):
  *   zero_f32  [out] float [rows, cols/group]: z_best before fp16 rounding.
+ *   err_out   [out] float [rows, cols/group]: the solver's binary32 error sum
+ *                   over the group of |W - s(Wq - z_best)|^p (the accepted
+ *                   minimum); +inf when iters = 0 (no evaluation is made).
  *   iters_out [out] uint8 [rows, cols/group]: accepted iterations (0..iters);
  *                   a group evaluated its error iters_out+1 times, or iters
  *                   times when it never stopped early.
@@ -108,7 +111,7 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int nbits, int group
 int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nbits, int group,
                     float p, float beta, float kappa, int iters,
                     void* packed, void* scale, void* zero,
-                    float* zero_f32, uint8_t* iters_out, void* stream);
+                    float* zero_f32, float* err_out, uint8_t* iters_out, void* stream);
 
 /*
  * hqq_dequantize -- Q^-1 of the method's section 2: W_hat = s (Wq - z), computed

@@ -41,7 +41,7 @@ def _load():
             lib = ctypes.CDLL(_LIB_PATH)
             P = ctypes.c_void_p
             I64, I, F = ctypes.c_int64, ctypes.c_int, ctypes.c_float
-            lib.hqq_oracle_quantize.argtypes = [P, I64, I, I, F, F, F, I, I, P, P, P, P, P, P]
+            lib.hqq_oracle_quantize.argtypes = [P, I64, I, I, F, F, F, I, I, P, P, P, P, P, P, P]
             lib.hqq_oracle_quantize.restype = I
             lib.hqq_oracle_trace_group.argtypes = [P, I, I, F, F, F, I, P, P, P, P, P, P, P, P, P]
             lib.hqq_oracle_trace_group.restype = I
@@ -85,7 +85,8 @@ def quantize(W: np.ndarray, nbits: int, group: int, p: float = 0.7, beta: float 
     groups are contiguous runs of ``group`` elements of the flat row-major order).
 
     Returns codes (uint8 per weight, flat), packed bytes, fp16 scale/zero per
-    group, the fp32 zero and scale, and the accepted-iteration count per group.
+    group, the fp32 zero and scale, the accepted minimum of the error sum
+    (+inf when iters = 0) and the accepted-iteration count per group.
     """
     lib = _load()
     W = np.ascontiguousarray(W, dtype=np.float16).reshape(-1)
@@ -99,15 +100,16 @@ def quantize(W: np.ndarray, nbits: int, group: int, p: float = 0.7, beta: float 
     zf = np.empty(ng, np.float32)
     sf = np.empty(ng, np.float32)
     it = np.empty(ng, np.uint8)
+    err = np.empty(ng, np.float32)
     if threads is None:
         threads = os.cpu_count() or 1
     st = lib.hqq_oracle_quantize(_ptr(W.view(np.uint16)), ng, group, nbits, p, beta, kappa,
                                  iters, threads, _ptr(codes), _ptr(scale), _ptr(zero),
-                                 _ptr(zf), _ptr(sf), _ptr(it))
+                                 _ptr(zf), _ptr(sf), _ptr(err), _ptr(it))
     if st:
         raise ValueError(f"oracle rejected the arguments (status {st})")
     return dict(codes=codes, packed=pack(codes, nbits), scale=scale.view(np.float16),
-                zero=zero.view(np.float16), zero_f32=zf, scale_f32=sf, iters=it)
+                zero=zero.view(np.float16), zero_f32=zf, scale_f32=sf, err=err, iters=it)
 
 
 def trace_group(w, nbits: int, p: float = 0.7, beta: float = 1.0, kappa: float = 1.01,

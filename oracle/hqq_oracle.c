@@ -250,7 +250,7 @@ typedef struct {
     int64_t g0, g1;
     uint8_t *codes;
     uint16_t *scale, *zero;
-    float *zero_f32, *scale_f32;
+    float *zero_f32, *scale_f32, *err;
     uint8_t *iters_out;
 } work_range;
 
@@ -267,6 +267,7 @@ static void *run_range(void *arg) {
         wr->zero[g] = float_to_half_bits(r.z_best);
         if (wr->zero_f32) wr->zero_f32[g] = r.z_best;
         if (wr->scale_f32) wr->scale_f32[g] = r.s;
+        if (wr->err) wr->err[g] = r.e_best;
         if (wr->iters_out) wr->iters_out[g] = (uint8_t)r.accepted;
     }
     return NULL;
@@ -274,11 +275,12 @@ static void *run_range(void *arg) {
 
 /* Quantize n_groups contiguous groups of G fp16 weights (row-major [out,in]
    with in % G == 0 is exactly this flat layout).  codes: one byte per weight.
-   scale/zero: fp16 bits per group.  zero_f32/scale_f32/iters_out nullable. */
+   scale/zero: fp16 bits per group.  zero_f32/scale_f32/err/iters_out nullable;
+   err is the accepted minimum of the error sum (+inf when iters = 0). */
 int hqq_oracle_quantize(const uint16_t *W, int64_t n_groups, int G, int nbits,
                         float p, float beta, float kappa, int iters, int nthreads,
                         uint8_t *codes, uint16_t *scale, uint16_t *zero,
-                        float *zero_f32, float *scale_f32, uint8_t *iters_out) {
+                        float *zero_f32, float *scale_f32, float *err, uint8_t *iters_out) {
     const int st = check_cfg(nbits, G, p, beta, kappa, iters);
     if (st) return st;
     if (n_groups <= 0) return 0;
@@ -299,6 +301,7 @@ int hqq_oracle_quantize(const uint16_t *W, int64_t n_groups, int G, int nbits,
         wr[k].zero = zero;
         wr[k].zero_f32 = zero_f32;
         wr[k].scale_f32 = scale_f32;
+        wr[k].err = err;
         wr[k].iters_out = iters_out;
     }
     if (nthreads == 1) {

@@ -8,6 +8,10 @@ Tolerances (stated once, used by every parity test):
   * codes:  identical on >= 99.99 % of the weights (only rounding-boundary flips
             are tolerated; 100 % is expected);
   * l_p:    per-tensor sum |W - W_hat|^0.7 (fp64) within 1e-4 relative;
+  * the solver's per-group binary32 error sums and accepted-iteration counts:
+            identical (the arithmetic is the same op for op on both sides, so a
+            one-ulp difference in an error sum is a defect even when it flips no
+            early-stop decision);
   * dequantize: fp16 bits identical (both sides compute fp16((c - z) * s) in
             binary32 from the same stored values).
 """
@@ -35,6 +39,7 @@ def to_np(q):
                 scale=q.scale.cpu().numpy().reshape(-1),
                 zero=q.zero.cpu().numpy().reshape(-1),
                 zero_f32=q.zero_f32.cpu().numpy().reshape(-1),
+                err=q.err.cpu().numpy().reshape(-1),
                 iters=q.iters.cpu().numpy().reshape(-1))
 
 
@@ -56,6 +61,11 @@ def compare_full(W_np, gq, ref, nbits, group, p=0.7, label=""):
     if match == 1.0:
         assert np.array_equal(gq["packed"], ref["packed"]), f"{label}: packed bytes differ"
     stats["iters_equal"] = float(np.mean(gq["iters"] == ref["iters"])) if gq["iters"].size else 1.0
+    # the solver's own binary32 error sums: identical arithmetic on both sides
+    stats["err_equal"] = float(np.mean(gq["err"].view(np.uint32) == ref["err"].view(np.uint32))) \
+        if gq["err"].size else 1.0
+    assert stats["iters_equal"] == 1.0, f"{label}: accepted iterations differ"
+    assert stats["err_equal"] == 1.0, f"{label}: solver error sums differ"
     Wh_g = oracle.dequantize(codes_gpu, gq["scale"], gq["zero"], group)
     Wh_r = oracle.dequantize(ref["codes"], ref["scale"], ref["zero"], group)
     # fp16 storage can overflow on groups spanning the whole fp16 range; such

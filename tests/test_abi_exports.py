@@ -89,7 +89,9 @@ def test_host_validation_without_gpu(lib):
     assert L.hqq_quantize(P(256), 64, 256, 4, 64, 0.7, 1.0, 1.01, 20, P(258), P(256), P(256),
                           None) == 5
     assert L.hqq_quantize_ex(P(256), 64, 256, 4, 64, 0.7, 1.0, 1.01, 20, P(256), P(256),
-                             P(256), P(258), None, None) == 5
+                             P(256), P(258), None, None, None) == 5
+    assert L.hqq_quantize_ex(P(256), 64, 256, 4, 64, 0.7, 1.0, 1.01, 20, P(256), P(256),
+                             P(256), None, P(262), None, None) == 5
     # empty matrices are valid no-ops (nothing launched, so no GPU needed)
     assert L.hqq_quantize(None, 0, 256, 4, 64, 0.7, 1.0, 1.01, 20, None, None, None, None) == 0
     assert L.hqq_dequantize(None, None, None, 16, 0, 3, 64, None, None) == 0

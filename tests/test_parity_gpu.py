@@ -90,6 +90,7 @@ def _adversarial(G):
     r = rng.standard_normal(G); rows.append(r)                   # unit scale (shrink on)
     r = rng.standard_normal(G) * 10; rows.append(r)              # large scale
     rows.append(np.full(G, 6e-8))                                # constant subnormal
+    r = np.zeros(G); r[1::2] = -0.0; r[::3] = 0.25; rows.append(r)  # signed zeros
     return np.array(rows, np.float64).astype(np.float16)
 
 
@@ -168,6 +169,8 @@ def test_full_size_sampled(hqq, label, shape, nbits, group, seed, stream):
     sc = q.scale.view(-1)[torch.from_numpy(g_idx).cuda()].cpu().numpy()
     zf = q.zero_f32.view(-1)[torch.from_numpy(g_idx).cuda()].cpu().numpy()
     it = q.iters.view(-1)[torch.from_numpy(g_idx).cuda()].cpu().numpy()
+    er = q.err.view(-1)[torch.from_numpy(g_idx).cuda()].cpu().numpy()
+    assert np.array_equal(er.view(np.uint32), ref["err"].view(np.uint32))
     assert np.array_equal(sc.view(np.uint16), ref["scale"].view(np.uint16))
     assert np.max(np.abs(zf.astype(np.float64) - ref["zero_f32"])) <= ZERO_TOL
     assert np.mean(codes.reshape(-1) == ref["codes"]) >= CODE_MATCH

@@ -33,7 +33,8 @@ _lib.hqq_status_string.argtypes = [_I]
 _lib.hqq_status_string.restype = ctypes.c_char_p
 _lib.hqq_quantize.argtypes = [_P, _I64, _I64, _I, _I, _F, _F, _F, _I, _P, _P, _P, _P]
 _lib.hqq_quantize.restype = _I
-_lib.hqq_quantize_ex.argtypes = [_P, _I64, _I64, _I, _I, _F, _F, _F, _I, _P, _P, _P, _P, _P, _P]
+_lib.hqq_quantize_ex.argtypes = [_P, _I64, _I64, _I, _I, _F, _F, _F, _I, _P, _P, _P, _P, _P, _P,
+                                 _P]
 _lib.hqq_quantize_ex.restype = _I
 _lib.hqq_dequantize.argtypes = [_P, _P, _P, _I64, _I64, _I, _I, _P, _P]
 _lib.hqq_dequantize.restype = _I
@@ -84,6 +85,7 @@ class QuantizedMatrix:
     group: int
     zero_f32: "torch.Tensor | None" = None
     iters: "torch.Tensor | None" = None
+    err: "torch.Tensor | None" = None
 
 
 def _outputs(W, nbits, group, packed, scale, zero):
@@ -125,13 +127,14 @@ def hqq_quantize(W, nbits: int = 4, group: int = 64, p: float = DEFAULT_P,
 def hqq_quantize_ex(W, nbits: int = 4, group: int = 64, p: float = DEFAULT_P,
                     beta: float = DEFAULT_BETA, kappa: float = DEFAULT_KAPPA,
                     iters: int = DEFAULT_ITERS, packed=None, scale=None, zero=None,
-                    zero_f32=None, iters_out=None, stream=None) -> QuantizedMatrix:
-    """hqq_quantize plus the fp32 zero and accepted-iteration count per group."""
+                    zero_f32=None, iters_out=None, err_out=None, stream=None) -> QuantizedMatrix:
+    """hqq_quantize plus the fp32 zero, the solver's l_p error sum and the
+    accepted-iteration count of every group."""
     import torch
     if W.dtype != torch.float16 or W.dim() != 2:
         raise ValueError("W must be a 2-D float16 tensor")
     for t, n in ((W, "W"), (packed, "packed"), (scale, "scale"), (zero, "zero"),
-                 (zero_f32, "zero_f32"), (iters_out, "iters_out")):
+                 (zero_f32, "zero_f32"), (iters_out, "iters_out"), (err_out, "err_out")):
         _check_tensor(t, n)
     packed, scale, zero = _outputs(W, nbits, group, packed, scale, zero)
     rows, cols = W.shape
@@ -140,10 +143,13 @@ def hqq_quantize_ex(W, nbits: int = 4, group: int = 64, p: float = DEFAULT_P,
         zero_f32 = torch.empty(meta, dtype=torch.float32, device=W.device)
     if iters_out is None:
         iters_out = torch.empty(meta, dtype=torch.uint8, device=W.device)
+    if err_out is None:
+        err_out = torch.empty(meta, dtype=torch.float32, device=W.device)
     _check(_lib.hqq_quantize_ex(_ptr(W), rows, cols, nbits, group, p, beta, kappa, iters,
                                 _ptr(packed), _ptr(scale), _ptr(zero), _ptr(zero_f32),
-                                _ptr(iters_out), _stream(stream)))
-    return QuantizedMatrix(packed, scale, zero, rows, cols, nbits, group, zero_f32, iters_out)
+                                _ptr(err_out), _ptr(iters_out), _stream(stream)))
+    return QuantizedMatrix(packed, scale, zero, rows, cols, nbits, group, zero_f32, iters_out,
+                           err_out)
 
 
 def hqq_dequantize(q: QuantizedMatrix, out=None, stream=None):

@@ -99,8 +99,8 @@ extern "C" const char* hqq_status_string(int status) {
 
 extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nbits, int group,
                                float p, float beta, float kappa, int iters, void* packed,
-                               void* scale, void* zero, float* zero_f32, uint8_t* iters_out,
-                               void* stream) {
+                               void* scale, void* zero, float* zero_f32, float* err_out,
+                               uint8_t* iters_out, void* stream) {
     int st = validate_common(rows, cols, nbits, group);
     if (st != HQQ_OK) return st;
     if (!(p > 0.0f && p <= 1.0f)) return HQQ_ERR_PARAM;
@@ -111,7 +111,7 @@ extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nb
     if (n == 0) return HQQ_OK;
     if (!W || !packed || !scale || !zero) return HQQ_ERR_NULL;
     if (!aligned(W, 16) || !aligned(packed, 4) || !aligned(scale, 2) || !aligned(zero, 2) ||
-        (zero_f32 && !aligned(zero_f32, 4)))
+        (zero_f32 && !aligned(zero_f32, 4)) || (err_out && !aligned(err_out, 4)))
         return HQQ_ERR_ALIGN;
 
     QuantParams prm;
@@ -121,6 +121,7 @@ extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nb
     prm.scale = static_cast<__half*>(scale);
     prm.zero = static_cast<__half*>(zero);
     prm.zero_f32 = zero_f32;
+    prm.err_out = err_out;
     prm.iters_out = iters_out;
     prm.n_groups = n / group;
     prm.n_elems = n;
@@ -157,7 +158,7 @@ extern "C" int hqq_quantize(const void* W, int64_t rows, int64_t cols, int nbits
                             float p, float beta, float kappa, int iters, void* packed,
                             void* scale, void* zero, void* stream) {
     return hqq_quantize_ex(W, rows, cols, nbits, group, p, beta, kappa, iters, packed, scale,
-                           zero, nullptr, nullptr, stream);
+                           zero, nullptr, nullptr, nullptr, stream);
 }
 
 extern "C" int hqq_dequantize(const void* packed, const void* scale, const void* zero,

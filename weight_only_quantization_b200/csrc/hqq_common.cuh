@@ -2,9 +2,10 @@
 //
 // Arithmetic contract of the solver (binary32, round-to-nearest-even, every
 // rounding explicit): products and sums that the method writes separately are
-// issued as __fmul_rn / __fadd_rn / __fsub_rn (never contracted), and the three
-// places that are defined as one fused multiply-add use __fmaf_rn.  The library
-// is also compiled with -fmad=false.
+// issued as __fmul_rn / __fadd_rn or their packed f32x2 forms (__fmul2_rn,
+// __fadd2_rn: two independent binary32 operations, each rounded to nearest),
+// never contracted, and the places defined as one fused multiply-add use
+// __fmaf_rn / __ffma2_rn.  The library is also compiled with -fmad=false.
 #pragma once
 
 #include <cstdint>
@@ -16,7 +17,7 @@ namespace hqq {
 // |x|^p by table-driven evaluation (after P. T. P. Tang, "Table-driven
 // implementation of the exponential function", ACM TOMS 15(2), 1989):
 //   x = 2^k m, m in [1,2); c_j = 1 + (2j+1)/64 is the centre of the 1/32-wide
-//   cell of m picked by its top five mantissa bits; r = (m - c_j) * (1/c_j),
+//   cell of m picked by its top five mantissa bits; r = fma(m, fl(1/c_j), -1),
 //   |r| <= 1/64, and (1+r)^p = 1 + r(a1 + r(a2 + r a3)) (binomial series).
 //   |x|^p = (2^(p k) * c_j^p) * (1+r)^p.
 // two_pk[e] for the biased exponent e (e = 0: +0 and subnormals -> 0, +inf or 1
@@ -28,7 +29,6 @@ struct PowTable {
     float a1, a2, a3;
 };
 
-constexpr int kTabFloats = 256 + 32 + 32;   // the part copied to shared memory
 constexpr int kMaxIters = 255;
 
 struct QuantParams {
@@ -37,6 +37,7 @@ struct QuantParams {
     __half* scale;
     __half* zero;
     float* zero_f32;       // nullable
+    float* err_out;        // nullable
     uint8_t* iters_out;    // nullable
     int64_t n_groups;
     int64_t n_elems;
@@ -57,18 +58,46 @@ struct DequantParams {
     int group;
 };
 
-// Table-driven |x|^p for x >= +0 (sign bit clear).  `tab` points at the
-// kTabFloats-long shared-memory copy of two_pk, cj_p, inv_cj.
-__device__ __forceinline__ float powp(const float* __restrict__ tab, float a1, float a2,
-                                      float a3, float x) {
+// Shared-memory image of one PowTable (separate arrays, so that the two values
+// of an f32x2 pair are loaded straight into the two halves of a register pair).
+struct PowSmem {
+    float te[256];   // 2^(p k) by biased exponent
+    float tc[32];    // c_j^p
+    float ic[32];    // fl(1 / c_j)
+};
+
+__device__ __forceinline__ void load_pow_smem(PowSmem& dst, const PowTable& t) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) dst.te[i] = t.two_pk[i];
+    for (int i = threadIdx.x; i < 32; i += blockDim.x) {
+        dst.tc[i] = t.cj_p[i];
+        dst.ic[i] = t.inv_cj[i];
+    }
+}
+
+// |x|^p of two values (any sign) with the table in shared memory.
+__device__ __forceinline__ float2 powp2(const PowSmem& T, float2 a1, float2 a2, float2 a3,
+                                        float2 x) {
+    const uint32_t bx = __float_as_uint(x.x), by = __float_as_uint(x.y);
+    const uint32_t ex = (bx >> 23) & 0xFFu, ey = (by >> 23) & 0xFFu;   // exponent of |x|
+    const uint32_t jx = (bx >> 18) & 31u, jy = (by >> 18) & 31u;       // mantissa cell
+    const float2 m = make_float2(__uint_as_float((bx & 0x007FFFFFu) | 0x3F800000u),
+                                 __uint_as_float((by & 0x007FFFFFu) | 0x3F800000u));
+    const float2 r = __ffma2_rn(m, make_float2(T.ic[jx], T.ic[jy]), make_float2(-1.0f, -1.0f));
+    float2 poly = __ffma2_rn(r, a3, a2);
+    poly = __ffma2_rn(poly, r, a1);
+    poly = __ffma2_rn(poly, r, make_float2(1.0f, 1.0f));
+    const float2 tt = __fmul2_rn(make_float2(T.te[ex], T.te[ey]), make_float2(T.tc[jx], T.tc[jy]));
+    return __fmul2_rn(tt, poly);
+}
+
+// Scalar form (same operations) for the shrink's |x|^(p-1), x >= +0.
+__device__ __forceinline__ float powp1(const PowSmem& T, float a1, float a2, float a3, float x) {
     const uint32_t b = __float_as_uint(x);
-    const uint32_t e = b >> 23;
     const uint32_t j = (b >> 18) & 31u;
     const float m = __uint_as_float((b & 0x007FFFFFu) | 0x3F800000u);
-    const float c = __uint_as_float((b & 0x007C0000u) | 0x3F820000u);
-    const float r = __fmul_rn(__fsub_rn(m, c), tab[288 + j]);   // m - c is exact
+    const float r = __fmaf_rn(m, T.ic[j], -1.0f);
     const float poly = __fmaf_rn(__fmaf_rn(__fmaf_rn(r, a3, a2), r, a1), r, 1.0f);
-    return __fmul_rn(__fmul_rn(tab[e], tab[256 + j]), poly);
+    return __fmul_rn(__fmul_rn(T.te[(b >> 23) & 0xFFu], T.tc[j]), poly);
 }
 
 // Round-half-even of v in [0, 2^22) by the 1.5*2^23 shift: the sum's last

@@ -49,24 +49,34 @@ dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
     const int64_t per_block = (int64_t)kDqThreads * kDqUnroll;
     for (int64_t base = (int64_t)blockIdx.x * per_block; base < prm.n_units;
          base += (int64_t)gridDim.x * per_block) {
+        // all loads of the kDqUnroll units first, so they are in flight together
+        uint32_t c[kDqUnroll][8];
+        float sf[kDqUnroll], zf[kDqUnroll];
+        bool ok[kDqUnroll];
 #pragma unroll
         for (int r = 0; r < kDqUnroll; ++r) {
             const int64_t u = base + r * kDqThreads + threadIdx.x;
-            if (u >= prm.n_units) break;
-            const int64_t g = (u * 8) >> log2_group;
-            const float sf = __half2float(prm.scale[g]);
-            const float zf = __half2float(prm.zero[g]);
-            uint32_t c[8];
-            unit_codes<NBITS>(prm.packed, u, c);
+            ok[r] = u < prm.n_units;
+            const int64_t uu = ok[r] ? u : 0;
+            const int64_t g = (uu * 8) >> log2_group;
+            sf[r] = __half2float(__ldg(prm.scale + g));
+            zf[r] = __half2float(__ldg(prm.zero + g));
+            unit_codes<NBITS>(prm.packed, uu, c[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < kDqUnroll; ++r) {
             uint32_t o[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const float a = __fmul_rn(__fsub_rn(code_to_float(c[2 * k]), zf), sf);
-                const float b = __fmul_rn(__fsub_rn(code_to_float(c[2 * k + 1]), zf), sf);
+                const float a = __fmul_rn(__fsub_rn(code_to_float(c[r][2 * k]), zf[r]), sf[r]);
+                const float b = __fmul_rn(__fsub_rn(code_to_float(c[r][2 * k + 1]), zf[r]), sf[r]);
                 const __half2 h = __floats2half2_rn(a, b);
                 o[k] = *reinterpret_cast<const uint32_t*>(&h);
             }
-            reinterpret_cast<uint4*>(prm.out)[u] = make_uint4(o[0], o[1], o[2], o[3]);
+            if (ok[r]) {
+                const int64_t u = base + r * kDqThreads + threadIdx.x;
+                reinterpret_cast<uint4*>(prm.out)[u] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
         }
     }
 }

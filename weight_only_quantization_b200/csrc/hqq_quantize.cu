@@ -4,228 +4,476 @@
 // (Q, Q^-1, l_p error, sp1 shrink, sp2 mean, beta <- kappa beta, 1/s held) and
 // section 4.1 (solver parameters, early exit when the error stops improving).
 //
-// Layout: a group of G weights is held by a sub-warp of K = G/8 lanes, each
-// lane owning 8 consecutive weights loaded with one 128-bit load, so a warp
-// holds 256 consecutive weights (32/K groups) and a CTA of 10 warps a tile of
-// 2560 weights -- five whole groups of any size at the 3-bit layout's 10 codes
-// per word, so every packed word of a tile is written by exactly one thread.
-// All solver state lives in registers; group sums are the pairwise sum over
-// contiguous halves (8 in-lane, then xor-shuffles 1, 2, .. K/2).  Every
-// sub-warp stops on its own; the warp iterates while any of its groups runs.
+// Work decomposition (persistent warps):
+//  * A group of G weights is held by a sub-warp of K = G/(8 NB) lanes, each lane
+//    owning NB blocks of 8 consecutive weights.  Within a block the weights sit
+//    in f32x2 register pairs (x_k, x_k+4), k = 0..3, for the packed element-wise
+//    arithmetic; the pairwise sum over contiguous halves then reads the halves
+//    with scalar adds, and lane sums are combined by xor-shuffles 1, 2, .., K/2
+//    (same pairwise order).
+//  * Each warp owns chunks of 2560 consecutive weights (five groups of any size
+//    fill whole 3-bit words), staged once into the warp's shared memory.
+//  * Phase A: every group of the chunk is initialised and runs its first two
+//    error evaluations in lock-step -- every group needs at least two, so no
+//    lane idles.  Groups that stop are finalised; the others are queued with
+//    their state in shared memory.
+//  * Phase B: each sub-warp pulls queued groups, iterates until its group stops,
+//    finalises it and pulls the next, so the early-stop divergence costs almost
+//    nothing.  No block-wide barrier is ever taken after start-up.
+//  * Two exact shortcuts, both tested per group and per step: when
+//    fma(min, 1/s, z) >= -1/2 and fma(max, 1/s, z) < L + 1/2 no code can leave
+//    [0, L] (fma is monotone in the weight), so the clamp is skipped; when a
+//    bound on |W - Q^-1(Q(W))| lies below the shrink threshold, W_e is exactly
+//    zero, so sp1 reduces to W - W_e = W.
 #include "hqq_common.cuh"
 
 namespace hqq {
 
-constexpr int kQuantThreads = 320;
-constexpr int kTileElems = kQuantThreads * 8;   // 2560
+constexpr int kQWarps = 4;                 // warps per CTA
+constexpr int kChunk = 2560;               // weights per warp chunk
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
+template <int NBITS, int G, int NB>
+struct QCfg {
+    static constexpr int EPL = 8 * NB;           // weights per lane
+    static constexpr int K = G / EPL;            // lanes per group
+    static constexpr int GPW = 32 / K;           // groups per warp round
+    static constexpr int ROUND = 32 * EPL;       // weights per warp round
+    static constexpr int ROUNDS = kChunk / ROUND;
+    static constexpr int CG = kChunk / G;        // groups per chunk
+    static constexpr int L = (1 << NBITS) - 1;
+    static constexpr int W_BYTES = kChunk * 2;
+    static constexpr int ST_BYTES = CG * 16;     // (z, zb, eb, s) of queued groups
+    static constexpr int ST2_BYTES = CG * 16;    // (1/s, min, max, -)
+    static constexpr int Q_BYTES = (CG + 15) / 16 * 16;
+    static constexpr int CODE_BYTES = NBITS == 3 ? kChunk : 0;
+    static constexpr int WARP_BYTES = W_BYTES + ST_BYTES + ST2_BYTES + Q_BYTES + CODE_BYTES;
+    static constexpr int SMEM = kQWarps * WARP_BYTES;
+    static_assert(K >= 1 && K <= 32 && kChunk % ROUND == 0, "bad layout");
+};
+
+struct QuantSmem {
+    PowSmem tp;                 // |x|^p
+    PowSmem tq;                 // |x|^(p-1)
+    float beta[kMaxIters + 1];  // beta_t = beta * kappa^t by repeated binary32 products
+    float thr[kMaxIters + 1];   // shrink thresholds
+};
+
 template <int K>
-__device__ __forceinline__ float group_sum(float v) {
+__device__ __forceinline__ float2 group_sum2(float2 v) {
 #pragma unroll
-    for (int o = 1; o < K; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, o));
+    for (int o = 1; o < K; o <<= 1) {
+        const float ux = __shfl_xor_sync(kFull, v.x, o), uy = __shfl_xor_sync(kFull, v.y, o);
+        v = make_float2(__fadd_rn(v.x, ux), __fadd_rn(v.y, uy));
+    }
     return v;
 }
 
 template <int K>
-__device__ __forceinline__ float group_min(float v) {
+__device__ __forceinline__ void group_minmax(float& mn, float& mx) {
 #pragma unroll
-    for (int o = 1; o < K; o <<= 1) v = fminf(v, __shfl_xor_sync(kFull, v, o));
-    return v;
+    for (int o = 1; o < K; o <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+    }
 }
 
-template <int K>
-__device__ __forceinline__ float group_max(float v) {
+// NB blocks of 8 fp16 weights -> pairs (x_k, x_k+4) of each block.
+template <int NB>
+__device__ __forceinline__ void load_lane(const __half* src, float2 (&w)[NB][4]) {
 #pragma unroll
-    for (int o = 1; o < K; o <<= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
-    return v;
+    for (int b = 0; b < NB; ++b) {
+        const uint4 raw = reinterpret_cast<const uint4*>(src)[b];
+        const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
+        const __half2 h23 = *reinterpret_cast<const __half2*>(&raw.y);
+        const __half2 h45 = *reinterpret_cast<const __half2*>(&raw.z);
+        const __half2 h67 = *reinterpret_cast<const __half2*>(&raw.w);
+        w[b][0] = make_float2(__low2float(h01), __low2float(h45));
+        w[b][1] = make_float2(__high2float(h01), __high2float(h45));
+        w[b][2] = make_float2(__low2float(h23), __low2float(h67));
+        w[b][3] = make_float2(__high2float(h23), __high2float(h67));
+    }
 }
 
-__device__ __forceinline__ float sum8(const float (&x)[8]) {
-    return __fadd_rn(__fadd_rn(__fadd_rn(x[0], x[1]), __fadd_rn(x[2], x[3])),
-                     __fadd_rn(__fadd_rn(x[4], x[5]), __fadd_rn(x[6], x[7])));
-}
+// Per-group constants of one evaluation, as f32x2 pairs.
+struct EvalConst {
+    float2 z, nz, ns, inv, ninv;
+    float s, invs;
+};
 
-// clamp(round(v), 0, L) with round half to even; returns the code as a float
-// and its integer value.
-template <int L>
-__device__ __forceinline__ float code_of(float v, uint32_t& ci) {
-    v = fminf(fmaxf(v, 0.0f), (float)L);
-    const float t = __fadd_rn(v, kRoundShift);
-    ci = __float_as_uint(t) & 0xFFu;
-    return __fsub_rn(t, kRoundShift);
-}
-
-__device__ __forceinline__ void load_table(float* dst, const PowTable& t) {
-    for (int i = threadIdx.x; i < kTabFloats; i += blockDim.x)
-        dst[i] = i < 256 ? t.two_pk[i] : (i < 288 ? t.cj_p[i - 256] : t.inv_cj[i - 288]);
-}
-
-template <int NBITS, int G>
-__global__ void __launch_bounds__(kQuantThreads, 2)
-quantize_kernel(const __grid_constant__ QuantParams prm) {
-    constexpr int K = G / 8;              // lanes per group
-    constexpr int GPW = 32 / K;           // groups per warp
-    constexpr int GPC = GPW * (kQuantThreads / 32);
-    constexpr int L = (1 << NBITS) - 1;
-    constexpr float kInvG = 1.0f / (float)G;
-
-    __shared__ float s_tp[kTabFloats];
-    __shared__ float s_tq[kTabFloats];
-    __shared__ float s_thr[kMaxIters];
-    __shared__ __align__(16) uint8_t s_codes[NBITS == 3 ? kTileElems : 16];
-
-    load_table(s_tp, prm.tp);
-    load_table(s_tq, prm.tq);
-    for (int i = threadIdx.x; i < prm.iters; i += blockDim.x) s_thr[i] = prm.shrink_thr[i];
-    __syncthreads();
-
-    const float pa1 = prm.tp.a1, pa2 = prm.tp.a2, pa3 = prm.tp.a3;
-    const float qa1 = prm.tq.a1, qa2 = prm.tq.a2, qa3 = prm.tq.a3;
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int kl = lane % K;
-    const int64_t n_tiles = (prm.n_groups + GPC - 1) / GPC;
-
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int64_t g = tile * GPC + warp * GPW + lane / K;
-        const bool valid = g < prm.n_groups;
-
-        // ---- load 8 fp16 weights (one 128-bit load) ------------------------------
-        float w[8];
-        {
-            uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-            if (valid) raw = __ldg(reinterpret_cast<const uint4*>(prm.W + g * G + kl * 8));
-            const uint32_t r4[4] = {raw.x, raw.y, raw.z, raw.w};
+// One error evaluation of the lane's weights at zero-point z.  Returns the
+// lane's pairwise sums of (|r|^p, sp2 term) where r = W - s(Wq - z) and the sp2
+// term is Wq - (W - W_e)/s.  CLAMP: codes may leave [0, L].  SHRINK: W_e is
+// evaluated exactly; otherwise W_e is known to be zero.
+template <int L, int NB, bool CLAMP, bool SHRINK>
+__device__ __forceinline__ float2 eval_lane(const QuantSmem& S, const float2 (&w)[NB][4],
+                                            const EvalConst& c, float2 pa1, float2 pa2,
+                                            float2 pa3, float qa1, float qa2, float qa3,
+                                            float beta) {
+    const float2 sh = make_float2(kRoundShift, kRoundShift);
+    const float2 nsh = make_float2(-kRoundShift, -kRoundShift);
+    float pe = 0.0f, pt = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r4[k]));
-                w[2 * k] = f.x;
-                w[2 * k + 1] = f.y;
+    for (int b = 0; b < NB; ++b) {
+        float2 P[4], T[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float2 v = __ffma2_rn(w[b][k], c.inv, c.z);                // W/s + z
+            if (CLAMP) {
+                v.x = fminf(fmaxf(v.x, 0.0f), (float)L);
+                v.y = fminf(fmaxf(v.y, 0.0f), (float)L);
             }
-        }
-
-        // ---- min-max initialisation ---------------------------------------------
-        float mn = w[0], mx = w[0];
+            const float2 q = __fadd2_rn(__fadd2_rn(v, sh), nsh);      // round half even
+            const float2 qz = __fadd2_rn(q, c.nz);                     // Wq - z
+            const float2 d = __ffma2_rn(qz, c.ns, w[b][k]);            // W - s(Wq - z)
+            P[k] = powp2(S.tp, pa1, pa2, pa3, d);
+            if (SHRINK) {
+                float we[2];
+                const float dd[2] = {d.x, d.y};
 #pragma unroll
-        for (int i = 1; i < 8; ++i) {
-            mn = fminf(mn, w[i]);
-            mx = fmaxf(mx, w[i]);
-        }
-        mn = group_min<K>(mn);
-        mx = group_max<K>(mx);
-        const float rng = __fsub_rn(mx, mn);
-        float s = 1.0f, inv = 1.0f;
-        if (rng != 0.0f) {
-            s = __fdiv_rn(rng, (float)L);
-            inv = __fdiv_rn(1.0f, s);
-        }
-        float z = -__fmul_rn(mn, inv);
-        float zb = z, eb = __int_as_float(0x7F800000);   // +inf
-        float bt = prm.beta;
-        int accepted = 0;
-        bool active = valid;
-
-        // ---- half-quadratic iterations -------------------------------------------
-        for (int t = 0; t < prm.iters; ++t) {
-            if (!__any_sync(kFull, active)) break;
-            float q[8], d[8], pw[8], tm[8];
-            float amax = 0.0f;
-            uint32_t ci;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                q[i] = code_of<L>(__fmaf_rn(w[i], inv, z), ci);
-                d[i] = __fmaf_rn(__fsub_rn(z, q[i]), s, w[i]);
-                const float a = fabsf(d[i]);
-                amax = fmaxf(amax, a);
-                pw[i] = powp(s_tp, pa1, pa2, pa3, a);
-                tm[i] = __fmaf_rn(-w[i], inv, q[i]);     // sp2 term when W_e == 0
-            }
-            const float e = group_sum<K>(sum8(pw));
-            const bool acc = active && (e < eb);
-            if (acc) {
-                eb = e;
-                zb = z;
-                ++accepted;
-            }
-            active = acc;
-            // sp1: W_e is exactly zero unless some |r| exceeds the threshold
-            if (__any_sync(kFull, active && amax > s_thr[t])) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float a = fabsf(d[i]);
-                    const float y = __fsub_rn(a, __fdiv_rn(powp(s_tq, qa1, qa2, qa3, a), bt));
-                    const float we = copysignf(fmaxf(y, 0.0f), d[i]);
-                    tm[i] = __fmaf_rn(-__fsub_rn(w[i], we), inv, q[i]);
+                for (int e = 0; e < 2; ++e) {
+                    const float a = fabsf(dd[e]);
+                    const float y = __fsub_rn(a, __fdiv_rn(powp1(S.tq, qa1, qa2, qa3, a), beta));
+                    we[e] = copysignf(fmaxf(y, 0.0f), dd[e]);
                 }
+                T[k].x = __fmaf_rn(-__fsub_rn(w[b][k].x, we[0]), c.invs, q.x);
+                T[k].y = __fmaf_rn(-__fsub_rn(w[b][k].y, we[1]), c.invs, q.y);
+            } else {
+                T[k] = __ffma2_rn(w[b][k], c.ninv, q);                 // Wq - W/s
             }
-            const float zs = group_sum<K>(sum8(tm));
-            if (active) z = __fmul_rn(zs, kInvG);
-            bt = __fmul_rn(bt, prm.kappa);
         }
+        // ((x0+x1)+(x2+x3)) + ((x4+x5)+(x6+x7)) with pairs (x_k, x_k+4).  The
+        // reduction reads the pair halves one by one with scalar adds: a packed
+        // f32x2 add fed by the packed power results was found to combine the
+        // halves in the wrong order on this toolchain (the sums came out as if
+        // the pairs held adjacent weights), so no packed add is used here.
+        const float bp = __fadd_rn(__fadd_rn(__fadd_rn(P[0].x, P[1].x), __fadd_rn(P[2].x, P[3].x)),
+                                   __fadd_rn(__fadd_rn(P[0].y, P[1].y), __fadd_rn(P[2].y, P[3].y)));
+        const float bt = __fadd_rn(__fadd_rn(__fadd_rn(T[0].x, T[1].x), __fadd_rn(T[2].x, T[3].x)),
+                                   __fadd_rn(__fadd_rn(T[0].y, T[1].y), __fadd_rn(T[2].y, T[3].y)));
+        if (b == 0) {
+            pe = bp;
+            pt = bt;
+        } else {
+            pe = __fadd_rn(pe, bp);
+            pt = __fadd_rn(pt, bt);
+        }
+    }
+    return make_float2(pe, pt);
+}
 
-        // ---- final codes, packing and stores ---------------------------------------
+struct GroupState {
+    float z, zb, eb, s, inv, mn, mx;
+    int t;    // evaluations done
+    int na;   // evaluations accepted
+};
+
+// One solver iteration (error evaluation, early-stop test, sp1 + sp2) for the
+// sub-warp's group; `live` lanes only change state.  Returns true when the
+// group has finished (stopped, or used its iterations).
+template <int NBITS, int G, int NB>
+__device__ __forceinline__ bool solver_step(const QuantSmem& S, const QuantParams& prm,
+                                            const float2 (&w)[NB][4], GroupState& g, bool live,
+                                            float2 pa1, float2 pa2, float2 pa3,
+                                            float qa1, float qa2, float qa3) {
+    using C = QCfg<NBITS, G, NB>;
+    constexpr float L = (float)C::L;
+    const int t = live ? g.t : 0;
+    const float beta = S.beta[t];
+    const float vmin = __fmaf_rn(g.mn, g.inv, g.z);
+    const float vmax = __fmaf_rn(g.mx, g.inv, g.z);
+    const bool inside = vmin >= -0.5f && vmax < L + 0.5f;
+    const float reach = fmaxf(0.5f, fmaxf(-vmin, vmax - L)) + 1e-3f * (1.0f + fabsf(g.z));
+    const bool shrink = 2.0f * g.s * reach > S.thr[t];
+    EvalConst c;
+    c.z = make_float2(g.z, g.z);
+    c.nz = make_float2(-g.z, -g.z);
+    c.ns = make_float2(-g.s, -g.s);
+    c.inv = make_float2(g.inv, g.inv);
+    c.ninv = make_float2(-g.inv, -g.inv);
+    c.s = g.s;
+    c.invs = g.inv;
+    float2 r;
+    if (__any_sync(kFull, live && shrink))
+        r = eval_lane<C::L, NB, true, true>(S, w, c, pa1, pa2, pa3, qa1, qa2, qa3, beta);
+    else if (__all_sync(kFull, !live || inside))
+        r = eval_lane<C::L, NB, false, false>(S, w, c, pa1, pa2, pa3, qa1, qa2, qa3, beta);
+    else
+        r = eval_lane<C::L, NB, true, false>(S, w, c, pa1, pa2, pa3, qa1, qa2, qa3, beta);
+    r = group_sum2<C::K>(r);                       // (error, sp2 sum) of the whole group
+    const bool acc = live && r.x < g.eb;
+    if (acc) {
+        g.eb = r.x;
+        g.zb = g.z;
+        g.z = __fmul_rn(r.y, 1.0f / (float)G);
+        ++g.na;
+    }
+    if (live) ++g.t;
+    return live && (!acc || g.t == prm.iters);
+}
+
+// Final codes of the sub-warp's group, packed, plus its scale and zero.
+template <int NBITS, int G, int NB>
+__device__ __forceinline__ void finalize(const QuantParams& prm, const float2 (&w)[NB][4],
+                                         const GroupState& g, int64_t chunk, int gl, int kl,
+                                         uint8_t* s_codes) {
+    using C = QCfg<NBITS, G, NB>;
+    constexpr float L = (float)C::L;
+    const float2 inv2 = make_float2(g.inv, g.inv), zb2 = make_float2(g.zb, g.zb);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
         uint32_t c[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) code_of<L>(__fmaf_rn(w[i], inv, zb), c[i]);
-
-        const int64_t chunk = tile * (kTileElems / 8) + threadIdx.x;   // 8-weight chunk id
+        for (int k = 0; k < 4; ++k) {
+            float2 v = __ffma2_rn(w[b][k], inv2, zb2);
+            v.x = fminf(fmaxf(v.x, 0.0f), L);
+            v.y = fminf(fmaxf(v.y, 0.0f), L);
+            const float2 t = __fadd2_rn(v, make_float2(kRoundShift, kRoundShift));
+            c[k] = __float_as_uint(t.x) & 0xFFu;
+            c[k + 4] = __float_as_uint(t.y) & 0xFFu;
+        }
+        const int64_t unit = chunk * (kChunk / 8) + gl * (G / 8) + kl * NB + b;   // 8-weight unit
         if constexpr (NBITS == 4) {
             uint32_t word = 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) word |= c[i] << (4 * i);
-            if (valid) reinterpret_cast<uint32_t*>(prm.packed)[chunk] = word;
+            reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
         } else if constexpr (NBITS == 2) {
             uint32_t h = 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) h |= c[i] << (2 * i);
-            if (valid) reinterpret_cast<uint16_t*>(prm.packed)[chunk] = (uint16_t)h;
+            reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)h;
         } else {
-            uint2 b;
-            b.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-            b.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-            reinterpret_cast<uint2*>(s_codes)[threadIdx.x] = b;   // zeros when !valid
-            __syncthreads();
-            if (threadIdx.x < kTileElems / 10) {
-                const int64_t word_id = tile * (kTileElems / 10) + threadIdx.x;
-                const int64_t n_words = (prm.n_elems + 9) / 10;
-                const uint16_t* src = reinterpret_cast<const uint16_t*>(s_codes) + threadIdx.x * 5;
-                uint32_t word = 0;
-#pragma unroll
-                for (int k = 0; k < 5; ++k) {
-                    const uint32_t two = src[k];
-                    word |= ((two & 0xFFu) | ((two >> 8) << 3)) << (6 * k);
-                }
-                if (word_id < n_words) reinterpret_cast<uint32_t*>(prm.packed)[word_id] = word;
-            }
-            __syncthreads();
+            uint2 bb;
+            bb.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+            bb.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+            *reinterpret_cast<uint2*>(s_codes + gl * G + (kl * NB + b) * 8) = bb;
         }
-        if (valid && kl == 0) {
-            prm.scale[g] = __float2half_rn(s);
-            prm.zero[g] = __float2half_rn(zb);
-            if (prm.zero_f32) prm.zero_f32[g] = zb;
-            if (prm.iters_out) prm.iters_out[g] = (uint8_t)accepted;
-        }
+    }
+    if (kl == 0) {
+        const int64_t gi = chunk * C::CG + gl;
+        prm.scale[gi] = __float2half_rn(g.s);
+        prm.zero[gi] = __float2half_rn(g.zb);
+        if (prm.zero_f32) prm.zero_f32[gi] = g.zb;
+        if (prm.err_out) prm.err_out[gi] = g.eb;
+        if (prm.iters_out) prm.iters_out[gi] = (uint8_t)g.na;
     }
 }
 
-template <int NBITS, int G>
+template <int NBITS, int G, int NB>
+__global__ void __launch_bounds__(kQWarps * 32, 5)
+quantize_kernel(const __grid_constant__ QuantParams prm) {
+    using C = QCfg<NBITS, G, NB>;
+    __shared__ QuantSmem S;
+    extern __shared__ __align__(16) uint8_t dyn[];
+
+    load_pow_smem(S.tp, prm.tp);
+    load_pow_smem(S.tq, prm.tq);
+    for (int i = threadIdx.x; i < prm.iters; i += blockDim.x) S.thr[i] = prm.shrink_thr[i];
+    if (threadIdx.x == 0) {
+        float b = prm.beta;
+        for (int t = 0; t < prm.iters; ++t) {
+            S.beta[t] = b;
+            b = __fmul_rn(b, prm.kappa);
+        }
+        S.beta[prm.iters] = b;
+        S.thr[prm.iters] = 0.0f;
+    }
+    __syncthreads();
+
+    const float2 pa1 = make_float2(prm.tp.a1, prm.tp.a1);
+    const float2 pa2 = make_float2(prm.tp.a2, prm.tp.a2);
+    const float2 pa3 = make_float2(prm.tp.a3, prm.tp.a3);
+    const float qa1 = prm.tq.a1, qa2 = prm.tq.a2, qa3 = prm.tq.a3;
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int sub = lane / C::K;
+    const int kl = lane % C::K;
+    const bool leader = kl == 0;
+    uint8_t* wb = dyn + warp * C::WARP_BYTES;
+    __half* s_w = reinterpret_cast<__half*>(wb);
+    float4* s_st = reinterpret_cast<float4*>(wb + C::W_BYTES);
+    float4* s_st2 = reinterpret_cast<float4*>(wb + C::W_BYTES + C::ST_BYTES);
+    uint8_t* s_q = wb + C::W_BYTES + C::ST_BYTES + C::ST2_BYTES;
+    uint8_t* s_codes = s_q + C::Q_BYTES;
+
+    const int64_t n_chunks = (prm.n_elems + kChunk - 1) / kChunk;
+    for (int64_t chunk = (int64_t)blockIdx.x * kQWarps + warp; chunk < n_chunks;
+         chunk += (int64_t)gridDim.x * kQWarps) {
+        const int64_t e0 = chunk * kChunk;
+        const int64_t left = prm.n_elems - e0;
+        const int n_here = left < kChunk ? (int)left : kChunk;
+        const int cg = n_here / G;
+
+        // ---- stage the chunk's weights (one pass over HBM) ---------------------
+        {
+            const uint4* src = reinterpret_cast<const uint4*>(prm.W + e0);
+            uint4* dst = reinterpret_cast<uint4*>(s_w);
+            for (int u = lane; u < n_here / 8; u += 32) dst[u] = __ldg(src + u);
+        }
+        __syncwarp();
+
+        // ---- phase A: initialise + first two iterations, all groups in step ---
+        int qn = 0;
+        for (int r = 0; r < C::ROUNDS; ++r) {
+            if (r * C::GPW >= cg) break;
+            const int gl = r * C::GPW + sub;
+            const bool valid = gl < cg;
+            float2 w[NB][4];
+            if (valid) {
+                load_lane<NB>(s_w + gl * G + kl * C::EPL, w);
+            } else {
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) w[b][k] = make_float2(0.0f, 0.0f);
+            }
+            GroupState g;
+            float mn = fminf(w[0][0].x, w[0][0].y), mx = fmaxf(w[0][0].x, w[0][0].y);
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    mn = fminf(mn, fminf(w[b][k].x, w[b][k].y));
+                    mx = fmaxf(mx, fmaxf(w[b][k].x, w[b][k].y));
+                }
+            group_minmax<C::K>(mn, mx);
+            g.mn = mn;
+            g.mx = mx;
+            const float rng = __fsub_rn(mx, mn);
+            g.s = 1.0f;
+            g.inv = 1.0f;
+            if (rng != 0.0f) {
+                g.s = __fdiv_rn(rng, (float)C::L);
+                g.inv = __fdiv_rn(1.0f, g.s);
+            }
+            g.z = -__fmul_rn(mn, g.inv);
+            g.zb = g.z;
+            g.eb = __int_as_float(0x7F800000);
+            g.t = 0;
+            g.na = 0;
+            bool live = valid && prm.iters > 0;
+            bool done = valid && prm.iters == 0;
+            const int ta = prm.iters < 2 ? prm.iters : 2;
+            for (int tt = 0; tt < ta; ++tt) {
+                const bool fin = solver_step<NBITS, G, NB>(S, prm, w, g, live, pa1, pa2, pa3,
+                                                           qa1, qa2, qa3);
+                done = done || fin;
+                live = live && !fin;
+            }
+            if (__any_sync(kFull, done)) {
+                if (done) finalize<NBITS, G, NB>(prm, w, g, chunk, gl, kl, s_codes);
+            }
+            const unsigned pmask = __ballot_sync(kFull, live && leader);
+            if (live && leader) {
+                const int slot = qn + __popc(pmask & ((1u << lane) - 1u));
+                s_q[slot] = (uint8_t)gl;
+                s_st[gl] = make_float4(g.z, g.zb, g.eb, g.s);
+                s_st2[gl] = make_float4(g.inv, g.mn, g.mx, 0.0f);
+            }
+            qn += __popc(pmask);
+        }
+        __syncwarp();
+
+        // ---- phase B: queued groups, refilled as each sub-warp finishes -------
+        {
+            int head = 0;
+            bool live = false;
+            int gl = 0;
+            GroupState g;
+            g.z = g.zb = g.eb = g.s = g.inv = g.mn = g.mx = 0.0f;
+            g.t = 0;
+            g.na = 0;
+            float2 w[NB][4];
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) w[b][k] = make_float2(0.0f, 0.0f);
+            while (true) {
+                const unsigned want = __ballot_sync(kFull, !live && leader);
+                if (head < qn && want) {
+                    const int slot = head + __popc(want & ((1u << (sub * C::K)) - 1u));
+                    if (!live && slot < qn) {
+                        gl = s_q[slot];
+                        load_lane<NB>(s_w + gl * G + kl * C::EPL, w);
+                        const float4 a = s_st[gl];
+                        const float4 b = s_st2[gl];
+                        g.z = a.x;
+                        g.zb = a.y;
+                        g.eb = a.z;
+                        g.s = a.w;
+                        g.inv = b.x;
+                        g.mn = b.y;
+                        g.mx = b.z;
+                        g.t = 2;
+                        g.na = 2;
+                        live = true;
+                    }
+                    head = min(qn, head + __popc(want));
+                }
+                if (!__any_sync(kFull, live)) break;
+                const bool fin = solver_step<NBITS, G, NB>(S, prm, w, g, live, pa1, pa2, pa3,
+                                                           qa1, qa2, qa3);
+                if (__any_sync(kFull, fin)) {
+                    if (fin) finalize<NBITS, G, NB>(prm, w, g, chunk, gl, kl, s_codes);
+                }
+                live = live && !fin;
+            }
+        }
+
+        // ---- 3-bit: whole words of this chunk from the staged codes ------------
+        if constexpr (NBITS == 3) {
+            __syncwarp();
+            const int n_words = (n_here + 9) / 10;
+            if (lane < n_words * 10 - n_here) s_codes[n_here + lane] = 0;   // zero padding
+            __syncwarp();
+            const int64_t total_words = (prm.n_elems + 9) / 10;
+            for (int k = lane; k < n_words; k += 32) {
+                const uint16_t* src = reinterpret_cast<const uint16_t*>(s_codes) + k * 5;
+                uint32_t word = 0;
+#pragma unroll
+                for (int i = 0; i < 5; ++i) {
+                    const uint32_t two = src[i];
+                    word |= ((two & 0xFFu) | ((two >> 8) << 3)) << (6 * i);
+                }
+                const int64_t wi = chunk * (kChunk / 10) + k;
+                if (wi < total_words) reinterpret_cast<uint32_t*>(prm.packed)[wi] = word;
+            }
+        }
+        __syncwarp();
+    }
+}
+
+template <int NBITS, int G, int NB>
 static cudaError_t launch_quantize_g(const QuantParams& prm, cudaStream_t stream) {
-    constexpr int GPC = (32 / (G / 8)) * (kQuantThreads / 32);
-    const int64_t tiles = (prm.n_groups + GPC - 1) / GPC;
-    const unsigned grid = (unsigned)(tiles < (1 << 30) ? tiles : (1 << 30));
-    quantize_kernel<NBITS, G><<<grid, kQuantThreads, 0, stream>>>(prm);
+    using C = QCfg<NBITS, G, NB>;
+    auto kern = quantize_kernel<NBITS, G, NB>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQWarps * 32, C::SMEM);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) per_sm = 1;
+    const int64_t n_chunks = (prm.n_elems + kChunk - 1) / kChunk;
+    const int64_t want = (n_chunks + kQWarps - 1) / kQWarps;
+    const int64_t cap = (int64_t)sms * per_sm;
+    const unsigned grid = (unsigned)(want < cap ? want : cap);
+    kern<<<grid, kQWarps * 32, C::SMEM, stream>>>(prm);
     return cudaGetLastError();
 }
 
+// Weights per lane: 16 (two 8-weight blocks) for every group size.
 template <int NBITS>
 static cudaError_t launch_quantize_b(const QuantParams& prm, int group, cudaStream_t stream) {
     switch (group) {
-        case 16: return launch_quantize_g<NBITS, 16>(prm, stream);
-        case 32: return launch_quantize_g<NBITS, 32>(prm, stream);
-        case 64: return launch_quantize_g<NBITS, 64>(prm, stream);
-        case 128: return launch_quantize_g<NBITS, 128>(prm, stream);
-        case 256: return launch_quantize_g<NBITS, 256>(prm, stream);
+        case 16: return launch_quantize_g<NBITS, 16, 2>(prm, stream);
+        case 32: return launch_quantize_g<NBITS, 32, 2>(prm, stream);
+        case 64: return launch_quantize_g<NBITS, 64, 2>(prm, stream);
+        case 128: return launch_quantize_g<NBITS, 128, 2>(prm, stream);
+        case 256: return launch_quantize_g<NBITS, 256, 2>(prm, stream);
         default: return cudaErrorInvalidValue;
     }
 }
