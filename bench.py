@@ -73,6 +73,15 @@ def workload(name: str, rank: int = 0, layers: int | None = None):
     return out
 
 
+def max_over_ranks(values, pg, device=None):
+    """Element-wise max of a list of floats over all ranks (identity at N = 1)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if pg is not None:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def meta_bytes(rows, cols, group):
     return 2 * 2 * rows * (cols // group)
 
@@ -153,6 +162,30 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return 6650.0, "fallback"
+
+
+def profiled_traffic(kernel: str, fmt: str):
+    """DRAM bytes per weight of `kernel` from the committed ncu summary, or None
+    when the kernel's sources changed since the counters were taken."""
+    import glob
+    import hashlib
+    srcs = {"quantize_kernel": ["hqq_quantize.cu", "hqq_common.cuh"],
+            "dequantize_kernel": ["hqq_dequantize.cu", "hqq_common.cuh"]}[kernel]
+    m = hashlib.sha256()
+    for f in srcs:
+        with open(os.path.join(ROOT, "weight_only_quantization_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    cur = m.hexdigest()[:16]
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_*{fmt}*.txt"))):
+        kv = {}
+        with open(path) as fh:
+            for line in fh:
+                if ":" in line and not line.startswith("#"):
+                    k, _, v = line.partition(":")
+                    kv[k.strip()] = v.strip()
+        if kv.get("source_sha256_16") == cur and "traffic_bytes_per_param" in kv:
+            return float(kv["traffic_bytes_per_param"]), os.path.relpath(path, ROOT)
+    return None, None
 
 
 def cpu_cores():
@@ -350,10 +383,7 @@ def run_gpu(args):
     ms = t_start.elapsed_time(t_end)
     q_ms = [evs[s][k][0].elapsed_time(evs[s][k][1]) for s in range(args.steps)
             for k in range(len(views))]
-    ms_t = torch.tensor([ms, sum(q_ms)], dtype=torch.float64, device=dev)
-    if pg is not None:
-        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
-    ms_max, qsum_max = float(ms_t[0]), float(ms_t[1])
+    ms_max, qsum_max = max_over_ranks([ms, sum(q_ms)], pg, dev)
     ms_step = ms_max / args.steps
     value = ws * params * args.steps / (ms_max / 1e3) / 1e9
 
@@ -390,6 +420,9 @@ def run_gpu(args):
     sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
     alu_peak = props.multi_processor_count * ALU_LANES_PER_SM * sm_mhz * 1e6 / 1e12  # Tops/s
     achieved = ops_per_launch / (q_launch_ms / 1e3) / 1e12
+    fmts = sorted({f"{m[2]}b_g{m[3]}" for m in mats})
+    tpp, tsrc = profiled_traffic("quantize_kernel", fmts[0]) if len(fmts) == 1 else (None, None)
+    traffic = tpp * params / len(views) if tpp is not None else None
 
     line = {"metric": METRIC, "value": value, "unit": "Gparam/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -404,7 +437,8 @@ def run_gpu(args):
                            "ms_per_pass": dq_ms_step},
             "roofline": {"kernel": "quantize_kernel", "bound": "alu", "achieved": achieved,
                          "peak": alu_peak, "unit": "Tops/s", "frac": achieved / alu_peak,
-                         "traffic": None,
+                         "traffic": traffic, "traffic_unit": "bytes per launch",
+                         "traffic_source": tsrc,
                          "peak_source": f"{props.multi_processor_count} SMs x "
                                         f"{ALU_LANES_PER_SM} fp32 lanes x {sm_mhz:.0f} MHz",
                          "ops_per_weight": ops_per_weight,
@@ -511,14 +545,11 @@ def run_e2e(args, mats, views, hqq, dev, pg, ws):
         one_step()
     t1.record(s_comp)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if pg is not None:
-        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
+    ms = max_over_ranks([t0.elapsed_time(t1)], pg, dev)[0]
     params = sum(r * c for _, (r, c), *_ in mats)
-    return {"value": ws * params * steps / (float(ms_t[0]) / 1e3) / 1e9, "unit": "Gparam/s",
+    return {"value": ws * params * steps / (ms / 1e3) / 1e9, "unit": "Gparam/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "warmup": 1, "ms_per_step": float(ms_t[0]) / steps}
+            "warmup": 1, "ms_per_step": ms / steps}
 
 
 def main():
