@@ -74,19 +74,28 @@ __device__ __forceinline__ void load_pow_smem(PowSmem& dst, const PowTable& t) {
     }
 }
 
-// |x|^p of two values (any sign) with the table in shared memory.
+// Word at byte offset `off` of a shared-memory table.
+__device__ __forceinline__ float tab_at(const float* t, uint32_t off) {
+    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(t) + off);
+}
+
+// |x|^p of two values (any sign) with the table in shared memory.  The table
+// offsets are taken straight from the bit pattern: bits 23..30 (exponent of
+// |x|) times 4 and bits 18..22 (mantissa cell) times 4.
 __device__ __forceinline__ float2 powp2(const PowSmem& T, float2 a1, float2 a2, float2 a3,
                                         float2 x) {
     const uint32_t bx = __float_as_uint(x.x), by = __float_as_uint(x.y);
-    const uint32_t ex = (bx >> 23) & 0xFFu, ey = (by >> 23) & 0xFFu;   // exponent of |x|
-    const uint32_t jx = (bx >> 18) & 31u, jy = (by >> 18) & 31u;       // mantissa cell
+    const uint32_t ex = (bx >> 21) & 0x3FCu, ey = (by >> 21) & 0x3FCu;
+    const uint32_t jx = (bx >> 16) & 0x7Cu, jy = (by >> 16) & 0x7Cu;
     const float2 m = make_float2(__uint_as_float((bx & 0x007FFFFFu) | 0x3F800000u),
                                  __uint_as_float((by & 0x007FFFFFu) | 0x3F800000u));
-    const float2 r = __ffma2_rn(m, make_float2(T.ic[jx], T.ic[jy]), make_float2(-1.0f, -1.0f));
+    const float2 r = __ffma2_rn(m, make_float2(tab_at(T.ic, jx), tab_at(T.ic, jy)),
+                                make_float2(-1.0f, -1.0f));
     float2 poly = __ffma2_rn(r, a3, a2);
     poly = __ffma2_rn(poly, r, a1);
     poly = __ffma2_rn(poly, r, make_float2(1.0f, 1.0f));
-    const float2 tt = __fmul2_rn(make_float2(T.te[ex], T.te[ey]), make_float2(T.tc[jx], T.tc[jy]));
+    const float2 tt = __fmul2_rn(make_float2(tab_at(T.te, ex), tab_at(T.te, ey)),
+                                 make_float2(tab_at(T.tc, jx), tab_at(T.tc, jy)));
     return __fmul2_rn(tt, poly);
 }
 

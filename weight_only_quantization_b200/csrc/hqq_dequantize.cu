@@ -2,81 +2,113 @@
 // Learning Models", section 2: W_hat = s (Wq - z), as fp16((code - z) * s) in
 // binary32 from the stored fp16 scale and zero.
 //
-// Streaming kernel: the unit of work is 8 consecutive weights (one 16-byte
-// store), which always lie in one group (8 divides every group size).  Lane l
-// of a warp takes unit base + l, so each warp instruction reads a contiguous
-// run of packed codes and writes 512 contiguous bytes.
+// Streaming kernel (HBM-bound).  The unit of work is 8 consecutive weights:
+// one 16-byte output, always inside one group (8 divides every group size).
+// Lane l of a block takes units base + r*256 + l, so every warp load is a
+// contiguous run of packed codes and every warp store writes 512 contiguous
+// bytes; all loads of a thread's units are issued before any store.  No shared
+// memory, so occupancy is limited only by registers (staging the output tile
+// in shared memory for TMA bulk stores measured slower: it cost occupancy).
+//
+// A code c at bit offset k of a field becomes an exact binary32 value without
+// a shift per code: OR-ing the masked field into the mantissa of 2^23 gives
+// 2^23 + c 2^k, and fma(x, 2^-k, -2^(23-k)) = c exactly (exact while
+// c 2^k < 2^23).  Two codes go through each f32x2 operation; (c - z) is exact
+// for fp16 z, so the only roundings are the product with s and the conversion
+// to fp16, as the definition requires.
 #include "hqq_common.cuh"
 
 namespace hqq {
 
 constexpr int kDqThreads = 256;
-constexpr int kDqUnroll = 4;
+constexpr int kDqUnits = 4;                          // units per thread per pass
+constexpr int kDqTile = kDqThreads * kDqUnits;
 
-__device__ __forceinline__ float code_to_float(uint32_t c) {
-    return __fsub_rn(__uint_as_float(0x4B000000u | c), 8388608.0f);   // exact for c < 2^23
+// Exact codes of the fields (mask0) of x0 and (mask1) of x1, as a pair.
+__device__ __forceinline__ float2 codes2(uint32_t x0, uint32_t mask0, float inv0, float off0,
+                                         uint32_t x1, uint32_t mask1, float inv1, float off1) {
+    const float2 f = make_float2(__uint_as_float((x0 & mask0) | 0x4B000000u),
+                                 __uint_as_float((x1 & mask1) | 0x4B000000u));
+    return __ffma2_rn(f, make_float2(inv0, inv1), make_float2(off0, off1));
 }
 
-template <int NBITS>
-__device__ __forceinline__ void unit_codes(const uint8_t* __restrict__ packed, int64_t u,
-                                           uint32_t (&c)[8]) {
+// fp16((c - z) * s) of a pair of codes, packed into one 32-bit word.
+__device__ __forceinline__ uint32_t dq2(float2 c, float z, float s) {
+    const float2 v = __fmul2_rn(__fadd2_rn(c, make_float2(-z, -z)), make_float2(s, s));
+    const __half2 h = __floats2half2_rn(v.x, v.y);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Eight codes of bit width B stored LSB-first in the low 8*B bits of `x`.
+template <int B>
+__device__ __forceinline__ uint4 unit8(uint32_t x, float z, float s) {
+    constexpr uint32_t M = (1u << B) - 1u;
+    const uint32_t lo = x, hi = x >> (4 * B);        // fields 0..3 and 4..7, each < 2^16
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int k0 = 2 * j * B, k1 = (2 * j + 1) * B;
+        const float2 a = codes2(lo, M << k0, 1.0f / (float)(1u << k0), -(float)(1u << (23 - k0)),
+                                lo, M << k1, 1.0f / (float)(1u << k1), -(float)(1u << (23 - k1)));
+        const float2 b = codes2(hi, M << k0, 1.0f / (float)(1u << k0), -(float)(1u << (23 - k0)),
+                                hi, M << k1, 1.0f / (float)(1u << k1), -(float)(1u << (23 - k1)));
+        o[j] = dq2(a, z, s);
+        o[j + 2] = dq2(b, z, s);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The 8*NBITS code bits of unit u, LSB-first.  4/2 bit: one aligned field.
+// 3 bit: codes 8u..8u+7 start at slot k0 = 8u mod 10 of word w0 = floor(8u/10)
+// and reach into word w0 + 1 when k0 > 2 (that word exists: it holds the
+// unit's own last code); words hold 10 codes in bits 0..29.  SMALL: 4u fits
+// in 32 bits, so w0 = floor(4u/5) is one multiply-high.
+template <int NBITS, bool SMALL>
+__device__ __forceinline__ uint32_t unit_bits(const uint8_t* __restrict__ packed, int64_t u) {
     if constexpr (NBITS == 4) {
-        const uint32_t wd = __ldg(reinterpret_cast<const uint32_t*>(packed) + u);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) c[i] = (wd >> (4 * i)) & 15u;
+        return __ldg(reinterpret_cast<const uint32_t*>(packed) + u);
     } else if constexpr (NBITS == 2) {
-        const uint32_t h = __ldg(reinterpret_cast<const uint16_t*>(packed) + u);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) c[i] = (h >> (2 * i)) & 3u;
+        return __ldg(reinterpret_cast<const uint16_t*>(packed) + u);
     } else {
-        const int64_t e0 = u * 8;
-        const int64_t w0 = e0 / 10;
-        const uint32_t k0 = (uint32_t)(e0 - w0 * 10);       // 0, 2, 4, 6 or 8
+        int64_t w0;
+        uint32_t k0;
+        if (SMALL) {
+            const uint32_t u4 = 4u * (uint32_t)u;
+            const uint32_t q = __umulhi(u4, 0xCCCCCCCDu) >> 2;      // floor(u4 / 5)
+            w0 = q;
+            k0 = 2u * (u4 - 5u * q);                                 // 8u mod 10
+        } else {
+            w0 = (4 * u) / 5;
+            k0 = (uint32_t)(8 * u - 10 * w0);
+        }
         const uint32_t* p32 = reinterpret_cast<const uint32_t*>(packed);
         const uint64_t lo = __ldg(p32 + w0);
-        // codes k0..k0+7 reach into the next word when k0 > 2 (that word exists:
-        // it holds the unit's own last code)
         const uint64_t hi = k0 > 2 ? (uint64_t)__ldg(p32 + w0 + 1) : 0ull;
-        const uint64_t v = (lo | (hi << 30)) >> (3 * k0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) c[i] = (uint32_t)(v >> (3 * i)) & 7u;
+        return (uint32_t)((lo | (hi << 30)) >> (3 * k0));
     }
 }
 
-template <int NBITS>
+template <int NBITS, bool SMALL>
 __global__ void __launch_bounds__(kDqThreads)
 dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
-    const int64_t per_block = (int64_t)kDqThreads * kDqUnroll;
-    for (int64_t base = (int64_t)blockIdx.x * per_block; base < prm.n_units;
-         base += (int64_t)gridDim.x * per_block) {
-        // all loads of the kDqUnroll units first, so they are in flight together
-        uint32_t c[kDqUnroll][8];
-        float sf[kDqUnroll], zf[kDqUnroll];
-        bool ok[kDqUnroll];
+    for (int64_t base = (int64_t)blockIdx.x * kDqTile; base < prm.n_units;
+         base += (int64_t)gridDim.x * kDqTile) {
+        uint32_t x[kDqUnits];
+        float sf[kDqUnits], zf[kDqUnits];
 #pragma unroll
-        for (int r = 0; r < kDqUnroll; ++r) {
-            const int64_t u = base + r * kDqThreads + threadIdx.x;
-            ok[r] = u < prm.n_units;
-            const int64_t uu = ok[r] ? u : 0;
-            const int64_t g = (uu * 8) >> log2_group;
+        for (int r = 0; r < kDqUnits; ++r) {        // all loads first
+            int64_t u = base + r * kDqThreads + threadIdx.x;
+            if (u >= prm.n_units) u = 0;
+            const int64_t g = (u * 8) >> log2_group;
             sf[r] = __half2float(__ldg(prm.scale + g));
             zf[r] = __half2float(__ldg(prm.zero + g));
-            unit_codes<NBITS>(prm.packed, uu, c[r]);
+            x[r] = unit_bits<NBITS, SMALL>(prm.packed, u);
         }
 #pragma unroll
-        for (int r = 0; r < kDqUnroll; ++r) {
-            uint32_t o[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float a = __fmul_rn(__fsub_rn(code_to_float(c[r][2 * k]), zf[r]), sf[r]);
-                const float b = __fmul_rn(__fsub_rn(code_to_float(c[r][2 * k + 1]), zf[r]), sf[r]);
-                const __half2 h = __floats2half2_rn(a, b);
-                o[k] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            if (ok[r]) {
-                const int64_t u = base + r * kDqThreads + threadIdx.x;
-                reinterpret_cast<uint4*>(prm.out)[u] = make_uint4(o[0], o[1], o[2], o[3]);
-            }
+        for (int r = 0; r < kDqUnits; ++r) {
+            const int64_t u = base + r * kDqThreads + threadIdx.x;
+            const uint4 o = unit8<NBITS>(x[r], zf[r], sf[r]);
+            if (u < prm.n_units) reinterpret_cast<uint4*>(prm.out)[u] = o;
         }
     }
 }
@@ -86,14 +118,18 @@ cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_grou
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t per_block = (int64_t)kDqThreads * kDqUnroll;
-    int64_t blocks = (prm.n_units + per_block - 1) / per_block;
+    int64_t blocks = (prm.n_units + kDqTile - 1) / kDqTile;
     const int64_t cap = (int64_t)sms * 32;
     if (blocks > cap) blocks = cap;
+    const bool small = prm.n_units < ((int64_t)1 << 30);
+    const unsigned g = (unsigned)blocks;
     switch (nbits) {
-        case 2: dequantize_kernel<2><<<(unsigned)blocks, kDqThreads, 0, stream>>>(prm, log2_group); break;
-        case 3: dequantize_kernel<3><<<(unsigned)blocks, kDqThreads, 0, stream>>>(prm, log2_group); break;
-        case 4: dequantize_kernel<4><<<(unsigned)blocks, kDqThreads, 0, stream>>>(prm, log2_group); break;
+        case 2: dequantize_kernel<2, true><<<g, kDqThreads, 0, stream>>>(prm, log2_group); break;
+        case 4: dequantize_kernel<4, true><<<g, kDqThreads, 0, stream>>>(prm, log2_group); break;
+        case 3:
+            if (small) dequantize_kernel<3, true><<<g, kDqThreads, 0, stream>>>(prm, log2_group);
+            else dequantize_kernel<3, false><<<g, kDqThreads, 0, stream>>>(prm, log2_group);
+            break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
