@@ -240,3 +240,20 @@ def test_repeat_calls_are_deterministic(hqq):
     b = hqq.hqq_quantize_ex(W, 4, 64)
     torch.cuda.synchronize()
     assert torch.equal(a.packed, b.packed) and torch.equal(a.zero_f32, b.zero_f32)
+
+
+# ------------------------------- several chunks per warp (group carry-over path)
+@pytest.mark.parametrize("nbits", [4, 3, 2])
+@pytest.mark.parametrize("group", [16, 32, 64, 128, 256])
+def test_multi_chunk_per_warp(hqq, nbits, group):
+    # 16.8 M weights = 6554 chunks of 2560: more than one chunk per resident warp,
+    # so groups still running at the end of a chunk are carried to the next one
+    W, Wn = _dev_weights((2048, 8192), seed=30, stream=group * 10 + nbits)
+    _, _, st = _check(hqq, W, Wn, nbits, group, f"multi-chunk {nbits}b g{group}")
+    assert st["code_match"] == 1.0
+
+
+@pytest.mark.parametrize("group", [64, 16])
+def test_multi_chunk_shrink_active(hqq, group):
+    W, Wn = _dev_weights((2048, 8192), seed=31, stream=group, std=1.0)
+    _check(hqq, W, Wn, 4, group, f"multi-chunk std 1 4b g{group}")

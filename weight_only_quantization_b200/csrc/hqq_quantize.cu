@@ -43,12 +43,19 @@ struct QCfg {
     static constexpr int CG = kChunk / G;        // groups per chunk
     static constexpr int L = (1 << NBITS) - 1;
     static constexpr int W_BYTES = kChunk * 2;
-    static constexpr int ST_BYTES = CG * 16;     // (z, zb, eb, s) of queued groups
-    static constexpr int ST2_BYTES = CG * 16;    // (1/s, min, max, -)
+    static constexpr int ST_BYTES = CG * 16;     // (z, zb, eb, s) per group
+    static constexpr int ST2_BYTES = CG * 16;    // (1/s, min, max, t << 16 | accepted)
     static constexpr int Q_BYTES = (CG + 15) / 16 * 16;
-    static constexpr int CODE_BYTES = NBITS == 3 ? kChunk : 0;
-    static constexpr int WARP_BYTES = W_BYTES + ST_BYTES + ST2_BYTES + Q_BYTES + CODE_BYTES;
-    static constexpr int SMEM = kQWarps * WARP_BYTES;
+    static constexpr int SLOTS = GPW;            // phase-B slots per warp (this layout)
+    static constexpr int POOL_W_BYTES = SLOTS * G * 2;
+    static constexpr int POOL_ST_BYTES = SLOTS * 32;
+    static constexpr int POOL_GI_BYTES = (SLOTS * 8 + 15) / 16 * 16;
+    static constexpr int CHUNK_BYTES = W_BYTES + ST_BYTES + ST2_BYTES + Q_BYTES;
+    static constexpr int POOL_BYTES = POOL_W_BYTES + POOL_ST_BYTES + POOL_GI_BYTES;
+    // every region starts on a 16-byte boundary (128-bit shared-memory accesses)
+    static_assert(W_BYTES % 16 == 0 && ST_BYTES % 16 == 0 && ST2_BYTES % 16 == 0 &&
+                  Q_BYTES % 16 == 0 && POOL_W_BYTES % 16 == 0 && POOL_ST_BYTES % 16 == 0 &&
+                  POOL_GI_BYTES % 16 == 0, "shared-memory regions must be 16-byte multiples");
     static_assert(K >= 1 && K <= 32 && kChunk % ROUND == 0, "bad layout");
 };
 
@@ -93,6 +100,32 @@ __device__ __forceinline__ void load_lane(const __half* src, float2 (&w)[NB][4])
         w[b][2] = make_float2(__low2float(h23), __low2float(h67));
         w[b][3] = make_float2(__high2float(h23), __high2float(h67));
     }
+}
+
+// load_lane plus the lane's min and max, taken on the packed fp16 values
+// (exact: the conversion to binary32 is exact and monotone).
+template <int NB>
+__device__ __forceinline__ void load_lane_minmax(const __half* src, float2 (&w)[NB][4],
+                                                 float& mn, float& mx) {
+    __half2 hmn, hmx;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const uint4 raw = reinterpret_cast<const uint4*>(src)[b];
+        const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
+        const __half2 h23 = *reinterpret_cast<const __half2*>(&raw.y);
+        const __half2 h45 = *reinterpret_cast<const __half2*>(&raw.z);
+        const __half2 h67 = *reinterpret_cast<const __half2*>(&raw.w);
+        const __half2 bmn = __hmin2(__hmin2(h01, h23), __hmin2(h45, h67));
+        const __half2 bmx = __hmax2(__hmax2(h01, h23), __hmax2(h45, h67));
+        hmn = b == 0 ? bmn : __hmin2(hmn, bmn);
+        hmx = b == 0 ? bmx : __hmax2(hmx, bmx);
+        w[b][0] = make_float2(__low2float(h01), __low2float(h45));
+        w[b][1] = make_float2(__high2float(h01), __high2float(h45));
+        w[b][2] = make_float2(__low2float(h23), __low2float(h67));
+        w[b][3] = make_float2(__high2float(h23), __high2float(h67));
+    }
+    mn = fminf(__low2float(hmn), __high2float(hmn));
+    mx = fmaxf(__low2float(hmx), __high2float(hmx));
 }
 
 // Per-group constants of one evaluation, as f32x2 pairs.
@@ -212,46 +245,101 @@ __device__ __forceinline__ bool solver_step(const QuantSmem& S, const QuantParam
     return live && (!acc || g.t == prm.iters);
 }
 
-// Final codes of the sub-warp's group, packed, plus its scale and zero.
-template <int NBITS, int G, int NB>
-__device__ __forceinline__ void finalize(const QuantParams& prm, const float2 (&w)[NB][4],
-                                         const GroupState& g, int64_t chunk, int gl, int kl,
-                                         uint8_t* s_codes) {
-    using C = QCfg<NBITS, G, NB>;
-    constexpr float L = (float)C::L;
-    const float2 inv2 = make_float2(g.inv, g.inv), zb2 = make_float2(g.zb, g.zb);
+// Group state kept in the chunk's shared memory between phases.
+__device__ __forceinline__ void save_state(float4* st, float4* st2, int gl, const GroupState& g) {
+    st[gl] = make_float4(g.z, g.zb, g.eb, g.s);
+    st2[gl] = make_float4(g.inv, g.mn, g.mx, __int_as_float((g.t << 16) | g.na));
+}
+
+__device__ __forceinline__ void load_state(const float4* st, const float4* st2, int gl,
+                                           GroupState& g) {
+    const float4 a = st[gl];
+    const float4 b = st2[gl];
+    g.z = a.x;
+    g.zb = a.y;
+    g.eb = a.z;
+    g.s = a.w;
+    g.inv = b.x;
+    g.mn = b.y;
+    g.mx = b.z;
+    const int tn = __float_as_int(b.w);
+    g.t = (tn >> 16) & 0xFF;
+    g.na = tn & 0xFFFF;
+}
+
+constexpr int kCarried = 1 << 30;   // flag in the packed (t, accepted) word
+constexpr int kPoolTag = 256;       // queue handles >= kPoolTag name pool entries
+
+// Pack the lane's weights back to fp16 in memory order (exact: they came from fp16).
+template <int NB>
+__device__ __forceinline__ void store_lane(__half* dst, const float2 (&w)[NB][4]) {
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-        uint32_t c[8];
+        const __half2 h01 = __floats2half2_rn(w[b][0].x, w[b][1].x);
+        const __half2 h23 = __floats2half2_rn(w[b][2].x, w[b][3].x);
+        const __half2 h45 = __floats2half2_rn(w[b][0].y, w[b][1].y);
+        const __half2 h67 = __floats2half2_rn(w[b][2].y, w[b][3].y);
+        uint4 raw;
+        raw.x = *reinterpret_cast<const uint32_t*>(&h01);
+        raw.y = *reinterpret_cast<const uint32_t*>(&h23);
+        raw.z = *reinterpret_cast<const uint32_t*>(&h45);
+        raw.w = *reinterpret_cast<const uint32_t*>(&h67);
+        reinterpret_cast<uint4*>(dst)[b] = raw;
+    }
+}
+
+// Final codes of one group finished after its chunk was written (a group
+// carried over to a later chunk): codes go straight to HBM; 3 bit codes are
+// OR-ed into the words, whose bits for this group were written as zero.
+template <int NBITS, int G, int NB>
+__device__ __forceinline__ void finalize_direct(const QuantParams& prm, const float2 (&w)[NB][4],
+                                                const GroupState& g, int64_t gi, int kl) {
+    constexpr float L = (float)((1 << NBITS) - 1);
+    const float2 inv2 = make_float2(g.inv, g.inv), zb2 = make_float2(g.zb, g.zb);
+    uint32_t c[NB][8];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             float2 v = __ffma2_rn(w[b][k], inv2, zb2);
             v.x = fminf(fmaxf(v.x, 0.0f), L);
             v.y = fminf(fmaxf(v.y, 0.0f), L);
             const float2 t = __fadd2_rn(v, make_float2(kRoundShift, kRoundShift));
-            c[k] = __float_as_uint(t.x) & 0xFFu;
-            c[k + 4] = __float_as_uint(t.y) & 0xFFu;
+            c[b][k] = __float_as_uint(t.x) & 0xFFu;
+            c[b][k + 4] = __float_as_uint(t.y) & 0xFFu;
         }
-        const int64_t unit = chunk * (kChunk / 8) + gl * (G / 8) + kl * NB + b;   // 8-weight unit
-        if constexpr (NBITS == 4) {
+    if constexpr (NBITS == 3) {
+        const int64_t e0 = gi * G + (int64_t)kl * 8 * NB;    // first element of the lane
+        const int64_t w0 = e0 / 10;
+        uint32_t acc[3] = {0u, 0u, 0u};                       // 8 NB <= 16 codes span <= 3 words
+        int off = (int)(e0 - w0 * 10);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int pos = off + 8 * b + i;
+                const int wi = pos / 10;
+                const uint32_t bits = c[b][i] << (3 * (pos - 10 * wi));
+                if (wi == 0) acc[0] |= bits;
+                else if (wi == 1) acc[1] |= bits;
+                else acc[2] |= bits;
+            }
+        uint32_t* p32 = reinterpret_cast<uint32_t*>(prm.packed);
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+            if (acc[k]) atomicOr(p32 + w0 + k, acc[k]);
+    } else {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            const int64_t unit = gi * (G / 8) + kl * NB + b;
             uint32_t word = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) word |= c[i] << (4 * i);
-            reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
-        } else if constexpr (NBITS == 2) {
-            uint32_t h = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) h |= c[i] << (2 * i);
-            reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)h;
-        } else {
-            uint2 bb;
-            bb.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-            bb.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-            *reinterpret_cast<uint2*>(s_codes + gl * G + (kl * NB + b) * 8) = bb;
+            for (int i = 0; i < 8; ++i) word |= c[b][i] << (NBITS * i);
+            if constexpr (NBITS == 4) reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
+            else reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)word;
         }
     }
     if (kl == 0) {
-        const int64_t gi = chunk * C::CG + gl;
         prm.scale[gi] = __float2half_rn(g.s);
         prm.zero[gi] = __float2half_rn(g.zb);
         if (prm.zero_f32) prm.zero_f32[gi] = g.zb;
@@ -260,10 +348,90 @@ __device__ __forceinline__ void finalize(const QuantParams& prm, const float2 (&
     }
 }
 
+// Final codes of every group of a chunk (one uniform pass, phase-A layout),
+// from the staged weights and each group's (z_best, 1/s); 4 and 2 bit codes
+// are stored straight to HBM, 3 bit code bytes overwrite the front of the
+// chunk's weight buffer (round r writes bytes [512r, 512r+512), never ahead of
+// the weights still to be read) for word packing.  Scale, zero and the
+// diagnostics are written by each group's first lane.
 template <int NBITS, int G, int NB>
+__device__ __forceinline__ void final_pass(const QuantParams& prm, __half* s_w, const float4* st,
+                                           const float4* st2, int64_t chunk, int cg, int lane) {
+    using C = QCfg<NBITS, G, NB>;
+    constexpr float L = (float)C::L;
+    const int sub = lane / C::K, kl = lane % C::K;
+    uint8_t* codes = reinterpret_cast<uint8_t*>(s_w);
+    for (int r = 0; r < C::ROUNDS; ++r) {
+        if (r * C::GPW >= cg) break;
+        const int gl = r * C::GPW + sub;
+        const bool valid = gl < cg;
+        float2 w[NB][4];
+        GroupState g;
+        bool mine = valid;                          // false: carried over, finalised later
+        if (valid) {
+            load_lane<NB>(s_w + gl * G + kl * C::EPL, w);
+            load_state(st, st2, gl, g);
+            mine = (__float_as_int(st2[gl].w) & kCarried) == 0;
+        } else {
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) w[b][k] = make_float2(0.0f, 0.0f);
+            g.zb = 0.0f;
+            g.inv = 1.0f;
+        }
+        if constexpr (NBITS == 3) __syncwarp();     // all reads of the round before any write
+        const float2 inv2 = make_float2(g.inv, g.inv), zb2 = make_float2(g.zb, g.zb);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            uint32_t c[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float2 v = __ffma2_rn(w[b][k], inv2, zb2);
+                v.x = fminf(fmaxf(v.x, 0.0f), L);
+                v.y = fminf(fmaxf(v.y, 0.0f), L);
+                const float2 t = __fadd2_rn(v, make_float2(kRoundShift, kRoundShift));
+                c[k] = mine ? __float_as_uint(t.x) & 0xFFu : 0u;
+                c[k + 4] = mine ? __float_as_uint(t.y) & 0xFFu : 0u;
+            }
+            if (!valid || (!mine && NBITS != 3)) continue;
+            const int64_t unit = chunk * (kChunk / 8) + gl * (G / 8) + kl * NB + b;
+            if constexpr (NBITS == 4) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) word |= c[i] << (4 * i);
+                reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
+            } else if constexpr (NBITS == 2) {
+                uint32_t h = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) h |= c[i] << (2 * i);
+                reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)h;
+            } else {
+                uint2 bb;
+                bb.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+                bb.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+                *reinterpret_cast<uint2*>(codes + gl * G + (kl * NB + b) * 8) = bb;
+            }
+        }
+        if (mine && kl == 0) {
+            const int64_t gi = chunk * C::CG + gl;
+            prm.scale[gi] = __float2half_rn(g.s);
+            prm.zero[gi] = __float2half_rn(g.zb);
+            if (prm.zero_f32) prm.zero_f32[gi] = g.zb;
+            if (prm.err_out) prm.err_out[gi] = g.eb;
+            if (prm.iters_out) prm.iters_out[gi] = (uint8_t)g.na;
+        }
+    }
+}
+
+// NB / NBB: 8-weight blocks per lane in phase A / phase B.  CARRY: park the
+// last busy groups of a chunk and resume them with the next chunk, parking
+// once at most PARK/4 of the phase-B slots are busy.
+template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK>
 __global__ void __launch_bounds__(kQWarps * 32, 5)
 quantize_kernel(const __grid_constant__ QuantParams prm) {
-    using C = QCfg<NBITS, G, NB>;
+    using C = QCfg<NBITS, G, NB>;      // phase A layout (and the chunk's shared memory)
+    using CB = QCfg<NBITS, G, NBB>;    // phase B layout
     __shared__ QuantSmem S;
     extern __shared__ __align__(16) uint8_t dyn[];
 
@@ -291,12 +459,17 @@ quantize_kernel(const __grid_constant__ QuantParams prm) {
     const int sub = lane / C::K;
     const int kl = lane % C::K;
     const bool leader = kl == 0;
-    uint8_t* wb = dyn + warp * C::WARP_BYTES;
+    constexpr int WARP_BYTES = C::CHUNK_BYTES + (CARRY ? CB::POOL_BYTES : 0);
+    uint8_t* wb = dyn + warp * WARP_BYTES;
     __half* s_w = reinterpret_cast<__half*>(wb);
     float4* s_st = reinterpret_cast<float4*>(wb + C::W_BYTES);
     float4* s_st2 = reinterpret_cast<float4*>(wb + C::W_BYTES + C::ST_BYTES);
     uint8_t* s_q = wb + C::W_BYTES + C::ST_BYTES + C::ST2_BYTES;
-    uint8_t* s_codes = s_q + C::Q_BYTES;
+    __half* pool_w = reinterpret_cast<__half*>(s_q + C::Q_BYTES);
+    float4* pool_st = reinterpret_cast<float4*>(s_q + C::Q_BYTES + CB::POOL_W_BYTES);
+    int64_t* pool_gi = reinterpret_cast<int64_t*>(s_q + C::Q_BYTES + CB::POOL_W_BYTES +
+                                                  CB::POOL_ST_BYTES);
+    int np = 0;                        // groups parked in the pool by the last yield
 
     const int64_t n_chunks = (prm.n_elems + kChunk - 1) / kChunk;
     for (int64_t chunk = (int64_t)blockIdx.x * kQWarps + warp; chunk < n_chunks;
@@ -321,23 +494,17 @@ quantize_kernel(const __grid_constant__ QuantParams prm) {
             const int gl = r * C::GPW + sub;
             const bool valid = gl < cg;
             float2 w[NB][4];
+            float mn, mx;
             if (valid) {
-                load_lane<NB>(s_w + gl * G + kl * C::EPL, w);
+                load_lane_minmax<NB>(s_w + gl * G + kl * C::EPL, w, mn, mx);
             } else {
 #pragma unroll
                 for (int b = 0; b < NB; ++b)
 #pragma unroll
                     for (int k = 0; k < 4; ++k) w[b][k] = make_float2(0.0f, 0.0f);
+                mn = mx = 0.0f;
             }
             GroupState g;
-            float mn = fminf(w[0][0].x, w[0][0].y), mx = fmaxf(w[0][0].x, w[0][0].y);
-#pragma unroll
-            for (int b = 0; b < NB; ++b)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    mn = fminf(mn, fminf(w[b][k].x, w[b][k].y));
-                    mx = fmaxf(mx, fmaxf(w[b][k].x, w[b][k].y));
-                }
             group_minmax<C::K>(mn, mx);
             g.mn = mn;
             g.mx = mx;
@@ -346,7 +513,7 @@ quantize_kernel(const __grid_constant__ QuantParams prm) {
             g.inv = 1.0f;
             if (rng != 0.0f) {
                 g.s = __fdiv_rn(rng, (float)C::L);
-                g.inv = __fdiv_rn(1.0f, g.s);
+                g.inv = __frcp_rn(g.s);             // correctly rounded 1/s
             }
             g.z = -__fmul_rn(mn, g.inv);
             g.zb = g.z;
@@ -362,68 +529,97 @@ quantize_kernel(const __grid_constant__ QuantParams prm) {
                 done = done || fin;
                 live = live && !fin;
             }
-            if (__any_sync(kFull, done)) {
-                if (done) finalize<NBITS, G, NB>(prm, w, g, chunk, gl, kl, s_codes);
-            }
+            if ((done || live) && leader) save_state(s_st, s_st2, gl, g);
             const unsigned pmask = __ballot_sync(kFull, live && leader);
-            if (live && leader) {
-                const int slot = qn + __popc(pmask & ((1u << lane) - 1u));
-                s_q[slot] = (uint8_t)gl;
-                s_st[gl] = make_float4(g.z, g.zb, g.eb, g.s);
-                s_st2[gl] = make_float4(g.inv, g.mn, g.mx, 0.0f);
-            }
+            if (live && leader) s_q[qn + __popc(pmask & ((1u << lane) - 1u))] = (uint8_t)gl;
             qn += __popc(pmask);
         }
         __syncwarp();
 
         // ---- phase B: queued groups, refilled as each sub-warp finishes -------
+        // The queue holds the groups parked by the previous chunk (pool entries
+        // 0..np-1) and then this chunk's continuing groups.  Once the queue is
+        // empty and at most half the slots are busy, the warp parks the busy
+        // groups in the pool and moves on (unless this is its last chunk), so the
+        // longest groups never leave the other slots idle.
         {
+            const int subb = lane / CB::K;
+            const int klb = lane % CB::K;
+            const bool leadb = klb == 0;
+            const bool more = CARRY && chunk + (int64_t)gridDim.x * kQWarps < n_chunks;
+            const int nq = np + qn;
             int head = 0;
             bool live = false;
-            int gl = 0;
+            int hnd = 0;                   // < kPoolTag: chunk group gl; else pool entry
+            int64_t gi = 0;
             GroupState g;
             g.z = g.zb = g.eb = g.s = g.inv = g.mn = g.mx = 0.0f;
             g.t = 0;
             g.na = 0;
-            float2 w[NB][4];
+            float2 w[NBB][4];
 #pragma unroll
-            for (int b = 0; b < NB; ++b)
+            for (int b = 0; b < NBB; ++b)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) w[b][k] = make_float2(0.0f, 0.0f);
+            int parked = 0;
             while (true) {
-                const unsigned want = __ballot_sync(kFull, !live && leader);
-                if (head < qn && want) {
-                    const int slot = head + __popc(want & ((1u << (sub * C::K)) - 1u));
-                    if (!live && slot < qn) {
-                        gl = s_q[slot];
-                        load_lane<NB>(s_w + gl * G + kl * C::EPL, w);
-                        const float4 a = s_st[gl];
-                        const float4 b = s_st2[gl];
-                        g.z = a.x;
-                        g.zb = a.y;
-                        g.eb = a.z;
-                        g.s = a.w;
-                        g.inv = b.x;
-                        g.mn = b.y;
-                        g.mx = b.z;
-                        g.t = 2;
-                        g.na = 2;
+                const unsigned want = __ballot_sync(kFull, !live && leadb);
+                if (head < nq && want) {
+                    const int slot = head + __popc(want & ((1u << (subb * CB::K)) - 1u));
+                    if (!live && slot < nq) {
+                        if (CARRY && slot < np) {
+                            hnd = kPoolTag + slot;
+                            load_lane<NBB>(pool_w + slot * G + klb * CB::EPL, w);
+                            load_state(pool_st, pool_st + CB::SLOTS, slot, g);
+                            gi = pool_gi[slot];
+                        } else {
+                            hnd = s_q[slot - np];
+                            load_lane<NBB>(s_w + hnd * G + klb * CB::EPL, w);
+                            load_state(s_st, s_st2, hnd, g);
+                            gi = chunk * C::CG + hnd;
+                        }
                         live = true;
                     }
-                    head = min(qn, head + __popc(want));
+                    head = min(nq, head + __popc(want));
                 }
-                if (!__any_sync(kFull, live)) break;
-                const bool fin = solver_step<NBITS, G, NB>(S, prm, w, g, live, pa1, pa2, pa3,
-                                                           qa1, qa2, qa3);
-                if (__any_sync(kFull, fin)) {
-                    if (fin) finalize<NBITS, G, NB>(prm, w, g, chunk, gl, kl, s_codes);
+                const unsigned lmask = __ballot_sync(kFull, live && leadb);
+                if (lmask == 0) break;
+                if (more && head >= nq && 4 * __popc(lmask) <= PARK * CB::SLOTS) {
+                    // park the busy groups (the pool's old entries are all taken)
+                    __syncwarp();
+                    if (live) {
+                        const int j = __popc(lmask & ((1u << (subb * CB::K)) - 1u));
+                        store_lane<NBB>(pool_w + j * G + klb * CB::EPL, w);
+                        if (leadb) {
+                            save_state(pool_st, pool_st + CB::SLOTS, j, g);
+                            pool_gi[j] = gi;
+                            if (hnd < kPoolTag)          // exclude it from the chunk pass
+                                s_st2[hnd].w = __int_as_float(__float_as_int(s_st2[hnd].w) |
+                                                              kCarried);
+                        }
+                    }
+                    parked = __popc(lmask);
+                    break;
+                }
+                const bool fin = solver_step<NBITS, G, NBB>(S, prm, w, g, live, pa1, pa2, pa3,
+                                                            qa1, qa2, qa3);
+                if (fin) {
+                    if (!CARRY || hnd < kPoolTag) {
+                        if (leadb) save_state(s_st, s_st2, hnd, g);
+                    } else {
+                        finalize_direct<NBITS, G, NBB>(prm, w, g, gi, klb);
+                    }
                 }
                 live = live && !fin;
             }
+            np = parked;
         }
 
-        // ---- 3-bit: whole words of this chunk from the staged codes ------------
+        // ---- final codes of the whole chunk, then 3-bit words -------------------
+        __syncwarp();
+        final_pass<NBITS, G, NB>(prm, s_w, s_st, s_st2, chunk, cg, lane);
         if constexpr (NBITS == 3) {
+            uint8_t* s_codes = reinterpret_cast<uint8_t*>(s_w);
             __syncwarp();
             const int n_words = (n_here + 9) / 10;
             if (lane < n_words * 10 - n_here) s_codes[n_here + lane] = 0;   // zero padding
@@ -445,35 +641,41 @@ quantize_kernel(const __grid_constant__ QuantParams prm) {
     }
 }
 
-template <int NBITS, int G, int NB>
+template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK>
 static cudaError_t launch_quantize_g(const QuantParams& prm, cudaStream_t stream) {
     using C = QCfg<NBITS, G, NB>;
-    auto kern = quantize_kernel<NBITS, G, NB>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    using CB = QCfg<NBITS, G, NBB>;
+    constexpr int SMEM = kQWarps * (C::CHUNK_BYTES + (CARRY ? CB::POOL_BYTES : 0));
+    auto kern = quantize_kernel<NBITS, G, NB, NBB, CARRY, PARK>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (err != cudaSuccess) return err;
     int dev = 0, sms = 148, per_sm = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQWarps * 32, C::SMEM);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQWarps * 32, SMEM);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) per_sm = 1;
     const int64_t n_chunks = (prm.n_elems + kChunk - 1) / kChunk;
     const int64_t want = (n_chunks + kQWarps - 1) / kQWarps;
     const int64_t cap = (int64_t)sms * per_sm;
     const unsigned grid = (unsigned)(want < cap ? want : cap);
-    kern<<<grid, kQWarps * 32, C::SMEM, stream>>>(prm);
+    kern<<<grid, kQWarps * 32, SMEM, stream>>>(prm);
     return cudaGetLastError();
 }
 
-// Weights per lane: 16 (two 8-weight blocks) for every group size.
+// 16 weights per lane in both phases.  4 bit: park the last busy groups of a
+// chunk once at most half the slots are busy (measured faster); 3 and 2 bit:
+// drain each chunk (measured faster: their carried groups cost more to
+// finalise one by one than the idle slots they save).
 template <int NBITS>
 static cudaError_t launch_quantize_b(const QuantParams& prm, int group, cudaStream_t stream) {
+    constexpr bool carry = NBITS == 4;
     switch (group) {
-        case 16: return launch_quantize_g<NBITS, 16, 2>(prm, stream);
-        case 32: return launch_quantize_g<NBITS, 32, 2>(prm, stream);
-        case 64: return launch_quantize_g<NBITS, 64, 2>(prm, stream);
-        case 128: return launch_quantize_g<NBITS, 128, 2>(prm, stream);
-        case 256: return launch_quantize_g<NBITS, 256, 2>(prm, stream);
+        case 16: return launch_quantize_g<NBITS, 16, 2, 2, carry, 2>(prm, stream);
+        case 32: return launch_quantize_g<NBITS, 32, 2, 2, carry, 2>(prm, stream);
+        case 64: return launch_quantize_g<NBITS, 64, 2, 2, carry, 2>(prm, stream);
+        case 128: return launch_quantize_g<NBITS, 128, 2, 2, carry, 2>(prm, stream);
+        case 256: return launch_quantize_g<NBITS, 256, 2, 2, carry, 2>(prm, stream);
         default: return cudaErrorInvalidValue;
     }
 }
