@@ -235,14 +235,20 @@ __device__ __forceinline__ bool solver_step(const QuantSmem& S, const QuantParam
         r = eval_lane<C::L, NB, true, false>(S, w, c, pa1, pa2, pa3, qa1, qa2, qa3, beta);
     r = group_sum2<C::K>(r);                       // (error, sp2 sum) of the whole group
     const bool acc = live && r.x < g.eb;
+    bool repeat = false;
     if (acc) {
+        const float zn = __fmul_rn(r.y, 1.0f / (float)G);
+        // the update reproduced the z just evaluated: the next evaluation would
+        // repeat this one exactly, its error would not fall, and the group would
+        // stop with the same best z -- so it stops now (identical outputs)
+        repeat = zn == g.z;
         g.eb = r.x;
         g.zb = g.z;
-        g.z = __fmul_rn(r.y, 1.0f / (float)G);
+        g.z = zn;
         ++g.na;
     }
     if (live) ++g.t;
-    return live && (!acc || g.t == prm.iters);
+    return live && (!acc || repeat || g.t == prm.iters);
 }
 
 // Group state kept in the chunk's shared memory between phases.
