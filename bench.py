@@ -462,6 +462,11 @@ def run_gpu(args):
         line["cpu_baseline"] = {"value": n / dt / 1e9, "unit": "Gparam/s", "cores": cores,
                                 "kind": "oracle", "sample": desc + f"; {n} params, {dt:.1f} s"}
 
+    # ---- model-shaped sets: one streamed pass, each layer's weights generated
+    # on the device into one reused buffer and then quantized (wall time)
+    if args.workload in ("llama2-70b", "llama2-7b") and not args.no_stream:
+        line["stream_pass"] = run_stream_pass(mats, hqq, dev, views)
+
     # ---- end to end through the public API with host buffers
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, mats, views, hqq, dev, pg, ws)
@@ -473,6 +478,29 @@ def run_gpu(args):
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def run_stream_pass(mats, hqq, dev, views):
+    """Generate + quantize layer by layer through one reused weight buffer
+    (outputs stay resident); CUDA-event wall time of the whole pass."""
+    import torch
+    import synth
+    maxn = max(r * c for _, (r, c), *_ in mats)
+    buf = torch.empty(maxn, dtype=torch.float16, device=dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record()
+    for k, (lab, (r, c), nb, g, seed, stream) in enumerate(mats):
+        W = buf[:r * c].view(r, c)
+        synth.fill_student_t_(W, seed=seed, stream=stream)
+        q = views[k][1]
+        hqq.hqq_quantize(W, nb, g, packed=q.packed, scale=q.scale, zero=q.zero)
+    t1.record()
+    torch.cuda.synchronize()
+    s = t0.elapsed_time(t1) / 1e3
+    params = sum(r * c for _, (r, c), *_ in mats)
+    return {"what": "per layer: generate fp16 weights on the device, then quantize",
+            "wall_s": s, "gparam_s": params / s / 1e9}
 
 
 def run_e2e(args, mats, views, hqq, dev, pg, ws):
@@ -563,6 +591,7 @@ def main():
     ap.add_argument("--layers", type=int, default=None,
                     help="first N layers only of a model-shaped set (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
+    ap.add_argument("--no-stream", action="store_true", help="skip the streamed generate+quantize pass")
     ap.add_argument("--impl", default="libhqq", choices=["libhqq", "reference"])
     ap.add_argument("--cpu-s", type=float, default=10.0, help="oracle CPU-baseline budget (s)")
     ap.add_argument("--ref-step-s", type=float, default=4.0, help="reference arm seconds per step")
