@@ -99,6 +99,55 @@ __device__ __forceinline__ float2 powp2(const PowSmem& T, float2 a1, float2 a2, 
     return __fmul2_rn(tt, poly);
 }
 
+// Combined table for the hot |x|^p: t2[e*32 + j] = fl(2^(p(e-127)) * c_j^p),
+// exactly the product the method's power forms first, so one lookup replaces
+// two and a multiplication.  Its byte offset comes straight from bits 18..30 of
+// x ((x >> 16) & 0x7FFC); the cell's 1/c_j from bits 18..22 ((x >> 16) & 0x7C).
+struct PowSmem2 {
+    float t2[256 * 32];
+    float ic[32];
+};
+
+// Lane l fills cell l of every exponent row; the row's 2^(pk) is warp-uniform,
+// so each warp reads kernel parameters without per-lane serialisation.
+__device__ __forceinline__ void load_pow_smem2(PowSmem2& dst, const PowTable& t) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const float cj = t.cj_p[lane];
+    for (int e = warp; e < 256; e += nw) dst.t2[e * 32 + lane] = __fmul_rn(t.two_pk[e], cj);
+    if (threadIdx.x < 32) dst.ic[threadIdx.x] = t.inv_cj[threadIdx.x];
+}
+
+// |x|^p of two values (any sign) with the combined table.
+__device__ __forceinline__ float2 powp2c(const PowSmem2& T, float2 a1, float2 a2, float2 a3,
+                                         float2 x) {
+    const uint32_t ux = __float_as_uint(x.x), uy = __float_as_uint(x.y);
+    const uint32_t hx = ux >> 16, hy = uy >> 16;
+    const float2 m = make_float2(__uint_as_float((ux & 0x007FFFFFu) | 0x3F800000u),
+                                 __uint_as_float((uy & 0x007FFFFFu) | 0x3F800000u));
+    const float2 r = __ffma2_rn(m, make_float2(tab_at(T.ic, hx & 0x7Cu), tab_at(T.ic, hy & 0x7Cu)),
+                                make_float2(-1.0f, -1.0f));
+    float2 poly = __ffma2_rn(r, a3, a2);
+    poly = __ffma2_rn(poly, r, a1);
+    poly = __ffma2_rn(poly, r, make_float2(1.0f, 1.0f));
+    return __fmul2_rn(make_float2(tab_at(T.t2, hx & 0x7FFCu), tab_at(T.t2, hy & 0x7FFCu)), poly);
+}
+
+// The hot power for either table layout.
+__device__ __forceinline__ float2 powp_hot(const PowSmem2& T, float2 a1, float2 a2, float2 a3,
+                                           float2 x) {
+    return powp2c(T, a1, a2, a3, x);
+}
+__device__ __forceinline__ float2 powp_hot(const PowSmem& T, float2 a1, float2 a2, float2 a3,
+                                           float2 x) {
+    return powp2(T, a1, a2, a3, x);
+}
+__device__ __forceinline__ void load_pow_hot(PowSmem2& dst, const PowTable& t) {
+    load_pow_smem2(dst, t);
+}
+__device__ __forceinline__ void load_pow_hot(PowSmem& dst, const PowTable& t) {
+    load_pow_smem(dst, t);
+}
+
 // Scalar form (same operations) for the shrink's |x|^(p-1), x >= +0.
 __device__ __forceinline__ float powp1(const PowSmem& T, float a1, float a2, float a3, float x) {
     const uint32_t b = __float_as_uint(x);

@@ -25,11 +25,13 @@
 //    [0, L] (fma is monotone in the weight), so the clamp is skipped; when a
 //    bound on |W - Q^-1(Q(W))| lies below the shrink threshold, W_e is exactly
 //    zero, so sp1 reduces to W - W_e = W.
+#include <type_traits>
+
 #include "hqq_common.cuh"
 
 namespace hqq {
 
-constexpr int kQWarps = 4;                 // warps per CTA
+constexpr int kQWarps = 8;                 // warps per CTA (share the 32 KiB table)
 constexpr int kChunk = 2560;               // weights per warp chunk
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -59,8 +61,11 @@ struct QCfg {
     static_assert(K >= 1 && K <= 32 && kChunk % ROUND == 0, "bad layout");
 };
 
+// TAB2: the hot |x|^p uses the combined 32 KiB exponent x cell table (one
+// lookup fewer); otherwise the separate small tables (less shared memory).
+template <bool TAB2>
 struct QuantSmem {
-    PowSmem tp;                 // |x|^p
+    std::conditional_t<TAB2, PowSmem2, PowSmem> tp;   // |x|^p
     PowSmem tq;                 // |x|^(p-1)
     float beta[kMaxIters + 1];  // beta_t = beta * kappa^t by repeated binary32 products
     float thr[kMaxIters + 1];   // shrink thresholds
@@ -138,8 +143,8 @@ struct EvalConst {
 // lane's pairwise sums of (|r|^p, sp2 term) where r = W - s(Wq - z) and the sp2
 // term is Wq - (W - W_e)/s.  CLAMP: codes may leave [0, L].  SHRINK: W_e is
 // evaluated exactly; otherwise W_e is known to be zero.
-template <int L, int NB, bool CLAMP, bool SHRINK>
-__device__ __forceinline__ float2 eval_lane(const QuantSmem& S, const float2 (&w)[NB][4],
+template <int L, int NB, bool CLAMP, bool SHRINK, class SM>
+__device__ __forceinline__ float2 eval_lane(const SM& S, const float2 (&w)[NB][4],
                                             const EvalConst& c, float2 pa1, float2 pa2,
                                             float2 pa3, float qa1, float qa2, float qa3,
                                             float beta) {
@@ -159,7 +164,7 @@ __device__ __forceinline__ float2 eval_lane(const QuantSmem& S, const float2 (&w
             const float2 q = __fadd2_rn(__fadd2_rn(v, sh), nsh);      // round half even
             const float2 qz = __fadd2_rn(q, c.nz);                     // Wq - z
             const float2 d = __ffma2_rn(qz, c.ns, w[b][k]);            // W - s(Wq - z)
-            P[k] = powp2(S.tp, pa1, pa2, pa3, d);
+            P[k] = powp_hot(S.tp, pa1, pa2, pa3, d);
             if (SHRINK) {
                 float we[2];
                 const float dd[2] = {d.x, d.y};
@@ -204,8 +209,8 @@ struct GroupState {
 // One solver iteration (error evaluation, early-stop test, sp1 + sp2) for the
 // sub-warp's group; `live` lanes only change state.  Returns true when the
 // group has finished (stopped, or used its iterations).
-template <int NBITS, int G, int NB>
-__device__ __forceinline__ bool solver_step(const QuantSmem& S, const QuantParams& prm,
+template <int NBITS, int G, int NB, class SM>
+__device__ __forceinline__ bool solver_step(const SM& S, const QuantParams& prm,
                                             const float2 (&w)[NB][4], GroupState& g, bool live,
                                             float2 pa1, float2 pa2, float2 pa3,
                                             float qa1, float qa2, float qa3) {
@@ -432,16 +437,18 @@ __device__ __forceinline__ void final_pass(const QuantParams& prm, __half* s_w, 
 
 // NB / NBB: 8-weight blocks per lane in phase A / phase B.  CARRY: park the
 // last busy groups of a chunk and resume them with the next chunk, parking
-// once at most PARK/4 of the phase-B slots are busy.
-template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK>
-__global__ void __launch_bounds__(kQWarps * 32, 5)
+// once at most PARK/4 of the phase-B slots are busy.  TAB2: combined power
+// table (off for G = 16, whose per-group state already fills the shared memory
+// that two resident CTAs per SM can have).
+template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK, bool TAB2>
+__global__ void __launch_bounds__(kQWarps * 32, 2)
 quantize_kernel(const __grid_constant__ QuantParams prm) {
     using C = QCfg<NBITS, G, NB>;      // phase A layout (and the chunk's shared memory)
     using CB = QCfg<NBITS, G, NBB>;    // phase B layout
-    __shared__ QuantSmem S;
+    __shared__ QuantSmem<TAB2> S;
     extern __shared__ __align__(16) uint8_t dyn[];
 
-    load_pow_smem(S.tp, prm.tp);
+    load_pow_hot(S.tp, prm.tp);
     load_pow_smem(S.tq, prm.tq);
     for (int i = threadIdx.x; i < prm.iters; i += blockDim.x) S.thr[i] = prm.shrink_thr[i];
     if (threadIdx.x == 0) {
@@ -647,12 +654,12 @@ quantize_kernel(const __grid_constant__ QuantParams prm) {
     }
 }
 
-template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK>
+template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK, bool TAB2 = (G > 16)>
 static cudaError_t launch_quantize_g(const QuantParams& prm, cudaStream_t stream) {
     using C = QCfg<NBITS, G, NB>;
     using CB = QCfg<NBITS, G, NBB>;
     constexpr int SMEM = kQWarps * (C::CHUNK_BYTES + (CARRY ? CB::POOL_BYTES : 0));
-    auto kern = quantize_kernel<NBITS, G, NB, NBB, CARRY, PARK>;
+    auto kern = quantize_kernel<NBITS, G, NB, NBB, CARRY, PARK, TAB2>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (err != cudaSuccess) return err;
     int dev = 0, sms = 148, per_sm = 1;
