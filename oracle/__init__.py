@@ -65,6 +65,10 @@ def _load():
             lib.hqq_oracle_dequantize.restype = I
             lib.hqq_oracle_f32_to_f16.argtypes = [P, I64, P]
             lib.hqq_oracle_f32_to_f16.restype = None
+            lib.hqq_oracle_meta_quantize.argtypes = [P, I64, I64, P, P, P]
+            lib.hqq_oracle_meta_quantize.restype = I
+            lib.hqq_oracle_meta_dequantize.argtypes = [P, P, P, I64, I64, P]
+            lib.hqq_oracle_meta_dequantize.restype = I
             _lib = lib
     return _lib
 
@@ -217,6 +221,61 @@ def dequantize(codes, scale, zero, group: int) -> np.ndarray:
     if st:
         raise ValueError(f"dequantize failed (status {st})")
     return out.view(np.float16)
+
+
+def meta_groups(n: int, group: int) -> int:
+    """Number of groups of an n-value meta tensor (group 0: one group)."""
+    if n == 0:
+        return 0
+    return 1 if group == 0 else -(-n // group)
+
+
+def meta_quantize(x, group: int) -> dict:
+    """8-bit min-max round-to-nearest of an fp16 vector (zero points or scales),
+    groups of ``group`` consecutive values (ragged last group; 0 = one group).
+    Returns uint8 codes and the fp16 scale and zero of every group."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float16).reshape(-1)
+    ng = meta_groups(x.size, group)
+    codes = np.empty(x.size, np.uint8)
+    scale = np.empty(ng, np.uint16)
+    zero = np.empty(ng, np.uint16)
+    st = lib.hqq_oracle_meta_quantize(_ptr(x.view(np.uint16)), x.size, group, _ptr(codes),
+                                      _ptr(scale), _ptr(zero))
+    if st:
+        raise ValueError(f"meta_quantize rejected the arguments (status {st})")
+    return dict(codes=codes, scale=scale.view(np.float16), zero=zero.view(np.float16))
+
+
+def meta_dequantize(codes, scale, zero, group: int) -> np.ndarray:
+    """fp16((c - z) * s) of 8-bit meta codes with their groups' fp16 s and z."""
+    lib = _load()
+    codes = np.ascontiguousarray(codes, dtype=np.uint8).reshape(-1)
+    scale = np.ascontiguousarray(scale, dtype=np.float16).reshape(-1)
+    zero = np.ascontiguousarray(zero, dtype=np.float16).reshape(-1)
+    out = np.empty(codes.size, np.uint16)
+    st = lib.hqq_oracle_meta_dequantize(_ptr(codes), _ptr(scale.view(np.uint16)),
+                                        _ptr(zero.view(np.uint16)), codes.size, group,
+                                        _ptr(out))
+    if st:
+        raise ValueError(f"meta_dequantize rejected the arguments (status {st})")
+    return out.view(np.float16)
+
+
+def dequantize_meta(codes, group: int, zero_q: dict, zero_group: int = 0,
+                    scale=None, scale_q: dict | None = None,
+                    scale_group: int = 128) -> np.ndarray:
+    """Weights from codes whose zero points (and optionally scales) are stored
+    8-bit: the zero points and scales are first restored to fp16 by
+    ``meta_dequantize``, then ``dequantize`` runs as usual.  Exactly one of
+    ``scale`` (fp16 per group) and ``scale_q`` (a ``meta_quantize`` result) is
+    given."""
+    z = meta_dequantize(zero_q["codes"], zero_q["scale"], zero_q["zero"], zero_group)
+    if (scale is None) == (scale_q is None):
+        raise ValueError("give exactly one of scale and scale_q")
+    s = scale if scale_q is None else meta_dequantize(
+        scale_q["codes"], scale_q["scale"], scale_q["zero"], scale_group)
+    return dequantize(codes, s, z, group)
 
 
 def f32_to_f16(x) -> np.ndarray:

@@ -444,3 +444,63 @@ int hqq_oracle_dequantize(const uint8_t *codes, const uint16_t *scale,
 void hqq_oracle_f32_to_f16(const float *x, int64_t n, uint16_t *h) {
     for (int64_t i = 0; i < n; ++i) h[i] = float_to_half_bits(x[i]);
 }
+
+/* ------------------------------------------------------------------------- */
+/* 8-bit meta-quantization of the stored zero points and scales              */
+/* ------------------------------------------------------------------------- */
+/* Section 4.1 ("Llama-2 benchmarks") of the page quantizes the zero points to
+   8 bits with neither grouping nor optimisation, and in its table's starred
+   row also the scales, to 8 bits in groups of 128.  Readings taken:
+     - "without optimisation" is section 2's Q with its min-max start and no
+       solver iterations: s = (max-min)/255 (s = 1 for a constant group),
+       1/s held, z = -min * (1/s), c = clamp(round(x * (1/s) + z), 0, 255);
+     - the input is the stored fp16 tensor in flat row-major order; groups are
+       `group` consecutive values and the last one may be shorter; group 0
+       means one group over all n values ("without grouping");
+     - each group's own scale and zero are stored in fp16 like the weights';
+     - the arithmetic is the weights' canonical binary32 sequence. */
+int hqq_oracle_meta_quantize(const uint16_t *x, int64_t n, int64_t group,
+                             uint8_t *codes, uint16_t *scale, uint16_t *zero) {
+    if (n < 0 || group < 0) return 3;
+    const float L = 255.0f;
+    const int64_t len = group == 0 ? n : group;
+    for (int64_t g0 = 0, gi = 0; g0 < n; g0 += len, ++gi) {
+        const int64_t m = n - g0 < len ? n - g0 : len;
+        float mn = half_bits_to_float(x[g0]), mx = mn;
+        for (int64_t i = 1; i < m; ++i) {
+            const float v = half_bits_to_float(x[g0 + i]);
+            if (v < mn) mn = v;
+            if (v > mx) mx = v;
+        }
+        const float rng = mx - mn;
+        float s, inv;
+        if (rng == 0.0f) {
+            s = 1.0f;
+            inv = 1.0f;
+        } else {
+            s = rng / L;
+            inv = 1.0f / s;
+        }
+        const float z = -(mn * inv);
+        for (int64_t i = 0; i < m; ++i)
+            codes[g0 + i] = (uint8_t)clamp_code(fmaf(half_bits_to_float(x[g0 + i]), inv, z), L);
+        scale[gi] = float_to_half_bits(s);
+        zero[gi] = float_to_half_bits(z);
+    }
+    return 0;
+}
+
+/* Its inverse, section 2's Q^-1 on the 8-bit codes: fp16((c - z) * s) with the
+   group's stored fp16 s and z (group 0: one group over all n values). */
+int hqq_oracle_meta_dequantize(const uint8_t *codes, const uint16_t *scale,
+                               const uint16_t *zero, int64_t n, int64_t group,
+                               uint16_t *out) {
+    if (n < 0 || group < 0) return 3;
+    const int64_t len = group == 0 ? (n > 0 ? n : 1) : group;
+    for (int64_t i = 0; i < n; ++i) {
+        const float s = half_bits_to_float(scale[i / len]);
+        const float z = half_bits_to_float(zero[i / len]);
+        out[i] = float_to_half_bits(((float)codes[i] - z) * s);
+    }
+    return 0;
+}

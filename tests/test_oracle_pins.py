@@ -375,3 +375,109 @@ def test_dequantize_definition():
     ref = ((codes.astype(np.float32) - np.repeat(zero.astype(np.float32), G))
            * np.repeat(scale.astype(np.float32), G)).astype(np.float16)
     assert np.array_equal(got.view(np.uint16), ref.view(np.uint16))
+
+
+# ------------------------------------------------------------ 8-bit meta data
+def _meta_inputs(seed):
+    """Realistic zero points and scales: those of HQQ-quantized synthetic weights."""
+    W = synth.student_t_host((192, 1024), seed=seed, stream=11).astype(np.float16)
+    r = oracle.quantize(W, 3, 64, iters=4)
+    return r["zero"].copy(), r["scale"].copy()
+
+
+@pytest.mark.parametrize("which", ["zero", "scale"])
+@pytest.mark.parametrize("group", [0, 128, 100])
+def test_meta_quantize_is_8bit_minmax_rtn(which, group):
+    """Section 4.1 stores the zero points (no grouping) and, in the table's
+    starred row, the scales (groups of 128) in 8 bits; with no optimisation this
+    is textbook min-max round-to-nearest with 255 levels, checked here in fp64
+    (ragged last group when 128 or 100 does not divide the length)."""
+    zero, scale = _meta_inputs(21)
+    x = (zero if which == "zero" else scale)[:700]
+    r = oracle.meta_quantize(x, group)
+    n = x.size
+    ln = n if group == 0 else group
+    xd = x.astype(np.float64)
+    for gi, g0 in enumerate(range(0, n, ln)):
+        seg = xd[g0:g0 + ln]
+        mn, mx = seg.min(), seg.max()
+        s = (mx - mn) / 255.0
+        z = -mn / s
+        u = seg / s + z
+        codes = np.clip(np.rint(u), 0, 255)
+        tie = np.abs(np.abs(u - np.floor(u)) - 0.5) < 1e-4
+        got = r["codes"][g0:g0 + ln]
+        assert np.all((got == codes) | tie), gi
+        assert got.min() == 0 and got.max() == 255
+        # stored fp16 values: the fp64 ones rounded to fp16 (one fp16 ulp slack
+        # for the fp32 intermediate)
+        for stored, exact in ((r["scale"][gi], s), (r["zero"][gi], z)):
+            ref = np.float16(exact)
+            ulp = np.spacing(np.abs(ref)).astype(np.float64)
+            assert abs(float(stored) - exact) <= float(ulp), (gi, stored, exact)
+    assert r["scale"].size == oracle.meta_groups(n, group)
+
+
+def test_meta_group_semantics():
+    """Group 0 is one group over the whole tensor; groups are independent runs
+    of consecutive values, the last one shorter."""
+    zero, _ = _meta_inputs(22)
+    x = zero[:1000]
+    a = oracle.meta_quantize(x, 0)
+    b = oracle.meta_quantize(x, 1000)
+    assert all(np.array_equal(a[k].view(np.uint8), b[k].view(np.uint8)) for k in a)
+    c = oracle.meta_quantize(x, 128)
+    for gi, g0 in enumerate(range(0, 1000, 128)):
+        d = oracle.meta_quantize(x[g0:g0 + 128], 0)
+        assert np.array_equal(c["codes"][g0:g0 + 128], d["codes"])
+        assert c["scale"][gi] == d["scale"][0] and c["zero"][gi] == d["zero"][0]
+
+
+def test_meta_constant_and_degenerate_groups():
+    """A constant group has one level (s = 1) and restores exactly; an empty
+    tensor has no groups."""
+    vals = np.array([0.0, 3.5, -0.25, 7.0, 6e-8, 1000.0], np.float16)
+    x = np.repeat(vals, 128)
+    r = oracle.meta_quantize(x, 128)
+    assert np.all(r["scale"] == 1.0) and np.all(r["codes"] == 0)
+    y = oracle.meta_dequantize(r["codes"], r["scale"], r["zero"], 128)
+    assert np.array_equal(y.astype(np.float32), x.astype(np.float32))
+    e = oracle.meta_quantize(np.zeros(0, np.float16), 0)
+    assert e["codes"].size == 0 and e["scale"].size == 0
+
+
+def test_meta_dequantize_and_composition_definition():
+    """Q^-1 on 8-bit codes is fp16((c - z) s) with the group's fp16 s and z
+    (numpy fp32 here); weights with 8-bit zero points (and scales) are restored
+    by restoring the zero points (and scales) first, then Q^-1 as usual."""
+    zero, scale = _meta_inputs(23)
+    zq = oracle.meta_quantize(zero, 0)
+    sq = oracle.meta_quantize(scale, 128)
+    n = zero.size
+    zr = ((zq["codes"].astype(np.float32) - np.float32(zq["zero"][0]))
+          * np.float32(zq["scale"][0])).astype(np.float16)
+    got = oracle.meta_dequantize(zq["codes"], zq["scale"], zq["zero"], 0)
+    assert np.array_equal(got.view(np.uint16), zr.view(np.uint16))
+    gidx = np.arange(n) // 128
+    sr = ((sq["codes"].astype(np.float32) - sq["zero"].astype(np.float32)[gidx])
+          * sq["scale"].astype(np.float32)[gidx]).astype(np.float16)
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 8, n * 64).astype(np.uint8)
+    w1 = oracle.dequantize_meta(codes, 64, zq, 0, scale=scale)
+    assert np.array_equal(w1.view(np.uint16), oracle.dequantize(codes, scale, zr, 64).view(np.uint16))
+    w2 = oracle.dequantize_meta(codes, 64, zq, 0, scale_q=sq, scale_group=128)
+    assert np.array_equal(w2.view(np.uint16), oracle.dequantize(codes, sr, zr, 64).view(np.uint16))
+
+
+def test_meta_zero_error_is_small_against_the_code_step():
+    """8 bits for the zero points of a 3-bit matrix cost little: every restored
+    zero point lies within half a step of the 8-bit grid of the stored fp16 s and
+    z (plus the fp16 rounding of the result) of its original."""
+    zero, _ = _meta_inputs(24)
+    zq = oracle.meta_quantize(zero, 0)
+    zr = oracle.meta_dequantize(zq["codes"], zq["scale"], zq["zero"], 0).astype(np.float64)
+    s16 = float(zq["scale"][0])
+    rng_ = float(zero.astype(np.float64).max() - zero.astype(np.float64).min())
+    bound = s16 / 2 + 255 * abs(s16 - rng_ / 255) + abs(float(zq["zero"][0]) - float(
+        -zero.astype(np.float64).min() / (rng_ / 255))) * s16 + np.spacing(np.float16(8.0))
+    assert np.max(np.abs(zr - zero.astype(np.float64))) <= bound
