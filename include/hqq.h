@@ -127,6 +127,80 @@ int hqq_dequantize(const void* packed, const void* scale, const void* zero,
                    int64_t rows, int64_t cols, int nbits, int group,
                    void* W_out, void* stream);
 
+/*
+ * 8-bit storage of the per-group zero points and scales (the method's section
+ * 4.1: its settings keep the zero points in 8 bits, with neither grouping nor
+ * optimisation; the starred row of its table also keeps the scales in 8 bits,
+ * in groups of 128).
+ *
+ * A meta tensor is an fp16 vector x of n values -- a matrix's zero or scale
+ * output of hqq_quantize, in flat row-major order.  It is cut into groups of
+ * `mgroup` consecutive values (the last group may be shorter); mgroup = 0 means
+ * one group over all n values.  mgroup is 0 or a power of two 1 .. 2^30.  Each
+ * group is min-max round-to-nearest quantized with 255 levels, in binary32:
+ *   s = (max - min) / 255 and 1/s (s = 1/s = 1 when max == min);
+ *   z = -min * (1/s);  c = clamp(round(x * (1/s) + z), 0, 255), half to even;
+ * and its s and z are stored in fp16.  The inverse restores
+ *   x' = fp16( (c - z) * s )  with the group's stored fp16 s and z.
+ */
+
+/* Second-level groups of an n-value meta tensor: 0 when n == 0, 1 when
+   mgroup == 0, else ceil(n / mgroup); -1 for negative arguments. */
+int64_t hqq_meta_groups(int64_t n, int64_t mgroup);
+
+/*
+ * hqq_meta_quantize -- 8-bit codes of a meta tensor.
+ *   x      [in]  fp16 [n], 16-byte aligned.
+ *   n      [in]  number of values (>= 0; n == 0 is a valid no-op).
+ *   mgroup [in]  0 or a power of two up to 2^30 (else HQQ_ERR_UNSUPPORTED).
+ *   codes  [out] uint8 [n], 8-byte aligned.
+ *   scale, zero [out] fp16 [hqq_meta_groups(n, mgroup)], 2-byte aligned.
+ *   stream [in]  cudaStream_t (NULL = legacy default stream).
+ * With mgroup = 0 (or one group covering all n values) the whole tensor is
+ * reduced by one cluster of thread blocks; that form is meant for the meta
+ * tensor of one matrix (millions of values), not for billions.
+ */
+int hqq_meta_quantize(const void* x, int64_t n, int64_t mgroup, uint8_t* codes,
+                      void* scale, void* zero, void* stream);
+
+/*
+ * hqq_meta_dequantize -- the inverse: out = fp16((c - z) * s) per value.
+ *   codes [in] uint8 [n], 8-byte aligned.   scale, zero [in] fp16, 2-byte aligned.
+ *   n, mgroup [in] as for hqq_meta_quantize.   out [out] fp16 [n], 16-byte aligned.
+ */
+int hqq_meta_dequantize(const uint8_t* codes, const void* scale, const void* zero,
+                        int64_t n, int64_t mgroup, void* out, void* stream);
+
+/* The 8-bit form of one meta tensor, as hqq_meta_quantize writes it (device
+   pointers; the struct itself lives in host memory). */
+typedef struct hqq_meta8 {
+    const uint8_t* codes;   /* uint8 [n]                                   */
+    const void* scale;      /* fp16 [hqq_meta_groups(n, group)]            */
+    const void* zero;       /* fp16 [hqq_meta_groups(n, group)]            */
+    int64_t group;          /* 0 or a power of two, as mgroup above         */
+} hqq_meta8;
+
+/*
+ * hqq_dequantize_meta -- hqq_dequantize for a matrix whose zero points (and,
+ * optionally, scales) are kept in their 8-bit form: each group's zero point is
+ * restored first, z' = fp16((c_z - z_z) * s_z), the scale likewise when scale_q
+ * is given, and then W_hat = fp16((code - z') * s') exactly as hqq_dequantize
+ * does.  The result equals hqq_meta_dequantize of the zero points (and scales)
+ * followed by hqq_dequantize, bit for bit, in one pass.
+ *   packed  [in]  codes, as for hqq_dequantize.
+ *   zero_q  [in]  HOST pointer to the zero points' 8-bit form (required; its
+ *                 codes hold rows*cols/group values).
+ *   scale   [in]  fp16 [rows, cols/group] scales, or NULL when scale_q is given.
+ *   scale_q [in]  HOST pointer to the scales' 8-bit form, or NULL.
+ *                 Exactly one of scale and scale_q must be non-NULL.
+ *   rows, cols, nbits, group, W_out, stream [in/out] as for hqq_dequantize.
+ * Alignment: packed 4 bytes, zero_q/scale_q codes 1, their fp16 arrays and
+ * scale 2, W_out 16.
+ */
+int hqq_dequantize_meta(const void* packed, const hqq_meta8* zero_q, const void* scale,
+                        const hqq_meta8* scale_q, int64_t rows, int64_t cols, int nbits,
+                        int group, void* W_out, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* hqq_status_string(int status);
 

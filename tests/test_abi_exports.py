@@ -100,3 +100,45 @@ def test_host_validation_without_gpu(lib):
     assert L.hqq_dequantize(P(256), P(256), None, 64, 256, 4, 64, P(256), None) == 1
     assert L.hqq_dequantize(P(256), P(256), P(256), 64, 256, 4, 64, P(264), None) == 5
     assert L.hqq_dequantize(P(256), P(256), P(256), 64, 100, 4, 64, P(256), None) == 2
+
+
+def test_meta_host_validation_without_gpu(lib):
+    L = lib._lib
+    P = lambda v: ctypes.c_void_p(v)
+    assert lib.hqq_meta_groups(0, 128) == 0
+    assert lib.hqq_meta_groups(1000, 0) == 1
+    assert lib.hqq_meta_groups(1000, 128) == 8
+    assert L.hqq_meta_groups(-1, 0) == -1
+    # quantize: shape, group, null, alignment; n == 0 is a no-op
+    assert L.hqq_meta_quantize(P(256), -1, 0, P(256), P(256), P(256), None) == 2
+    assert L.hqq_meta_quantize(P(256), 100, 100, P(256), P(256), P(256), None) == 3
+    assert L.hqq_meta_quantize(P(256), 100, 1 << 31, P(256), P(256), P(256), None) == 3
+    assert L.hqq_meta_quantize(None, 100, 0, P(256), P(256), P(256), None) == 1
+    assert L.hqq_meta_quantize(P(258), 100, 0, P(256), P(256), P(256), None) == 5
+    assert L.hqq_meta_quantize(P(256), 100, 0, P(260), P(256), P(256), None) == 5
+    assert L.hqq_meta_quantize(P(256), 100, 128, P(256), P(257), P(256), None) == 5
+    assert L.hqq_meta_quantize(None, 0, 0, None, None, None, None) == 0
+    # dequantize
+    assert L.hqq_meta_dequantize(P(256), P(256), P(256), 100, 3, P(256), None) == 3
+    assert L.hqq_meta_dequantize(P(256), None, P(256), 100, 0, P(256), None) == 1
+    assert L.hqq_meta_dequantize(P(256), P(256), P(256), 100, 0, P(264), None) == 5
+    assert L.hqq_meta_dequantize(None, None, None, 0, 0, None, None) == 0
+    # fused weight dequantize with 8-bit meta data
+    M = lib._CMeta8
+    good = M(256, 256, 256, 0)
+    bad_group = M(256, 256, 256, 96)
+    no_codes = M(None, 256, 256, 0)
+    r = ctypes.byref
+    assert L.hqq_dequantize_meta(P(256), r(good), P(256), r(good), 64, 256, 4, 64, P(256),
+                                 None) == 4
+    assert L.hqq_dequantize_meta(P(256), r(good), None, None, 64, 256, 4, 64, P(256), None) == 1
+    assert L.hqq_dequantize_meta(P(256), None, P(256), None, 64, 256, 4, 64, P(256), None) == 1
+    assert L.hqq_dequantize_meta(P(256), r(no_codes), P(256), None, 64, 256, 4, 64, P(256),
+                                 None) == 1
+    assert L.hqq_dequantize_meta(P(256), r(bad_group), P(256), None, 64, 256, 4, 64, P(256),
+                                 None) == 3
+    assert L.hqq_dequantize_meta(P(256), r(good), P(256), None, 64, 256, 4, 64, P(260),
+                                 None) == 5
+    assert L.hqq_dequantize_meta(P(256), r(good), P(256), None, 64, 256, 5, 64, P(256),
+                                 None) == 3
+    assert L.hqq_dequantize_meta(None, None, None, None, 0, 256, 4, 64, None, None) == 0

@@ -14,6 +14,8 @@ from dataclasses import dataclass
 
 __all__ = ["HQQError", "hqq_quantize", "hqq_quantize_ex", "hqq_dequantize",
            "hqq_packed_bytes", "hqq_status_string", "QuantizedMatrix", "LIB_PATH",
+           "Meta8", "hqq_meta_groups", "hqq_meta_quantize", "hqq_meta_dequantize",
+           "hqq_dequantize_meta",
            "DEFAULT_P", "DEFAULT_BETA", "DEFAULT_KAPPA", "DEFAULT_ITERS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -38,6 +40,22 @@ _lib.hqq_quantize_ex.argtypes = [_P, _I64, _I64, _I, _I, _F, _F, _F, _I, _P, _P,
 _lib.hqq_quantize_ex.restype = _I
 _lib.hqq_dequantize.argtypes = [_P, _P, _P, _I64, _I64, _I, _I, _P, _P]
 _lib.hqq_dequantize.restype = _I
+_lib.hqq_meta_groups.argtypes = [_I64, _I64]
+_lib.hqq_meta_groups.restype = _I64
+_lib.hqq_meta_quantize.argtypes = [_P, _I64, _I64, _P, _P, _P, _P]
+_lib.hqq_meta_quantize.restype = _I
+_lib.hqq_meta_dequantize.argtypes = [_P, _P, _P, _I64, _I64, _P, _P]
+_lib.hqq_meta_dequantize.restype = _I
+
+
+class _CMeta8(ctypes.Structure):
+    """struct hqq_meta8 of include/hqq.h."""
+    _fields_ = [("codes", _P), ("scale", _P), ("zero", _P), ("group", _I64)]
+
+
+_lib.hqq_dequantize_meta.argtypes = [_P, ctypes.POINTER(_CMeta8), _P, ctypes.POINTER(_CMeta8),
+                                     _I64, _I64, _I, _I, _P, _P]
+_lib.hqq_dequantize_meta.restype = _I
 
 
 class HQQError(RuntimeError):
@@ -161,4 +179,77 @@ def hqq_dequantize(q: QuantizedMatrix, out=None, stream=None):
         out = torch.empty((q.rows, q.cols), dtype=torch.float16, device=q.packed.device)
     _check(_lib.hqq_dequantize(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols,
                                q.nbits, q.group, _ptr(out), _stream(stream)))
+    return out
+
+
+@dataclass
+class Meta8:
+    """8-bit form of a meta tensor (a matrix's zero points or scales)."""
+    codes: "torch.Tensor"      # uint8 [n]
+    scale: "torch.Tensor"      # fp16 [hqq_meta_groups(n, group)]
+    zero: "torch.Tensor"       # fp16 [hqq_meta_groups(n, group)]
+    group: int                 # 0 (one group) or a power of two
+
+    def _c(self):
+        return _CMeta8(self.codes.data_ptr(), self.scale.data_ptr(), self.zero.data_ptr(),
+                       self.group)
+
+
+def hqq_meta_groups(n: int, mgroup: int) -> int:
+    g = _lib.hqq_meta_groups(n, mgroup)
+    if g < 0:
+        raise HQQError(2)
+    return int(g)
+
+
+def hqq_meta_quantize(x, mgroup: int = 0, codes=None, scale=None, zero=None,
+                      stream=None) -> Meta8:
+    """8-bit min-max round-to-nearest of an fp16 meta tensor (flat order;
+    ``mgroup`` consecutive values per group, 0 = one group); see include/hqq.h."""
+    import torch
+    if x.dtype != torch.float16:
+        raise ValueError("x must be float16")
+    _check_tensor(x, "x")
+    n = x.numel()
+    ng = hqq_meta_groups(n, mgroup)
+    if codes is None:
+        codes = torch.empty(n, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty(ng, dtype=torch.float16, device=x.device)
+    if zero is None:
+        zero = torch.empty(ng, dtype=torch.float16, device=x.device)
+    for t, nm in ((codes, "codes"), (scale, "scale"), (zero, "zero")):
+        _check_tensor(t, nm)
+    _check(_lib.hqq_meta_quantize(_ptr(x), n, mgroup, _ptr(codes), _ptr(scale), _ptr(zero),
+                                  _stream(stream)))
+    return Meta8(codes, scale, zero, mgroup)
+
+
+def hqq_meta_dequantize(m: Meta8, out=None, stream=None):
+    """fp16 [n] = (code - zero) * scale per value of an 8-bit meta tensor."""
+    import torch
+    for t, nm in ((m.codes, "codes"), (m.scale, "scale"), (m.zero, "zero"), (out, "out")):
+        _check_tensor(t, nm)
+    n = m.codes.numel()
+    if out is None:
+        out = torch.empty(n, dtype=torch.float16, device=m.codes.device)
+    _check(_lib.hqq_meta_dequantize(_ptr(m.codes), _ptr(m.scale), _ptr(m.zero), n, m.group,
+                                    _ptr(out), _stream(stream)))
+    return out
+
+
+def hqq_dequantize_meta(packed, zero_q: Meta8, rows: int, cols: int, nbits: int, group: int,
+                        scale=None, scale_q: Meta8 | None = None, out=None, stream=None):
+    """Dequantize a matrix whose zero points (and optionally scales) are kept in
+    8-bit form, in one pass (see include/hqq.h)."""
+    import torch
+    for t, nm in ((packed, "packed"), (scale, "scale"), (out, "out")):
+        _check_tensor(t, nm)
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.float16, device=packed.device)
+    zc = zero_q._c()
+    sc = scale_q._c() if scale_q is not None else None
+    _check(_lib.hqq_dequantize_meta(_ptr(packed), ctypes.byref(zc), _ptr(scale),
+                                    ctypes.byref(sc) if sc is not None else None,
+                                    rows, cols, nbits, group, _ptr(out), _stream(stream)))
     return out

@@ -11,7 +11,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["hqq_api.cu", "hqq_quantize.cu", "hqq_dequantize.cu"]
+SOURCES = ["hqq_api.cu", "hqq_quantize.cu", "hqq_dequantize.cu", "hqq_meta.cu"]
 HEADERS = ["hqq_common.cuh"]
 LIB = os.path.join(PKG, "libhqq.so")
 

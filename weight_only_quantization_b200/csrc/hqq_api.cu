@@ -11,6 +11,10 @@ namespace hqq {
 cudaError_t launch_quantize(const QuantParams& prm, int nbits, int group, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_group,
                               cudaStream_t stream);
+cudaError_t launch_meta_quantize(const __half* x, int64_t n, int log2g, uint8_t* codes,
+                                 __half* scale, __half* zero, cudaStream_t stream);
+cudaError_t launch_meta_dequantize(const uint8_t* codes, const __half* scale, const __half* zero,
+                                   int64_t n, int log2g, __half* out, cudaStream_t stream);
 
 namespace {
 
@@ -58,6 +62,15 @@ struct TableCache {
 };
 thread_local TableCache g_cache;
 
+// log2 of a second-level (meta) group: -1 for 0 (one group over everything),
+// -2 when the size is not a power of two up to 2^30.
+int meta_log2(int64_t mgroup) {
+    if (mgroup == 0) return -1;
+    for (int k = 0; k <= 30; ++k)
+        if (mgroup == ((int64_t)1 << k)) return k;
+    return -2;
+}
+
 int validate_common(int64_t rows, int64_t cols, int nbits, int group) {
     if (rows < 0 || cols < 0) return HQQ_ERR_SHAPE;
     if (nbits != 2 && nbits != 3 && nbits != 4) return HQQ_ERR_UNSUPPORTED;
@@ -89,9 +102,9 @@ extern "C" const char* hqq_status_string(int status) {
         case HQQ_OK: return "HQQ_OK";
         case HQQ_ERR_NULL: return "HQQ_ERR_NULL: a required pointer is NULL";
         case HQQ_ERR_SHAPE: return "HQQ_ERR_SHAPE: bad rows/cols or cols not a multiple of group";
-        case HQQ_ERR_UNSUPPORTED: return "HQQ_ERR_UNSUPPORTED: nbits must be 2/3/4, group 16..256 (power of two)";
+        case HQQ_ERR_UNSUPPORTED: return "HQQ_ERR_UNSUPPORTED: nbits must be 2/3/4, group 16..256 (power of two), meta group 0 or a power of two up to 2^30";
         case HQQ_ERR_PARAM: return "HQQ_ERR_PARAM: need 0<p<=1, beta>0, kappa>0 (finite), 0<=iters<=255";
-        case HQQ_ERR_ALIGN: return "HQQ_ERR_ALIGN: W/W_out need 16-byte, packed/zero_f32 4-byte, scale/zero 2-byte alignment";
+        case HQQ_ERR_ALIGN: return "HQQ_ERR_ALIGN: W/W_out/meta x/meta out need 16-byte, meta codes 8-byte, packed/zero_f32 4-byte, scale/zero 2-byte alignment";
         case HQQ_ERR_CUDA: return "HQQ_ERR_CUDA: kernel launch failed (see cudaGetLastError)";
         default: return "HQQ: unknown status";
     }
@@ -172,9 +185,88 @@ extern "C" int hqq_dequantize(const void* packed, const void* scale, const void*
     if (!aligned(packed, 4) || !aligned(scale, 2) || !aligned(zero, 2) || !aligned(W_out, 16))
         return HQQ_ERR_ALIGN;
     DequantParams prm;
+    std::memset(&prm, 0, sizeof prm);
     prm.packed = static_cast<const uint8_t*>(packed);
     prm.scale = static_cast<const __half*>(scale);
     prm.zero = static_cast<const __half*>(zero);
+    prm.out = static_cast<__half*>(W_out);
+    prm.n_units = n / 8;
+    prm.group = group;
+    const cudaError_t err = launch_dequantize(prm, nbits, log2_of_group(group),
+                                              static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
+extern "C" int64_t hqq_meta_groups(int64_t n, int64_t mgroup) {
+    if (n < 0 || mgroup < 0) return -1;
+    if (n == 0) return 0;
+    if (mgroup == 0) return 1;
+    return (n + mgroup - 1) / mgroup;
+}
+
+extern "C" int hqq_meta_quantize(const void* x, int64_t n, int64_t mgroup, uint8_t* codes,
+                                 void* scale, void* zero, void* stream) {
+    if (n < 0 || mgroup < 0 || n > ((int64_t)1 << 40)) return HQQ_ERR_SHAPE;
+    const int lg = meta_log2(mgroup);
+    if (lg == -2) return HQQ_ERR_UNSUPPORTED;
+    if (n == 0) return HQQ_OK;
+    if (!x || !codes || !scale || !zero) return HQQ_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(codes, 8) || !aligned(scale, 2) || !aligned(zero, 2))
+        return HQQ_ERR_ALIGN;
+    const cudaError_t err = launch_meta_quantize(
+        static_cast<const __half*>(x), n, lg, codes, static_cast<__half*>(scale),
+        static_cast<__half*>(zero), static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
+extern "C" int hqq_meta_dequantize(const uint8_t* codes, const void* scale, const void* zero,
+                                   int64_t n, int64_t mgroup, void* out, void* stream) {
+    if (n < 0 || mgroup < 0 || n > ((int64_t)1 << 40)) return HQQ_ERR_SHAPE;
+    const int lg = meta_log2(mgroup);
+    if (lg == -2) return HQQ_ERR_UNSUPPORTED;
+    if (n == 0) return HQQ_OK;
+    if (!codes || !scale || !zero || !out) return HQQ_ERR_NULL;
+    if (!aligned(codes, 8) || !aligned(scale, 2) || !aligned(zero, 2) || !aligned(out, 16))
+        return HQQ_ERR_ALIGN;
+    const cudaError_t err = launch_meta_dequantize(
+        codes, static_cast<const __half*>(scale), static_cast<const __half*>(zero), n, lg,
+        static_cast<__half*>(out), static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
+namespace {
+// Checks one 8-bit meta form and fills its kernel image; HQQ_OK or an error.
+int meta8_image(const hqq_meta8* m, Meta8& out) {
+    if (!m->codes || !m->scale || !m->zero) return HQQ_ERR_NULL;
+    if (m->group < 0) return HQQ_ERR_SHAPE;
+    const int lg = meta_log2(m->group);
+    if (lg == -2) return HQQ_ERR_UNSUPPORTED;
+    if (!aligned(m->scale, 2) || !aligned(m->zero, 2)) return HQQ_ERR_ALIGN;
+    out.codes = m->codes;
+    out.scale = static_cast<const __half*>(m->scale);
+    out.zero = static_cast<const __half*>(m->zero);
+    out.shift = lg < 0 ? 62 : lg;
+    return HQQ_OK;
+}
+}  // namespace
+
+extern "C" int hqq_dequantize_meta(const void* packed, const hqq_meta8* zero_q, const void* scale,
+                                   const hqq_meta8* scale_q, int64_t rows, int64_t cols,
+                                   int nbits, int group, void* W_out, void* stream) {
+    int st = validate_common(rows, cols, nbits, group);
+    if (st != HQQ_OK) return st;
+    if (scale && scale_q) return HQQ_ERR_PARAM;
+    const int64_t n = rows * cols;
+    if (n == 0) return HQQ_OK;
+    if (!packed || !zero_q || !W_out || (!scale && !scale_q)) return HQQ_ERR_NULL;
+    DequantParams prm;
+    std::memset(&prm, 0, sizeof prm);
+    if ((st = meta8_image(zero_q, prm.zq)) != HQQ_OK) return st;
+    if (scale_q && (st = meta8_image(scale_q, prm.sq)) != HQQ_OK) return st;
+    if (!aligned(packed, 4) || !aligned(W_out, 16) || (scale && !aligned(scale, 2)))
+        return HQQ_ERR_ALIGN;
+    prm.packed = static_cast<const uint8_t*>(packed);
+    prm.scale = static_cast<const __half*>(scale);
     prm.out = static_cast<__half*>(W_out);
     prm.n_units = n / 8;
     prm.group = group;

@@ -49,13 +49,23 @@ struct QuantParams {
     float shrink_thr[kMaxIters];  // |r| <= thr[t] guarantees W_e == 0 at step t
 };
 
-struct DequantParams {
-    const uint8_t* packed;
+// 8-bit form of a meta tensor (zero points or scales): codes, the fp16 s and z
+// of each second-level group, and log2 of that group (62: one group).
+struct Meta8 {
+    const uint8_t* codes;
     const __half* scale;
     const __half* zero;
+    int shift;
+};
+
+struct DequantParams {
+    const uint8_t* packed;
+    const __half* scale;   // fp16 scales, unless given in 8-bit form (sq)
+    const __half* zero;    // fp16 zero points, unless given in 8-bit form (zq)
     __half* out;
     int64_t n_units;       // n_elems / 8
     int group;
+    Meta8 zq, sq;
 };
 
 // Shared-memory image of one PowTable (separate arrays, so that the two values

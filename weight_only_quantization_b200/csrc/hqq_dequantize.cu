@@ -88,7 +88,18 @@ __device__ __forceinline__ uint32_t unit_bits(const uint8_t* __restrict__ packed
     }
 }
 
-template <int NBITS, bool SMALL>
+// Zero point or scale of group g restored from its 8-bit form (method section
+// 4.1's 8-bit meta data): fp16((c - z2) s2) with the second-level fp16 s2, z2.
+__device__ __forceinline__ float restore_meta(const Meta8& m, int64_t g) {
+    const int64_t k = g >> m.shift;
+    const float c = (float)__ldg(m.codes + g);
+    const float v = __fmul_rn(__fsub_rn(c, __half2float(__ldg(m.zero + k))),
+                              __half2float(__ldg(m.scale + k)));
+    return __half2float(__float2half_rn(v));
+}
+
+// META bit 0: zero points in 8-bit form; bit 1: scales in 8-bit form.
+template <int NBITS, bool SMALL, int META>
 __global__ void __launch_bounds__(kDqThreads)
 dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
     for (int64_t base = (int64_t)blockIdx.x * kDqTile; base < prm.n_units;
@@ -100,8 +111,8 @@ dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
             int64_t u = base + r * kDqThreads + threadIdx.x;
             if (u >= prm.n_units) u = 0;
             const int64_t g = (u * 8) >> log2_group;
-            sf[r] = __half2float(__ldg(prm.scale + g));
-            zf[r] = __half2float(__ldg(prm.zero + g));
+            sf[r] = (META & 2) ? restore_meta(prm.sq, g) : __half2float(__ldg(prm.scale + g));
+            zf[r] = (META & 1) ? restore_meta(prm.zq, g) : __half2float(__ldg(prm.zero + g));
             x[r] = unit_bits<NBITS, SMALL>(prm.packed, u);
         }
 #pragma unroll
@@ -110,6 +121,17 @@ dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
             const uint4 o = unit8<NBITS>(x[r], zf[r], sf[r]);
             if (u < prm.n_units) reinterpret_cast<uint4*>(prm.out)[u] = o;
         }
+    }
+}
+
+template <int NBITS, bool SMALL>
+static void launch_dq(const DequantParams& prm, int log2_group, unsigned grid, cudaStream_t stream) {
+    const int meta = (prm.zq.codes ? 1 : 0) | (prm.sq.codes ? 2 : 0);
+    switch (meta) {
+        case 0: dequantize_kernel<NBITS, SMALL, 0><<<grid, kDqThreads, 0, stream>>>(prm, log2_group); break;
+        case 1: dequantize_kernel<NBITS, SMALL, 1><<<grid, kDqThreads, 0, stream>>>(prm, log2_group); break;
+        case 2: dequantize_kernel<NBITS, SMALL, 2><<<grid, kDqThreads, 0, stream>>>(prm, log2_group); break;
+        default: dequantize_kernel<NBITS, SMALL, 3><<<grid, kDqThreads, 0, stream>>>(prm, log2_group); break;
     }
 }
 
@@ -124,11 +146,11 @@ cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_grou
     const bool small = prm.n_units < ((int64_t)1 << 30);
     const unsigned g = (unsigned)blocks;
     switch (nbits) {
-        case 2: dequantize_kernel<2, true><<<g, kDqThreads, 0, stream>>>(prm, log2_group); break;
-        case 4: dequantize_kernel<4, true><<<g, kDqThreads, 0, stream>>>(prm, log2_group); break;
+        case 2: launch_dq<2, true>(prm, log2_group, g, stream); break;
+        case 4: launch_dq<4, true>(prm, log2_group, g, stream); break;
         case 3:
-            if (small) dequantize_kernel<3, true><<<g, kDqThreads, 0, stream>>>(prm, log2_group);
-            else dequantize_kernel<3, false><<<g, kDqThreads, 0, stream>>>(prm, log2_group);
+            if (small) launch_dq<3, true>(prm, log2_group, g, stream);
+            else launch_dq<3, false>(prm, log2_group, g, stream);
             break;
         default: return cudaErrorInvalidValue;
     }
