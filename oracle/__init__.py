@@ -278,6 +278,21 @@ def dequantize_meta(codes, group: int, zero_q: dict, zero_group: int = 0,
     return dequantize(codes, s, z, group)
 
 
+def linear(X, W_hat) -> dict:
+    """Weight-only linear layer on dequantized weights: Y = X W_hat^T.
+
+    X is fp16 [M, K] (tokens x input features), W_hat the fp16 [N, K] matrix
+    that ``dequantize`` restores (output x input features).  The products and
+    their sum are formed in fp64 (numpy matmul), then rounded once to fp16.
+    Returns the fp16 result, the fp64 result and sum_k |x||w| per output (the
+    scale of the rounding bound of any binary32 summation order)."""
+    X64 = np.asarray(X, dtype=np.float16).astype(np.float64)
+    W64 = np.asarray(W_hat, dtype=np.float16).astype(np.float64)
+    Y64 = X64 @ W64.T
+    absum = np.abs(X64) @ np.abs(W64).T
+    return dict(y=Y64.astype(np.float16), y64=Y64, absum=absum)
+
+
 def f32_to_f16(x) -> np.ndarray:
     lib = _load()
     x = np.ascontiguousarray(x, dtype=np.float32)

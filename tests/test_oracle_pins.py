@@ -481,3 +481,29 @@ def test_meta_zero_error_is_small_against_the_code_step():
     bound = s16 / 2 + 255 * abs(s16 - rng_ / 255) + abs(float(zq["zero"][0]) - float(
         -zero.astype(np.float64).min() / (rng_ / 255))) * s16 + np.spacing(np.float16(8.0))
     assert np.max(np.abs(zr - zero.astype(np.float64))) <= bound
+
+
+# ------------------------------------------------- weight-only linear layer
+def test_linear_is_x_times_w_transposed():
+    """Y = X W_hat^T: with X the identity, row k of Y is column k of W_hat
+    (output features along Y's columns), exactly; a plain triple loop on a tiny
+    case gives the same fp64 values; the fp16 result is the fp64 one rounded
+    once."""
+    rng = np.random.default_rng(40)
+    N, K = 24, 64
+    W = synth.student_t_host((N, K), seed=40, stream=1).astype(np.float16)
+    r = oracle.quantize(W, 4, 32, iters=3)
+    Wh = oracle.dequantize(r["codes"], r["scale"], r["zero"], 32).reshape(N, K)
+    eye = np.eye(K, dtype=np.float16)
+    out = oracle.linear(eye, Wh)
+    assert np.array_equal(out["y"], Wh.T)
+    X = (rng.standard_normal((5, K))).astype(np.float16)
+    out = oracle.linear(X, Wh)
+    for m in range(5):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += float(X[m, k]) * float(Wh[n, k])
+            assert abs(acc - out["y64"][m, n]) <= 1e-12 * out["absum"][m, n]
+            assert out["y"][m, n] == np.float16(out["y64"][m, n])
+    assert np.all(out["absum"] >= np.abs(out["y64"]))
