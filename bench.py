@@ -242,7 +242,7 @@ def config_dict(name, mats, n_gpus):
                                         "early_stop": "per group"},
             "step": "quantize + dequantize of every matrix",
             "l2": "inputs larger than L2 (no flush needed)" if params * 2 > 4 * 126e6
-            else "L2 flushed between steps",
+            else "L2 flushed between steps (256 MiB written, outside the step events)",
             "parallelism": f"replicas x{n_gpus} (weak)"}
 
 
@@ -348,15 +348,38 @@ def run_gpu(args):
 
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        for k, (W, q, O) in enumerate(views):
-            if ev is not None:
-                ev[k][0].record(stream)
+    def quantize_all():
+        for W, q, O in views:
             hqq.hqq_quantize(W, q.nbits, q.group, packed=q.packed, scale=q.scale,
                              zero=q.zero)
-            if ev is not None:
-                ev[k][1].record(stream)
+
+    def dequantize_all():
+        for W, q, O in views:
             hqq.hqq_dequantize(q, out=O)
+
+    # one pass = every matrix quantized, then every matrix dequantized; the two
+    # loops of library calls are captured once in CUDA graphs (host launch cost
+    # out of the way of small matrices) unless --no-graph
+    quantize_all()
+    dequantize_all()
+    torch.cuda.synchronize()
+    if not args.no_graph:
+        gq, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gq):
+            quantize_all()
+        with torch.cuda.graph(gd):
+            dequantize_all()
+        run_q, run_d = gq.replay, gd.replay
+    else:
+        run_q, run_d = quantize_all, dequantize_all
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        run_q()
+        if ev is not None:
+            ev[1].record(stream)
+        run_d()
 
     def barrier():
         if pg is not None:
@@ -366,8 +389,13 @@ def run_gpu(args):
         step()
     torch.cuda.synchronize()
 
-    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in views] for _ in range(args.steps)]
+    # small workloads: overwrite a buffer twice the size of L2 before every step,
+    # outside the step's own events (the step time is the sum of those)
+    flush = None
+    if params * 2 <= 4 * 126e6:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
+           for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     barrier()
@@ -375,20 +403,22 @@ def run_gpu(args):
     clocks.start()
     t_start.record(stream)
     for s in range(args.steps):
+        if flush is not None:
+            flush.fill_(s & 0xFF)
         step(evs[s])
+        evs[s][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    ms = t_start.elapsed_time(t_end)
-    q_ms = [evs[s][k][0].elapsed_time(evs[s][k][1]) for s in range(args.steps)
-            for k in range(len(views))]
+    ms = sum(evs[s][0].elapsed_time(evs[s][2]) for s in range(args.steps))
+    q_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(args.steps)]
     ms_max, qsum_max = max_over_ranks([ms, sum(q_ms)], pg, dev)
     ms_step = ms_max / args.steps
     value = ws * params * args.steps / (ms_max / 1e3) / 1e9
 
     # ---- per-kernel figures (rank 0's launches)
-    q_launch_ms = sum(q_ms) / len(q_ms)
+    q_launch_ms = sum(q_ms) / args.steps / len(views)
     dq_ms_step = ms_step - sum(q_ms) / args.steps
     hbm_peak, peak_kind = measured_peaks()
     qbytes = algorithmic_bytes(mats)
@@ -447,6 +477,10 @@ def run_gpu(args):
             "gpu_launches": 2 * len(views) * args.steps,
             "clocks": clk}
 
+    # ---- 8-bit meta data (zero points: one group; scales: groups of 128)
+    if not args.no_meta:
+        line["meta8"] = run_meta8(args, views, hqq, dev, hbm_peak, pg)
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     if ws == 1 and not args.no_cpu_baseline:
         def W_source(lab, shape, rows, seed, stream_):
@@ -478,6 +512,87 @@ def run_gpu(args):
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def run_meta8(args, views, hqq, dev, hbm_peak, pg):
+    """Times, over the whole workload, the 8-bit storage of every matrix's zero
+    points (one group per matrix) and scales (groups of 128), and the one-pass
+    weight dequantization from that 8-bit form (CUDA events, summed per kernel
+    kind; inputs resident)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    metas = []
+    for W, q, O in views:
+        mg = q.scale.numel()
+        zq = hqq.Meta8(torch.empty(mg, dtype=torch.uint8, device=dev),
+                       torch.empty(1, dtype=torch.float16, device=dev),
+                       torch.empty(1, dtype=torch.float16, device=dev), 0)
+        ng = hqq.hqq_meta_groups(mg, 128)
+        sq = hqq.Meta8(torch.empty(mg, dtype=torch.uint8, device=dev),
+                       torch.empty(ng, dtype=torch.float16, device=dev),
+                       torch.empty(ng, dtype=torch.float16, device=dev), 128)
+        metas.append((zq, sq))
+
+    def meta_all():
+        for k, (W, q, O) in enumerate(views):
+            zq, sq = metas[k]
+            hqq.hqq_meta_quantize(q.zero.view(-1), 0, codes=zq.codes, scale=zq.scale,
+                                  zero=zq.zero)
+            hqq.hqq_meta_quantize(q.scale.view(-1), 128, codes=sq.codes, scale=sq.scale,
+                                  zero=sq.zero)
+
+    def dq_all():
+        for k, (W, q, O) in enumerate(views):
+            zq, sq = metas[k]
+            hqq.hqq_dequantize_meta(q.packed, zq, q.rows, q.cols, q.nbits, q.group, scale_q=sq,
+                                    out=O)
+
+    meta_all()
+    dq_all()
+    torch.cuda.synchronize()
+    if not args.no_graph:
+        gm, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gm):
+            meta_all()
+        with torch.cuda.graph(gd):
+            dq_all()
+        run_m, run_d = gm.replay, gd.replay
+    else:
+        run_m, run_d = meta_all, dq_all
+    reps = 3
+    for _ in range(3):
+        run_m()
+        run_d()
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(reps)]
+    torch.cuda.synchronize()
+    for r in range(reps):
+        evs[r][0].record(stream)
+        run_m()
+        evs[r][1].record(stream)
+        run_d()
+        evs[r][2].record(stream)
+    torch.cuda.synchronize()
+    mq_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / reps
+    dq_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / reps
+    mq_ms, dq_ms = max_over_ranks([mq_ms, dq_ms], pg, dev)
+    mq_bytes = dq_bytes = 0
+    for W, q, O in views:
+        mg = q.scale.numel()
+        ng = hqq.hqq_meta_groups(mg, 128)
+        mq_bytes += 2 * (2 * mg + mg) + 2 * 2 + 2 * 2 * ng      # read fp16, write codes + s,z
+        dq_bytes += (q.packed.numel() + 2 * mg + 2 * 2 + 2 * 2 * ng
+                     + 2 * q.rows * q.cols)
+    mq_gbs = mq_bytes / (mq_ms / 1e3) / 1e9
+    dq_gbs = dq_bytes / (dq_ms / 1e3) / 1e9
+    params = sum(q.rows * q.cols for _, q, _ in views)
+    return {"what": "zero points 8-bit (one group per matrix), scales 8-bit (groups of 128); "
+                    "weights dequantized in one pass from that form",
+            "meta_quantize": {"ms_per_pass": mq_ms, "gbs": mq_gbs, "hbm_frac": mq_gbs / hbm_peak,
+                              "launches_per_pass": 2 * len(views)},
+            "dequantize_meta": {"ms_per_pass": dq_ms, "gbs": dq_gbs,
+                                "hbm_frac": dq_gbs / hbm_peak,
+                                "gparam_s": params / (dq_ms / 1e3) / 1e9,
+                                "bytes_per_param": dq_bytes / params}}
 
 
 def run_stream_pass(mats, hqq, dev, views):
@@ -592,6 +707,10 @@ def main():
                     help="first N layers only of a model-shaped set (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
     ap.add_argument("--no-stream", action="store_true", help="skip the streamed generate+quantize pass")
+    ap.add_argument("--no-meta", action="store_true", help="skip the 8-bit meta-data timing")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every library call from Python each pass instead of replaying "
+                         "CUDA graphs of the passes")
     ap.add_argument("--impl", default="libhqq", choices=["libhqq", "reference"])
     ap.add_argument("--cpu-s", type=float, default=10.0, help="oracle CPU-baseline budget (s)")
     ap.add_argument("--ref-step-s", type=float, default=4.0, help="reference arm seconds per step")
