@@ -201,6 +201,34 @@ int hqq_dequantize_meta(const void* packed, const hqq_meta8* zero_q, const void*
                         const hqq_meta8* scale_q, int64_t rows, int64_t cols, int nbits,
                         int group, void* W_out, void* stream);
 
+/*
+ * hqq_linear -- weight-only linear layer on a quantized matrix: the matrix
+ * product with section 2's Q^-1 fused in,
+ *   Y[m, n] = sum over k of X[m, k] * W_hat[n, k],
+ *   W_hat   = fp16((code - z) * s), exactly the values hqq_dequantize writes,
+ * without W_hat ever being stored.  Products and sums are formed in the
+ * tensor cores' fp32 accumulator (summation order unspecified) and Y is
+ * rounded to fp16 once.
+ *
+ *   X      [in]  fp16 [M, cols] row-major (tokens x input features),
+ *                16-byte aligned.
+ *   M      [in]  number of tokens, 0 <= M <= 65535*256 (M == 0: no-op).
+ *   packed, scale, zero, rows, cols, nbits, group [in]  the quantized
+ *                [rows, cols] matrix as hqq_quantize writes it (alignment as
+ *                for hqq_dequantize).
+ *   Y      [out] fp16 [M, rows] row-major (tokens x output features), 2-byte
+ *                aligned.
+ *   status [out] optional device int (NULL allowed), 4-byte aligned.  The
+ *                kernel stores 1 there when one of its internal waits ran
+ *                out (a device fault, never a consequence of valid arguments;
+ *                Y is then unspecified).  It never stores 0: clear it first.
+ *   stream [in]  cudaStream_t (NULL = legacy default stream).
+ * HQQ_ERR_CUDA also covers a driver without the tensor-map entry point.
+ */
+int hqq_linear(const void* X, int64_t M, const void* packed, const void* scale,
+               const void* zero, int64_t rows, int64_t cols, int nbits, int group,
+               void* Y, int* status, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* hqq_status_string(int status);
 

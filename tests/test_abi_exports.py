@@ -14,8 +14,12 @@ HEADER = os.path.join(ROOT, "include", "hqq.h")
 
 @pytest.fixture(scope="module")
 def lib():
-    from weight_only_quantization_b200 import build
-    build.build()
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "hqq_build", os.path.join(ROOT, "weight_only_quantization_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
     import weight_only_quantization_b200 as hqq
     return hqq
 

@@ -15,7 +15,7 @@ from dataclasses import dataclass
 __all__ = ["HQQError", "hqq_quantize", "hqq_quantize_ex", "hqq_dequantize",
            "hqq_packed_bytes", "hqq_status_string", "QuantizedMatrix", "LIB_PATH",
            "Meta8", "hqq_meta_groups", "hqq_meta_quantize", "hqq_meta_dequantize",
-           "hqq_dequantize_meta",
+           "hqq_dequantize_meta", "hqq_linear",
            "DEFAULT_P", "DEFAULT_BETA", "DEFAULT_KAPPA", "DEFAULT_ITERS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -25,7 +25,7 @@ DEFAULT_P, DEFAULT_BETA, DEFAULT_KAPPA, DEFAULT_ITERS = 0.7, 1.0, 1.01, 20
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m weight_only_quantization_b200.build`")
+                      "`python weight_only_quantization_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 _P, _I64, _I, _F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
@@ -56,6 +56,8 @@ class _CMeta8(ctypes.Structure):
 _lib.hqq_dequantize_meta.argtypes = [_P, ctypes.POINTER(_CMeta8), _P, ctypes.POINTER(_CMeta8),
                                      _I64, _I64, _I, _I, _P, _P]
 _lib.hqq_dequantize_meta.restype = _I
+_lib.hqq_linear.argtypes = [_P, _I64, _P, _P, _P, _I64, _I64, _I, _I, _P, _P, _P]
+_lib.hqq_linear.restype = _I
 
 
 class HQQError(RuntimeError):
@@ -252,4 +254,24 @@ def hqq_dequantize_meta(packed, zero_q: Meta8, rows: int, cols: int, nbits: int,
     _check(_lib.hqq_dequantize_meta(_ptr(packed), ctypes.byref(zc), _ptr(scale),
                                     ctypes.byref(sc) if sc is not None else None,
                                     rows, cols, nbits, group, _ptr(out), _stream(stream)))
+    return out
+
+
+def hqq_linear(X, q: QuantizedMatrix, out=None, status=None, stream=None):
+    """Y = X W_hat^T for fp16 X [M, cols] and a quantized [rows, cols] matrix,
+    with the dequantization fused into the tensor-core product (see
+    include/hqq.h).  ``status`` is an optional int32 CUDA tensor of one element
+    (cleared by the caller) that the kernel sets to 1 if an internal wait ran
+    out."""
+    import torch
+    if X.dtype != torch.float16 or X.dim() != 2 or X.shape[1] != q.cols:
+        raise ValueError("X must be a float16 [M, cols] tensor")
+    for t, nm in ((X, "X"), (q.packed, "packed"), (q.scale, "scale"), (q.zero, "zero"),
+                  (out, "out"), (status, "status")):
+        _check_tensor(t, nm)
+    if out is None:
+        out = torch.empty((X.shape[0], q.rows), dtype=torch.float16, device=X.device)
+    _check(_lib.hqq_linear(_ptr(X), X.shape[0], _ptr(q.packed), _ptr(q.scale), _ptr(q.zero),
+                           q.rows, q.cols, q.nbits, q.group, _ptr(out), _ptr(status),
+                           _stream(stream)))
     return out

@@ -1,6 +1,8 @@
 """Build libhqq.so in-tree for sm_100a (nvcc; no JIT cache, no torch extension).
 
-    python -m weight_only_quantization_b200.build [--force]
+    python weight_only_quantization_b200/build.py [--force]
+
+(run as a file: importing the package loads the library this script builds)
 """
 from __future__ import annotations
 
@@ -11,8 +13,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["hqq_api.cu", "hqq_quantize.cu", "hqq_dequantize.cu", "hqq_meta.cu"]
-HEADERS = ["hqq_common.cuh"]
+SOURCES = ["hqq_api.cu", "hqq_quantize.cu", "hqq_dequantize.cu", "hqq_meta.cu", "hqq_linear.cu"]
+HEADERS = ["hqq_common.cuh", "hqq_unpack.cuh"]
 LIB = os.path.join(PKG, "libhqq.so")
 
 NVCC_FLAGS = [

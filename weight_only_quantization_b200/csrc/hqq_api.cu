@@ -11,6 +11,16 @@ namespace hqq {
 cudaError_t launch_quantize(const QuantParams& prm, int nbits, int group, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_group,
                               cudaStream_t stream);
+struct LinearParams {
+    const uint8_t* packed;
+    const __half* scale;
+    const __half* zero;
+    __half* Y;
+    int* status;
+    int64_t M, N, K;
+    int log2_group;
+};
+cudaError_t launch_linear(const LinearParams& prm, const void* X, int nbits, cudaStream_t stream);
 cudaError_t launch_meta_quantize(const __half* x, int64_t n, int log2g, uint8_t* codes,
                                  __half* scale, __half* zero, cudaStream_t stream);
 cudaError_t launch_meta_dequantize(const uint8_t* codes, const __half* scale, const __half* zero,
@@ -272,5 +282,32 @@ extern "C" int hqq_dequantize_meta(const void* packed, const hqq_meta8* zero_q, 
     prm.group = group;
     const cudaError_t err = launch_dequantize(prm, nbits, log2_of_group(group),
                                               static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
+extern "C" int hqq_linear(const void* X, int64_t M, const void* packed, const void* scale,
+                          const void* zero, int64_t rows, int64_t cols, int nbits, int group,
+                          void* Y, int* status, void* stream) {
+    int st = validate_common(rows, cols, nbits, group);
+    if (st != HQQ_OK) return st;
+    // one launch covers 65535 CTA rows of 256 tokens
+    if (M < 0 || M > (int64_t)65535 * 256) return HQQ_ERR_SHAPE;
+    if (M == 0 || rows == 0 || cols == 0) return HQQ_OK;
+    if (!X || !packed || !scale || !zero || !Y) return HQQ_ERR_NULL;
+    if (!aligned(X, 16) || !aligned(packed, 4) || !aligned(scale, 2) || !aligned(zero, 2) ||
+        !aligned(Y, 2) || (status && !aligned(status, 4)))
+        return HQQ_ERR_ALIGN;
+    LinearParams prm;
+    std::memset(&prm, 0, sizeof prm);
+    prm.packed = static_cast<const uint8_t*>(packed);
+    prm.scale = static_cast<const __half*>(scale);
+    prm.zero = static_cast<const __half*>(zero);
+    prm.Y = static_cast<__half*>(Y);
+    prm.status = status;
+    prm.M = M;
+    prm.N = rows;
+    prm.K = cols;
+    prm.log2_group = log2_of_group(group);
+    const cudaError_t err = launch_linear(prm, X, nbits, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }

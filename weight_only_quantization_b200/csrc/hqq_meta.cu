@@ -10,9 +10,11 @@
 // restored as fp16((c - z) s) from the stored fp16 s and z.
 //
 // Kernels
-//  - meta_group_kernel: groups of 2^k values; a segment of min(2^k, 32) lanes
-//    per group, exact min/max by shuffles, then the codes.  Meta tensors are
-//    1/16..1/256 of the weights, so this is a small memory-bound pass.
+//  - meta_group_kernel / meta_group_vec_kernel: groups of 2^k values; a
+//    segment of lanes per group (one value, or for 2^k >= 8 one 16-byte vector
+//    of 8 values, per lane and step), exact min/max by shuffles, then the
+//    codes.  Meta tensors are 1/16..1/256 of the weights: a small
+//    memory-bound pass.
 //  - meta_whole_kernel: one group over the whole tensor ("no grouping").  One
 //    thread-block cluster reduces the tensor: every CTA takes an interleaved
 //    share of 16-byte vectors, the CTAs exchange their min/max through
@@ -118,8 +120,67 @@ meta_group_kernel(const __half* __restrict__ x, int64_t n, int log2g, int64_t ng
     }
 }
 
+// Groups of 2^k >= 8 values: each lane takes 16-byte vectors (8 values), a
+// segment of min(2^k/8, 32) lanes per group.  The vector that holds the end of
+// a ragged last group is read value by value.
+__global__ void __launch_bounds__(kGroupThreads)
+meta_group_vec_kernel(const __half* __restrict__ x, int64_t n, int log2g, int64_t ngroups,
+                      uint8_t* __restrict__ codes, __half* __restrict__ scale,
+                      __half* __restrict__ zero) {
+    const int lane = threadIdx.x & 31;
+    const int lv = log2g - 3;                         // log2(vectors per group)
+    const int lseg = lv < 5 ? lv : 5;
+    const int seg = 1 << lseg;
+    const int per_warp = 32 >> lseg;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int k0 = lane & (seg - 1);
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    const int64_t nfull = n >> 3;                     // vectors entirely inside x
+    for (int64_t gb = warp * per_warp; gb < ngroups; gb += nwarps * per_warp) {
+        const int64_t gi = gb + (lane >> lseg);
+        const bool valid = gi < ngroups;
+        const int64_t v0 = gi << lv;                  // first vector of the group
+        const int64_t vend = valid ? min(v0 + ((int64_t)1 << lv), (n + 7) >> 3) : v0;
+        __half2 hmn = __float2half2_rn(INFINITY), hmx = __float2half2_rn(-INFINITY);
+        float mn = INFINITY, mx = -INFINITY;
+        for (int64_t v = v0 + k0; v < vend; v += seg) {
+            if (v < nfull) {
+                minmax8(__ldg(xv + v), hmn, hmx);
+            } else {
+                for (int64_t i = v << 3; i < n; ++i) {
+                    const float f = __half2float(x[i]);
+                    mn = fminf(mn, f);
+                    mx = fmaxf(mx, f);
+                }
+            }
+        }
+        mn = fminf(mn, fminf(__low2float(hmn), __high2float(hmn)));
+        mx = fmaxf(mx, fmaxf(__low2float(hmx), __high2float(hmx)));
+        for (int o = seg >> 1; o > 0; o >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        if (valid) {
+            const MetaAffine a = meta_affine(mn, mx);
+            for (int64_t v = v0 + k0; v < vend; v += seg) {
+                if (v < nfull) {
+                    reinterpret_cast<uint2*>(codes)[v] = meta_codes8(__ldg(xv + v), a);
+                } else {
+                    for (int64_t i = v << 3; i < n; ++i)
+                        codes[i] = (uint8_t)meta_code(__half2float(x[i]), a);
+                }
+            }
+            if (k0 == 0) {
+                scale[gi] = __float2half_rn(a.s);
+                zero[gi] = __float2half_rn(a.z);
+            }
+        }
+    }
+}
+
 constexpr int kWholeThreads = 1024;
-constexpr int kWholeBatch = 4;                        // 16-byte loads in flight per thread
+constexpr int kWholeBatch = 8;                        // 16-byte loads in flight per thread
 
 __global__ void __launch_bounds__(kWholeThreads)
 meta_whole_kernel(const __half* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
@@ -315,13 +376,19 @@ cudaError_t launch_meta_quantize(const __half* x, int64_t n, int log2g, uint8_t*
         lg = 0;
         while (((int64_t)1 << lg) < n) ++lg;
     }
-    const int lseg = lg < 5 ? lg : 5;
+    const bool vec = lg >= 3;                         // 16-byte vectors never straddle groups
+    const int lanes_log = vec ? lg - 3 : lg;
+    const int lseg = lanes_log < 5 ? lanes_log : 5;
     const int64_t warps = (ngroups + (32 >> lseg) - 1) / (32 >> lseg);
     int64_t blocks = (warps + kGroupThreads / 32 - 1) / (kGroupThreads / 32);
     const int64_t cap = (int64_t)sm_count() * 16;
     if (blocks > cap) blocks = cap;
-    meta_group_kernel<<<(unsigned)blocks, kGroupThreads, 0, stream>>>(x, n, lg, ngroups, codes,
-                                                                      scale, zero);
+    if (vec)
+        meta_group_vec_kernel<<<(unsigned)blocks, kGroupThreads, 0, stream>>>(
+            x, n, lg, ngroups, codes, scale, zero);
+    else
+        meta_group_kernel<<<(unsigned)blocks, kGroupThreads, 0, stream>>>(x, n, lg, ngroups,
+                                                                          codes, scale, zero);
     return cudaGetLastError();
 }
 
