@@ -10,14 +10,18 @@
 // One CTA computes a 128-feature x BN-token tile of Y^T on the 5th-generation
 // tensor cores (tcgen05.mma, kind::f16, accumulator in tensor memory):
 //   A = W_hat tile [128 features x 64 k], K-major, 128-byte swizzle, written to
-//       shared memory by 4 producer warps that unpack and dequantize the codes
-//       (one feature row per thread, eight 16-byte units per k-tile);
+//       shared memory by 8 producer warps that unpack and dequantize the codes
+//       (four 16-byte units per thread and k-tile; the 8 lanes of a row read
+//       its codes as one contiguous run);
 //   B = X tile [BN tokens x 64 k], K-major, 128-byte swizzle, loaded by TMA
 //       (rows past M and columns past K read as zeros);
 //   D = [128 x BN] fp32 in tensor memory, read back by the producer warps with
 //       tcgen05.ld after the last k-tile and stored as fp16.
 // Warp 0 issues the TMA loads, warp 1 owns the tensor memory and issues the
-// MMAs (one elected thread), warps 2..5 produce A and run the epilogue.  A
+// MMAs (one elected thread), warps 2..9 produce A and run the epilogue.  For
+// few tokens (BN <= 32) and a grid short of two CTAs per SM, a cluster of 2 or
+// 4 CTAs splits the k-tiles of one output tile and reduces the partial sums
+// through distributed shared memory.  A
 // STAGES-deep ring of (A, B) stages is handed over with mbarriers: full_a (128
 // producer arrivals), full_b (TMA transaction bytes), empty (tcgen05.commit of
 // the MMAs that read the stage).
@@ -26,18 +30,21 @@
 // records a status, makes every later wait of the CTA return at once, and the
 // CTA still drains its own TMA loads and MMAs (again with a bound) before it
 // frees its tensor memory and exits; the result is then unspecified.
+#include <cooperative_groups.h>
 #include <cuda.h>
 
 #include "hqq_unpack.cuh"
 
 namespace hqq {
 
+namespace cg = cooperative_groups;
+
 namespace {
 
 constexpr int kBM = 128;                 // features per CTA (MMA M)
 constexpr int kBK = 64;                  // k per stage: one 128-byte swizzle row
 constexpr int kStages = 4;
-constexpr int kThreads = 192;            // 6 warps
+constexpr int kThreads = 320;            // 10 warps
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s per wait
 
@@ -146,21 +153,6 @@ __device__ __forceinline__ void fence_after_sync() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// 16 consecutive fp32 columns of this warp's 32 tensor-memory lanes.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 }  // namespace
 
 struct LinearParams {
@@ -175,35 +167,82 @@ struct LinearParams {
 
 namespace {
 
+constexpr int kProducerWarps = 8;                     // warps 2..9
+constexpr int kProducers = kProducerWarps * 32;
+constexpr int kUnitsPerThread = kBM * (kBK / 8) / kProducers;   // 4
+constexpr int kMaxSplit = 4;                          // k-slices per cluster (decode shapes)
+
+// The units one producer thread writes per k-tile: unit column j = lane % 8 of
+// tile rows pw*16 + lane/8 + 4i (i < 4).  The 8 lanes of a row read that row's
+// codes for the k-tile as one contiguous run (24 bytes at 3 bits), so a warp
+// load touches 4 rows, not 32.
 template <int NBITS, bool SMALL>
-struct KTileCodes {          // one feature row's codes and group data for one k-tile
-    uint32_t bits[8];
-    float s[8], z[8];
-    uint32_t present;        // bit j: unit j lies inside the matrix
+struct KTileCodes {
+    UnitRaw raw[kUnitsPerThread];                     // loaded words, merged at use
+    __half2 sz[kUnitsPerThread];                      // (s, z) of each unit's group
+    uint32_t present;                                 // bit i: unit i lies inside the matrix
 };
 
-template <int NBITS, bool SMALL>
-__device__ __forceinline__ void load_ktile(const LinearParams& p, int64_t n, int kt,
-                                           KTileCodes<NBITS, SMALL>& c) {
-    c.present = 0u;
+// Per-thread constants of the producer: the unit index (of the flat code
+// stream) and the group index of its four rows at k = 0.  Rows past N hold
+// no unit.
+struct ProducerRows {
+    int64_t u0[kUnitsPerThread];
+    int64_t g0[kUnitsPerThread];
+    uint32_t row_ok;                                  // bit i: row i inside the matrix
+};
+
+__device__ __forceinline__ void producer_rows(const LinearParams& p, int64_t row0, int j,
+                                              ProducerRows& pr) {
+    pr.row_ok = 0u;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int64_t kk = (int64_t)kt * kBK + 8 * j;
-        if (n < p.N && kk < p.K) {
-            const int64_t flat = n * p.K + kk;
-            const int64_t g = flat >> p.log2_group;
-            c.bits[j] = unit_bits<NBITS, SMALL>(p.packed, flat >> 3);
-            c.s[j] = __half2float(__ldg(p.scale + g));
-            c.z[j] = __half2float(__ldg(p.zero + g));
-            c.present |= 1u << j;
+    for (int i = 0; i < kUnitsPerThread; ++i) {
+        const int64_t n = row0 + 4 * i;
+        pr.u0[i] = (n * p.K) / 8 + j;
+        pr.g0[i] = (n * p.K) >> p.log2_group;
+        if (n < p.N) pr.row_ok |= 1u << i;
+    }
+}
+
+template <int NBITS, bool SMALL>
+__device__ __forceinline__ void load_ktile(const LinearParams& p, const ProducerRows& pr, int j,
+                                           int kt, KTileCodes<NBITS, SMALL>& c) {
+    const int64_t kk = (int64_t)kt * kBK + 8 * j;
+    c.present = kk < p.K ? pr.row_ok : 0u;
+    const int64_t du = (int64_t)kt * (kBK / 8);
+    const int64_t dg = kk >> p.log2_group;
+#pragma unroll
+    for (int i = 0; i < kUnitsPerThread; ++i) {
+        if (c.present & (1u << i)) {
+            const int64_t g = pr.g0[i] + dg;
+            c.raw[i] = unit_fetch<NBITS, SMALL>(p.packed, pr.u0[i] + du);
+            c.sz[i] = __halves2half2(__ldg(p.scale + g), __ldg(p.zero + g));
         } else {
-            c.bits[j] = 0u;
-            c.s[j] = 0.0f;
-            c.z[j] = 0.0f;
+            c.raw[i].w0 = c.raw[i].w1 = c.raw[i].shift = 0u;
+            c.sz[i] = __float2half2_rn(0.0f);
         }
     }
 }
 
+// 8 consecutive fp32 columns of this warp's 32 tensor-memory lanes.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+constexpr int kPrefetch = 2;                          // k-tiles of codes in flight per thread (2 keeps two CTAs per SM; 3 and 4 measured slower for few tokens)
+
+// gridDim.z > 1: the CTAs of a (1, 1, gridDim.z) cluster split the k-tiles of
+// one output tile; each keeps its partial sums in its own tensor memory, the
+// others write theirs into rank 0's (then idle) stage buffers through
+// distributed shared memory, and rank 0 adds them and stores Y.
 template <int NBITS, bool SMALL, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ LinearParams prm) {
@@ -216,12 +255,16 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
     uint8_t* b_st = smem + kStages * kABytes;              // kStages x BN*128 B
     uint64_t* bars = reinterpret_cast<uint64_t*>(b_st + kStages * kBBytes);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
+    float* red = reinterpret_cast<float*>(smem);           // split-k partials (rank 0)
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n0 = (int64_t)blockIdx.x * kBM;
     const int64_t m0 = (int64_t)blockIdx.y * BN;
+    const int ks = (int)gridDim.z, rank = (int)blockIdx.z;
     const int KT = (int)((prm.K + kBK - 1) / kBK);
+    const int kt0 = (int)((int64_t)KT * rank / ks);
+    const int nkt = (int)((int64_t)KT * (rank + 1) / ks) - kt0;
     const uint32_t bar0 = smem_u32(bars);
     // full_a[s] = bar0 + 8s, full_b[s] = bar0 + 8(S+s), empty[s] = bar0 + 8(2S+s), done
     auto full_a = [&](int s) { return bar0 + 8u * s; };
@@ -232,7 +275,7 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
     if (threadIdx.x == 0) {
         abort_flag = 0;
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(full_a(s), kBM);
+            mbar_init(full_a(s), kProducers);
             mbar_init(full_b(s), 1);
             mbar_init(empty(s), 1);
         }
@@ -256,21 +299,22 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
 
     if (warp == 0) {
         if (lane == 0) {                                    // X tiles by TMA
-            for (int kt = 0; kt < KT; ++kt) {
+            for (int kt = 0; kt < nkt; ++kt) {
                 const int s = kt % kStages;
                 const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
                 mbar_wait(empty(s), ph ^ 1u, abrt, prm.status, false);
                 mbar_expect_tx(full_b(s), kBBytes);
-                tma_load_2d(smem_u32(b_st + s * kBBytes), &xmap, full_b(s), kt * kBK, (int)m0);
+                tma_load_2d(smem_u32(b_st + s * kBBytes), &xmap, full_b(s), (kt0 + kt) * kBK,
+                            (int)m0);
             }
-            for (int kt = KT > kStages ? KT - kStages : 0; kt < KT; ++kt)   // own loads landed
+            for (int kt = nkt > kStages ? nkt - kStages : 0; kt < nkt; ++kt)  // own loads landed
                 mbar_wait(full_b(kt % kStages), (uint32_t)(kt / kStages) & 1u, abrt, prm.status,
                           true);
         }
     } else if (warp == 1) {
         if (lane == 0) {                                    // MMA issue
             const uint32_t idesc = f16_idesc<BN>();
-            for (int kt = 0; kt < KT; ++kt) {
+            for (int kt = 0; kt < nkt; ++kt) {
                 const int s = kt % kStages;
                 const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
                 mbar_wait(full_b(s), ph, abrt, prm.status, false);
@@ -287,38 +331,86 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
             mma_commit(done);
         }
     } else {
-        // ---- producers of W_hat: thread r writes feature row n0 + r of every stage
-        const int r = threadIdx.x - 64;
-        const int64_t n = n0 + r;
-        KTileCodes<NBITS, SMALL> cur, nxt;
-        load_ktile<NBITS, SMALL>(prm, n, 0, cur);
-        for (int kt = 0; kt < KT; ++kt) {
-            const int s = kt % kStages;
-            const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
-            if (kt + 1 < KT) load_ktile<NBITS, SMALL>(prm, n, kt + 1, nxt);
-            mbar_wait(empty(s), ph ^ 1u, abrt, prm.status, false);
-            uint8_t* row = a_st + s * kABytes + r * 128;
+        // ---- producers of W_hat
+        const int pw = warp - 2, j = lane & 7;
+        const int rbase = pw * 16 + (lane >> 3);            // tile row of unit i: rbase + 4i
+        ProducerRows pr;
+        producer_rows(prm, n0 + rbase, j, pr);
+        // a ring of kPrefetch k-tiles of codes in registers (indices fixed by unrolling)
+        KTileCodes<NBITS, SMALL> ring[kPrefetch];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (cur.present & (1u << j)) v = unit8<NBITS>(cur.bits[j], cur.z[j], cur.s[j]);
-                *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) << 4)) = v;
+        for (int u = 0; u < kPrefetch - 1; ++u)
+            if (u < nkt) load_ktile<NBITS, SMALL>(prm, pr, j, kt0 + u, ring[u]);
+        for (int kb = 0; kb < nkt; kb += kPrefetch) {
+#pragma unroll
+            for (int u = 0; u < kPrefetch; ++u) {
+                const int kt = kb + u;
+                if (kt < nkt) {
+                    if (kt + kPrefetch - 1 < nkt)
+                        load_ktile<NBITS, SMALL>(prm, pr, j, kt0 + kt + kPrefetch - 1,
+                                                 ring[(u + kPrefetch - 1) % kPrefetch]);
+                    const int s = kt % kStages;
+                    const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                    mbar_wait(empty(s), ph ^ 1u, abrt, prm.status, false);
+                    uint8_t* a = a_st + s * kABytes;
+                    const KTileCodes<NBITS, SMALL>& cur = ring[u];
+#pragma unroll
+                    for (int i = 0; i < kUnitsPerThread; ++i) {
+                        const int r = rbase + 4 * i;
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (cur.present & (1u << i))
+                            v = unit8<NBITS>(unit_merge<NBITS>(cur.raw[i]),
+                                             __high2float(cur.sz[i]), __low2float(cur.sz[i]));
+                        *reinterpret_cast<uint4*>(a + r * 128 + ((j ^ (r & 7)) << 4)) = v;
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    mbar_arrive(full_a(s));
+                }
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(full_a(s));
-            cur = nxt;
         }
-        // ---- epilogue: D[feature][token] -> Y[token][feature] in fp16
-        mbar_wait(done, 0u, abrt, prm.status, true);
+        mbar_wait(done, 0u, abrt, prm.status, true);        // every MMA of this CTA ended
         fence_after_sync();
-        const int q = warp & 3;                             // tensor-memory lane quarter
-        const int64_t nf = n0 + 32 * q + lane;
+    }
+
+    // ---- epilogue: D[feature][token] -> Y[token][feature] in fp16.  Producer
+    // warp w reads tensor-memory lanes 32 (w % 4) .. +31 (its quarter); warps
+    // 2..5 take the first half of the BN columns, warps 6..9 the second.
+    const bool epi = warp >= 2;
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int f = 32 * q + lane;                            // feature row within the tile
+    const int64_t nf = n0 + f;
+    constexpr int kHalf = BN / 2;
+    const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
+    if (ks > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
+        __syncwarp();
+        cluster.sync();                                     // rank 0's stages are free
+        if (epi && rank != 0) {
+            float* dst = cluster.map_shared_rank(red, 0) + (size_t)(rank - 1) * BN * kBM;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-            float v[16];
-            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+            for (int c0 = half * kHalf; c0 < (half + 1) * kHalf; c0 += 8) {
+                float v[8];
+                tmem_ld8(trow + (uint32_t)c0, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 8; ++i) dst[(c0 + i) * kBM + f] = v[i];
+            }
+        }
+        __syncwarp();
+        cluster.sync();                                     // every partial has arrived
+    }
+    if (epi && rank == 0) {
+#pragma unroll 1
+        for (int c0 = half * kHalf; c0 < (half + 1) * kHalf; c0 += 8) {
+            float v[8];
+            tmem_ld8(trow + (uint32_t)c0, v);
+            for (int r = 1; r < ks; ++r) {
+                const float* src = red + (size_t)(r - 1) * BN * kBM;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] += src[(c0 + i) * kBM + f];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
                 const int64_t m = m0 + c0 + i;
                 if (m < prm.M && nf < prm.N) prm.Y[m * prm.N + nf] = __float2half_rn(v[i]);
             }
@@ -376,12 +468,33 @@ cudaError_t launch_bn(const LinearParams& prm, const void* X, cudaStream_t strea
         return cudaErrorInvalidValue;
     auto kern = linear_kernel<NBITS, SMALL, BN>;
     constexpr size_t smem = linear_smem<BN>();
+    // split-k partials of up to kMaxSplit - 1 ranks fit in rank 0's stage buffers
+    static_assert(BN > 32 || (size_t)(kMaxSplit - 1) * BN * kBM * 4 <= (size_t)kStages * kABytes,
+                  "split-k buffer");
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)((prm.N + kBM - 1) / kBM), (unsigned)((prm.M + BN - 1) / BN));
-    kern<<<grid, kThreads, smem, stream>>>(map, prm);
-    return cudaGetLastError();
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t tiles_n = (prm.N + kBM - 1) / kBM, tiles_m = (prm.M + BN - 1) / BN;
+    const int KT = (int)((prm.K + kBK - 1) / kBK);
+    int ks = 1;                               // split k while the grid is short of 2 CTAs/SM
+    while (BN <= 32 && ks < kMaxSplit && tiles_n * tiles_m * ks < 2 * sms && KT >= 4 * ks)
+        ks *= 2;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 1;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = (unsigned)ks;
+    cfg.gridDim = dim3((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)ks);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, map, prm);
 }
 
 template <int NBITS, bool SMALL>

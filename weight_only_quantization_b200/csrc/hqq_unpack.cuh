@@ -56,6 +56,49 @@ __device__ __forceinline__ uint4 unit8(uint32_t x, float z, float s) {
 // and reach into word w0 + 1 when k0 > 2 (that word exists: it holds the
 // unit's own last code); words hold 10 codes in bits 0..29.  SMALL: 4u fits
 // in 32 bits, so w0 = floor(4u/5) is one multiply-high.
+// unit_bits in two steps, so that a caller can keep loads in flight: the raw
+// words of unit u (w0 and, for 3 bits, w1 and the bit shift) and their merge.
+struct UnitRaw {
+    uint32_t w0, w1, shift;
+};
+
+template <int NBITS, bool SMALL>
+__device__ __forceinline__ UnitRaw unit_fetch(const uint8_t* __restrict__ packed, int64_t u) {
+    UnitRaw r;
+    r.w1 = 0u;
+    r.shift = 0u;
+    if constexpr (NBITS == 4) {
+        r.w0 = __ldg(reinterpret_cast<const uint32_t*>(packed) + u);
+    } else if constexpr (NBITS == 2) {
+        r.w0 = __ldg(reinterpret_cast<const uint16_t*>(packed) + u);
+    } else {
+        int64_t w0;
+        uint32_t k0;
+        if (SMALL) {
+            const uint32_t u4 = 4u * (uint32_t)u;
+            const uint32_t q = __umulhi(u4, 0xCCCCCCCDu) >> 2;      // floor(u4 / 5)
+            w0 = q;
+            k0 = 2u * (u4 - 5u * q);                                 // 8u mod 10
+        } else {
+            w0 = (4 * u) / 5;
+            k0 = (uint32_t)(8 * u - 10 * w0);
+        }
+        const uint32_t* p32 = reinterpret_cast<const uint32_t*>(packed);
+        r.w0 = __ldg(p32 + w0);
+        r.w1 = k0 > 2 ? __ldg(p32 + w0 + 1) : 0u;
+        r.shift = 3u * k0;
+    }
+    return r;
+}
+
+template <int NBITS>
+__device__ __forceinline__ uint32_t unit_merge(const UnitRaw& r) {
+    if constexpr (NBITS == 3)
+        return (uint32_t)(((uint64_t)r.w0 | ((uint64_t)r.w1 << 30)) >> r.shift);
+    else
+        return r.w0;
+}
+
 template <int NBITS, bool SMALL>
 __device__ __forceinline__ uint32_t unit_bits(const uint8_t* __restrict__ packed, int64_t u) {
     if constexpr (NBITS == 4) {
