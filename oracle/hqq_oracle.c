@@ -378,14 +378,18 @@ void hqq_oracle_powp_table(float p, float *two_pk256, float *cj_p32, float *inv_
 float hqq_oracle_psum(const float *x, int n) { return psum(x, n); }
 
 /* Packing over the flat row-major element index.
+   8 bit: one code per byte.
    4 bit: two codes per byte, even index in the low nibble.
    2 bit: four codes per byte, first code in the least significant bits.
+   1 bit: eight codes per byte, first code in the least significant bit.
    3 bit: ten codes per little-endian 32-bit word in bits 0..29; bits 30..31
           and the codes past the end of the last word are zero. */
 int64_t hqq_oracle_packed_bytes(int64_t n, int nbits) {
     if (n < 0) return -1;
+    if (nbits == 8) return n;
     if (nbits == 4) return (n + 1) / 2;
     if (nbits == 2) return (n + 3) / 4;
+    if (nbits == 1) return (n + 7) / 8;
     if (nbits == 3) return 4 * ((n + 9) / 10);
     return -1;
 }
@@ -396,8 +400,12 @@ int hqq_oracle_pack(const uint8_t *codes, int64_t n, int nbits, uint8_t *out) {
     memset(out, 0, (size_t)nb);
     for (int64_t i = 0; i < n; ++i) {
         const uint32_t c = codes[i];
-        if (c >> nbits) return 4;
-        if (nbits == 4) {
+        if (nbits < 8 && (c >> nbits)) return 4;
+        if (nbits == 8) {
+            out[i] = (uint8_t)c;
+        } else if (nbits == 1) {
+            out[i / 8] |= (uint8_t)(c << (i % 8));
+        } else if (nbits == 4) {
             out[i / 2] |= (uint8_t)(c << (4 * (i % 2)));
         } else if (nbits == 2) {
             out[i / 4] |= (uint8_t)(c << (2 * (i % 4)));
@@ -414,7 +422,11 @@ int hqq_oracle_pack(const uint8_t *codes, int64_t n, int nbits, uint8_t *out) {
 int hqq_oracle_unpack(const uint8_t *packed, int64_t n, int nbits, uint8_t *codes) {
     if (hqq_oracle_packed_bytes(n, nbits) < 0) return 3;
     for (int64_t i = 0; i < n; ++i) {
-        if (nbits == 4) {
+        if (nbits == 8) {
+            codes[i] = packed[i];
+        } else if (nbits == 1) {
+            codes[i] = (packed[i / 8] >> (i % 8)) & 1u;
+        } else if (nbits == 4) {
             codes[i] = (packed[i / 2] >> (4 * (i % 2))) & 15u;
         } else if (nbits == 2) {
             codes[i] = (packed[i / 4] >> (2 * (i % 4))) & 3u;

@@ -81,7 +81,7 @@ def test_shrink_threshold_closed_form(p, beta):
 
 
 # --------------------------------------------------------------------------- P3
-@pytest.mark.parametrize("nbits,G", [(4, 64), (2, 32), (3, 64), (2, 128)])
+@pytest.mark.parametrize("nbits,G", [(4, 64), (2, 32), (3, 64), (2, 128), (8, 128), (1, 32)])
 def test_residual_within_half_step(nbits, G):
     """Section 2: Wq = round(W/s + z), W_hat = s(Wq - z).  With W_e = 0, every
     weight whose W/s + z lies in [-1/2, L + 1/2] is reconstructed within s/2."""
@@ -100,7 +100,8 @@ def test_residual_within_half_step(nbits, G):
 
 
 # --------------------------------------------------------------------------- P4
-@pytest.mark.parametrize("nbits,G", [(4, 64), (2, 32), (3, 64), (2, 128), (4, 16)])
+@pytest.mark.parametrize("nbits,G", [(4, 64), (2, 32), (3, 64), (2, 128), (4, 16), (8, 128),
+                                     (1, 64)])
 def test_error_sequence_and_early_stop(nbits, G):
     """Section 4.1: the solver runs at most 20 iterations and exits once the error
     stops improving.  Accepted errors fall strictly; the first non-decrease ends
@@ -153,7 +154,8 @@ def test_components_compose_into_the_solver():
 
 
 # --------------------------------------------------------------------------- P5
-@pytest.mark.parametrize("nbits,G", [(4, 64), (2, 32), (3, 64), (2, 128), (4, 16)])
+@pytest.mark.parametrize("nbits,G", [(4, 64), (2, 32), (3, 64), (2, 128), (4, 16), (8, 128),
+                                     (1, 64)])
 def test_zero_iterations_is_minmax_rtn(nbits, G):
     """iters = 0 is textbook asymmetric min-max round-to-nearest: scale =
     (max - min)/(2^b - 1), zero = -min/scale, code = clip(round(W/scale + zero))."""
@@ -175,7 +177,7 @@ def test_zero_iterations_is_minmax_rtn(nbits, G):
 
 
 # --------------------------------------------------------------------------- P6
-@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 8])
 def test_constant_groups_reconstruct_exactly(nbits):
     """A group with max == min has a single level; Q^-1(Q(W)) must equal W."""
     G = 32
@@ -208,7 +210,7 @@ def test_pack_golden(case):
     assert oracle.unpack(got, len(codes), nbits).tolist() == codes
 
 
-@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 8])
 def test_pack_roundtrip_all_values_and_positions(nbits):
     rng = np.random.default_rng(9)
     for n in [1, 7, 10, 31, 320, 1001]:
@@ -217,7 +219,7 @@ def test_pack_roundtrip_all_values_and_positions(nbits):
         assert pk.size == oracle.packed_bytes(n, nbits)
         assert np.array_equal(oracle.unpack(pk, n, nbits), codes)
     # every value at every slot of a word
-    per = {4: 8, 2: 16, 3: 10}[nbits]
+    per = {8: 4, 4: 8, 2: 16, 1: 32, 3: 10}[nbits]
     for v in range(2 ** nbits):
         for pos in range(per):
             codes = np.zeros(per, np.uint8)
@@ -345,7 +347,7 @@ def test_matrix_equals_independent_groups():
         assert np.float16(tr["s"]) == r["scale"][g]
 
 
-@pytest.mark.parametrize("nbits,G", [(4, 64), (2, 32), (3, 64)])
+@pytest.mark.parametrize("nbits,G", [(4, 64), (2, 32), (3, 64), (8, 128), (1, 64)])
 def test_hqq_not_worse_than_rtn(nbits, G):
     """Per group, the chosen z never has a larger l_p error than the min-max z it
     starts from (fp64 recomputation from the final codes, fp32 scale and zero)."""
