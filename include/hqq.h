@@ -39,11 +39,13 @@ typedef enum hqq_status {
     HQQ_OK = 0,
     HQQ_ERR_NULL = 1,        /* a required pointer is NULL                       */
     HQQ_ERR_SHAPE = 2,       /* rows/cols negative, cols % group != 0, too large */
-    HQQ_ERR_UNSUPPORTED = 3, /* nbits not in {2,3,4}, group not in {16..256, 2^k} */
+    HQQ_ERR_UNSUPPORTED = 3, /* nbits not in {1,2,3,4,8}, group not in {16..256,
+                                2^k}, meta group not 0 or 2^k                    */
     HQQ_ERR_PARAM = 4,       /* p not in (0,1], beta/kappa not > 0 and finite,
                                 iters not in [0,255]                             */
-    HQQ_ERR_ALIGN = 5,       /* W / W_out not 16-byte aligned; packed, zero_f32
-                                or err_out not 4-byte; scale/zero not 2-byte     */
+    HQQ_ERR_ALIGN = 5,       /* W / W_out / X not 16-byte aligned; packed not
+                                4-byte (8-byte at 8 bits); zero_f32 or err_out
+                                not 4-byte; scale/zero not 2-byte                */
     HQQ_ERR_CUDA = 6         /* the kernel launch failed                         */
 } hqq_status;
 
@@ -55,12 +57,15 @@ typedef enum hqq_status {
 
 /*
  * Packed code layout (over the flat row-major element index i):
+ *   nbits 8: byte  i    holds code i
  *   nbits 4: byte  i/2  holds code i in bits 4*(i%2)   (even index = low nibble)
  *   nbits 2: byte  i/4  holds code i in bits 2*(i%4)   (first code = lowest bits)
+ *   nbits 1: byte  i/8  holds code i in bit  i%8       (first code = lowest bit)
  *   nbits 3: little-endian uint32 word i/10 holds code i in bits 3*(i%10);
  *            bits 30..31 and the slots past the last code are zero.
  * Returns the byte size of the packed buffer for rows*cols codes
- * (4 bit: N/2, 2 bit: N/4, 3 bit: 4*ceil(N/10)), or -1 for bad arguments.
+ * (8 bit: N, 4 bit: ceil(N/2), 2 bit: ceil(N/4), 1 bit: ceil(N/8),
+ * 3 bit: 4*ceil(N/10)), or -1 for bad arguments.
  */
 int64_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits);
 
@@ -81,12 +86,14 @@ int64_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits);
  *
  *   W        [in]  fp16 [rows, cols] row-major, 16-byte aligned.
  *   rows     [in]  output features (>= 0).  cols: input features (>= 0).
- *   nbits    [in]  2, 3 or 4.
+ *   nbits    [in]  1, 2, 3, 4 or 8 (section 4.1's table has 8/4/3/2; 1 bit
+ *                  is the same operator with two levels).
  *   group    [in]  16, 32, 64, 128 or 256; cols % group == 0.
  *   p, beta, kappa, iters [in]  solver parameters (0 < p <= 1, beta > 0,
  *                  kappa > 0, 0 <= iters <= 255; iters = 0 gives min-max
  *                  round-to-nearest).
- *   packed   [out] hqq_packed_bytes(rows, cols, nbits) bytes, 4-byte aligned.
+ *   packed   [out] hqq_packed_bytes(rows, cols, nbits) bytes, 4-byte aligned
+ *                  (8-byte aligned at 8 bits).
  *   scale    [out] fp16 [rows, cols/group]: s of each group (multiply to
  *                  dequantize), 2-byte aligned.
  *   zero     [out] fp16 [rows, cols/group]: z_best of each group.
@@ -117,7 +124,7 @@ int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nbits, int gr
  * hqq_dequantize -- Q^-1 of the method's section 2: W_hat = s (Wq - z), computed
  * as fp16( (code - z) * s ) in binary32 from the stored fp16 s and z.
  *
- *   packed [in]  codes in the layout above, 4-byte aligned.
+ *   packed [in]  codes in the layout above, 4-byte aligned (8 at 8 bits).
  *   scale, zero [in] fp16 [rows, cols/group], 2-byte aligned.
  *   rows, cols, nbits, group [in] as for hqq_quantize.
  *   W_out  [out] fp16 [rows, cols] row-major, 16-byte aligned.

@@ -86,12 +86,10 @@ def group_codes(packed, nbits, group, g_idx):
     out = np.empty((g_idx.size, group), np.uint8)
     for k, g in enumerate(g_idx):
         e0 = int(g) * group
-        if nbits == 4:
-            b = packed[e0 // 2:(e0 + group) // 2]
-            out[k] = oracle.unpack(b, group, 4)
-        elif nbits == 2:
-            b = packed[e0 // 4:(e0 + group) // 4]
-            out[k] = oracle.unpack(b, group, 2)
+        if nbits in (8, 4, 2, 1):                 # groups are whole bytes (8 | group)
+            per = 8 // nbits
+            b = packed[e0 // per:(e0 + group) // per]
+            out[k] = oracle.unpack(b, group, nbits)
         else:
             w0, w1 = e0 // 10, (e0 + group - 1) // 10
             b = packed[4 * w0:4 * (w1 + 1)]

@@ -61,6 +61,9 @@ def test_packed_bytes(lib):
     assert lib.hqq_packed_bytes(1, 64, 3) == 28
     assert lib._lib.hqq_packed_bytes(-1, 64, 4) == -1
     assert lib._lib.hqq_packed_bytes(4, 64, 5) == -1
+    assert lib.hqq_packed_bytes(4096, 4096, 8) == 4096 * 4096
+    assert lib.hqq_packed_bytes(3, 7, 1) == 3
+    assert lib.hqq_packed_bytes(4096, 4096, 1) == 4096 * 4096 // 8
 
 
 def test_status_strings(lib):
@@ -74,7 +77,7 @@ def test_host_validation_without_gpu(lib):
     P = lambda v: ctypes.c_void_p(v)
     a = dict(rows=64, cols=256, nbits=4, group=64, p=0.7, beta=1.0, kappa=1.01, iters=20)
     cases = [
-        (dict(nbits=5), 3), (dict(nbits=1), 3), (dict(group=48), 3), (dict(group=8), 3),
+        (dict(nbits=5), 3), (dict(nbits=0), 3), (dict(nbits=6), 3), (dict(group=48), 3), (dict(group=8), 3),
         (dict(group=512), 3), (dict(cols=250), 2), (dict(rows=-3), 2),
         (dict(p=0.0), 4), (dict(p=1.0001), 4), (dict(p=float("nan")), 4),
         (dict(beta=0.0), 4), (dict(beta=float("inf")), 4), (dict(kappa=0.0), 4),

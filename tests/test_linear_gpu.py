@@ -54,7 +54,8 @@ def _check(Y_gpu, X, Wh, label):
     return float((err / tol).max())
 
 
-@pytest.mark.parametrize("nbits,group", [(4, 64), (3, 64), (2, 32), (4, 128), (2, 16), (3, 256)])
+@pytest.mark.parametrize("nbits,group", [(4, 64), (3, 64), (2, 32), (4, 128), (2, 16), (3, 256),
+                                         (8, 128), (1, 64)])
 @pytest.mark.parametrize("M", [1, 16, 100, 256])
 def test_linear_formats_and_token_counts(hqq, nbits, group, M):
     rows, cols = 256, 1024

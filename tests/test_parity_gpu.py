@@ -48,7 +48,7 @@ def test_c2_4096(hqq, nbits, group):
 
 
 # ------------------------------------------------- every width x group, ragged
-@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 8])
 @pytest.mark.parametrize("group", [16, 32, 64, 128, 256])
 def test_all_formats_ragged(hqq, nbits, group):
     # 37 rows x 13 groups: not a multiple of a CTA tile nor of 5 groups (3-bit words)
@@ -58,7 +58,7 @@ def test_all_formats_ragged(hqq, nbits, group):
 
 
 @pytest.mark.parametrize("shape", [(1, 64), (1, 128), (3, 64), (1, 640), (5, 192)])
-@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 8])
 def test_odd_shapes(hqq, shape, nbits):
     W, Wn = _dev_weights(shape, seed=22, stream=shape[0] * 7 + shape[1])
     _check(hqq, W, Wn, nbits, 64, f"shape {shape} {nbits}b")
@@ -94,7 +94,7 @@ def _adversarial(G):
     return np.array(rows, np.float64).astype(np.float16)
 
 
-@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 8])
 @pytest.mark.parametrize("group", [16, 64, 128])
 def test_adversarial_groups(hqq, nbits, group):
     Wn = _adversarial(group)
@@ -103,7 +103,7 @@ def test_adversarial_groups(hqq, nbits, group):
 
 
 # ------------------------------------------------- sp1 active: unit-scale weights
-@pytest.mark.parametrize("nbits,group", [(4, 64), (2, 32), (3, 64), (2, 128)])
+@pytest.mark.parametrize("nbits,group", [(4, 64), (2, 32), (3, 64), (2, 128), (8, 128), (1, 64)])
 @pytest.mark.parametrize("std", [1.0, 3.0])
 def test_shrink_active(hqq, nbits, group, std):
     W, Wn = _dev_weights((256, 1024), seed=24, stream=group, std=std)
@@ -124,7 +124,7 @@ def test_solver_parameters(hqq, kw):
 
 
 # ------------------------------------------------------------------ dequantize
-@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 8])
 @pytest.mark.parametrize("group", [16, 32, 64, 128, 256])
 def test_dequantize_bitwise(hqq, nbits, group):
     W, Wn = _dev_weights((29, 7 * group), seed=26, stream=group + nbits)
@@ -147,6 +147,8 @@ FULL = [
     ("70B down 8192x28672 3b g64", (8192, 28672), 3, 64, 5, 6),
     ("7B up 11008x4096 4b g64", (11008, 4096), 4, 64, 2, 5),
     ("7B down 4096x11008 4b g64", (4096, 11008), 4, 64, 2, 6),
+    ("8192x8192 8b g128", (8192, 8192), 8, 128, 7, 0),
+    ("8192x8192 1b g64", (8192, 8192), 1, 64, 7, 1),
 ]
 
 
@@ -243,7 +245,7 @@ def test_repeat_calls_are_deterministic(hqq):
 
 
 # ------------------------------- several chunks per warp (group carry-over path)
-@pytest.mark.parametrize("nbits", [4, 3, 2])
+@pytest.mark.parametrize("nbits", [8, 4, 3, 2, 1])
 @pytest.mark.parametrize("group", [16, 32, 64, 128, 256])
 def test_multi_chunk_per_warp(hqq, nbits, group):
     # 16.8 M weights = 6554 chunks of 2560: more than one chunk per resident warp,

@@ -73,7 +73,7 @@ def hqq_status_string(status: int) -> str:
 def hqq_packed_bytes(rows: int, cols: int, nbits: int) -> int:
     n = _lib.hqq_packed_bytes(rows, cols, nbits)
     if n < 0:
-        raise HQQError(2 if nbits in (2, 3, 4) else 3)
+        raise HQQError(2 if nbits in (1, 2, 3, 4, 8) else 3)
     return int(n)
 
 

@@ -72,6 +72,10 @@ struct TableCache {
 };
 thread_local TableCache g_cache;
 
+// Alignment of the packed codes: the kernels move 8-bit units as 8-byte words,
+// the other widths in units of at most 4 bytes.
+uintptr_t packed_align(int nbits) { return nbits == 8 ? 8 : 4; }
+
 // log2 of a second-level (meta) group: -1 for 0 (one group over everything),
 // -2 when the size is not a power of two up to 2^30.
 int meta_log2(int64_t mgroup) {
@@ -83,7 +87,8 @@ int meta_log2(int64_t mgroup) {
 
 int validate_common(int64_t rows, int64_t cols, int nbits, int group) {
     if (rows < 0 || cols < 0) return HQQ_ERR_SHAPE;
-    if (nbits != 2 && nbits != 3 && nbits != 4) return HQQ_ERR_UNSUPPORTED;
+    if (nbits != 1 && nbits != 2 && nbits != 3 && nbits != 4 && nbits != 8)
+        return HQQ_ERR_UNSUPPORTED;
     if (log2_of_group(group) < 0) return HQQ_ERR_UNSUPPORTED;
     if (cols % group != 0) return HQQ_ERR_SHAPE;
     if (rows > 0 && cols > ((int64_t)1 << 46) / rows) return HQQ_ERR_SHAPE;
@@ -100,8 +105,10 @@ extern "C" int64_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits) {
     if (rows > 0 && cols > ((int64_t)1 << 46) / rows) return -1;
     const int64_t n = rows * cols;
     switch (nbits) {
+        case 8: return n;
         case 4: return (n + 1) / 2;
         case 2: return (n + 3) / 4;
+        case 1: return (n + 7) / 8;
         case 3: return 4 * ((n + 9) / 10);
         default: return -1;
     }
@@ -112,9 +119,9 @@ extern "C" const char* hqq_status_string(int status) {
         case HQQ_OK: return "HQQ_OK";
         case HQQ_ERR_NULL: return "HQQ_ERR_NULL: a required pointer is NULL";
         case HQQ_ERR_SHAPE: return "HQQ_ERR_SHAPE: bad rows/cols or cols not a multiple of group";
-        case HQQ_ERR_UNSUPPORTED: return "HQQ_ERR_UNSUPPORTED: nbits must be 2/3/4, group 16..256 (power of two), meta group 0 or a power of two up to 2^30";
+        case HQQ_ERR_UNSUPPORTED: return "HQQ_ERR_UNSUPPORTED: nbits must be 1/2/3/4/8, group 16..256 (power of two), meta group 0 or a power of two up to 2^30";
         case HQQ_ERR_PARAM: return "HQQ_ERR_PARAM: need 0<p<=1, beta>0, kappa>0 (finite), 0<=iters<=255";
-        case HQQ_ERR_ALIGN: return "HQQ_ERR_ALIGN: W/W_out/meta x/meta out need 16-byte, meta codes 8-byte, packed/zero_f32 4-byte, scale/zero 2-byte alignment";
+        case HQQ_ERR_ALIGN: return "HQQ_ERR_ALIGN: W/W_out/X/meta x/meta out need 16-byte, meta codes and 8-bit packed 8-byte, packed/zero_f32 4-byte, scale/zero 2-byte alignment";
         case HQQ_ERR_CUDA: return "HQQ_ERR_CUDA: kernel launch failed (see cudaGetLastError)";
         default: return "HQQ: unknown status";
     }
@@ -133,8 +140,9 @@ extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nb
     const int64_t n = rows * cols;
     if (n == 0) return HQQ_OK;
     if (!W || !packed || !scale || !zero) return HQQ_ERR_NULL;
-    if (!aligned(W, 16) || !aligned(packed, 4) || !aligned(scale, 2) || !aligned(zero, 2) ||
-        (zero_f32 && !aligned(zero_f32, 4)) || (err_out && !aligned(err_out, 4)))
+    if (!aligned(W, 16) || !aligned(packed, packed_align(nbits)) || !aligned(scale, 2) ||
+        !aligned(zero, 2) || (zero_f32 && !aligned(zero_f32, 4)) ||
+        (err_out && !aligned(err_out, 4)))
         return HQQ_ERR_ALIGN;
 
     QuantParams prm;
@@ -192,7 +200,8 @@ extern "C" int hqq_dequantize(const void* packed, const void* scale, const void*
     const int64_t n = rows * cols;
     if (n == 0) return HQQ_OK;
     if (!packed || !scale || !zero || !W_out) return HQQ_ERR_NULL;
-    if (!aligned(packed, 4) || !aligned(scale, 2) || !aligned(zero, 2) || !aligned(W_out, 16))
+    if (!aligned(packed, packed_align(nbits)) || !aligned(scale, 2) || !aligned(zero, 2) ||
+        !aligned(W_out, 16))
         return HQQ_ERR_ALIGN;
     DequantParams prm;
     std::memset(&prm, 0, sizeof prm);
@@ -273,7 +282,8 @@ extern "C" int hqq_dequantize_meta(const void* packed, const hqq_meta8* zero_q, 
     std::memset(&prm, 0, sizeof prm);
     if ((st = meta8_image(zero_q, prm.zq)) != HQQ_OK) return st;
     if (scale_q && (st = meta8_image(scale_q, prm.sq)) != HQQ_OK) return st;
-    if (!aligned(packed, 4) || !aligned(W_out, 16) || (scale && !aligned(scale, 2)))
+    if (!aligned(packed, packed_align(nbits)) || !aligned(W_out, 16) ||
+        (scale && !aligned(scale, 2)))
         return HQQ_ERR_ALIGN;
     prm.packed = static_cast<const uint8_t*>(packed);
     prm.scale = static_cast<const __half*>(scale);
@@ -294,8 +304,8 @@ extern "C" int hqq_linear(const void* X, int64_t M, const void* packed, const vo
     if (M < 0 || M > (int64_t)65535 * 256) return HQQ_ERR_SHAPE;
     if (M == 0 || rows == 0 || cols == 0) return HQQ_OK;
     if (!X || !packed || !scale || !zero || !Y) return HQQ_ERR_NULL;
-    if (!aligned(X, 16) || !aligned(packed, 4) || !aligned(scale, 2) || !aligned(zero, 2) ||
-        !aligned(Y, 2) || (status && !aligned(status, 4)))
+    if (!aligned(X, 16) || !aligned(packed, packed_align(nbits)) || !aligned(scale, 2) ||
+        !aligned(zero, 2) || !aligned(Y, 2) || (status && !aligned(status, 4)))
         return HQQ_ERR_ALIGN;
     LinearParams prm;
     std::memset(&prm, 0, sizeof prm);

@@ -34,7 +34,9 @@ __global__ void __launch_bounds__(kDqThreads)
 dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
     for (int64_t base = (int64_t)blockIdx.x * kDqTile; base < prm.n_units;
          base += (int64_t)gridDim.x * kDqTile) {
+        // 8-bit units are 64 bits (fetched raw); narrower ones one word
         uint32_t x[kDqUnits];
+        UnitRaw x8[NBITS == 8 ? kDqUnits : 1];
         float sf[kDqUnits], zf[kDqUnits];
 #pragma unroll
         for (int r = 0; r < kDqUnits; ++r) {        // all loads first
@@ -43,12 +45,19 @@ dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
             const int64_t g = (u * 8) >> log2_group;
             sf[r] = (META & 2) ? restore_meta(prm.sq, g) : __half2float(__ldg(prm.scale + g));
             zf[r] = (META & 1) ? restore_meta(prm.zq, g) : __half2float(__ldg(prm.zero + g));
-            x[r] = unit_bits<NBITS, SMALL>(prm.packed, u);
+            if constexpr (NBITS == 8)
+                x8[r] = unit_fetch<8, SMALL>(prm.packed, u);
+            else
+                x[r] = unit_bits<NBITS, SMALL>(prm.packed, u);
         }
 #pragma unroll
         for (int r = 0; r < kDqUnits; ++r) {
             const int64_t u = base + r * kDqThreads + threadIdx.x;
-            const uint4 o = unit8<NBITS>(x[r], zf[r], sf[r]);
+            uint4 o;
+            if constexpr (NBITS == 8)
+                o = unit8_raw<8>(x8[r], zf[r], sf[r]);
+            else
+                o = unit8<NBITS>(x[r], zf[r], sf[r]);
             if (u < prm.n_units) reinterpret_cast<uint4*>(prm.out)[u] = o;
         }
     }
@@ -76,8 +85,10 @@ cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_grou
     const bool small = prm.n_units < ((int64_t)1 << 30);
     const unsigned g = (unsigned)blocks;
     switch (nbits) {
+        case 1: launch_dq<1, true>(prm, log2_group, g, stream); break;
         case 2: launch_dq<2, true>(prm, log2_group, g, stream); break;
         case 4: launch_dq<4, true>(prm, log2_group, g, stream); break;
+        case 8: launch_dq<8, true>(prm, log2_group, g, stream); break;
         case 3:
             if (small) launch_dq<3, true>(prm, log2_group, g, stream);
             else launch_dq<3, false>(prm, log2_group, g, stream);

@@ -359,8 +359,8 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
                         const int r = rbase + 4 * i;
                         uint4 v = make_uint4(0u, 0u, 0u, 0u);
                         if (cur.present & (1u << i))
-                            v = unit8<NBITS>(unit_merge<NBITS>(cur.raw[i]),
-                                             __high2float(cur.sz[i]), __low2float(cur.sz[i]));
+                            v = unit8_raw<NBITS>(cur.raw[i], __high2float(cur.sz[i]),
+                                                 __low2float(cur.sz[i]));
                         *reinterpret_cast<uint4*>(a + r * 128 + ((j ^ (r & 7)) << 4)) = v;
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -511,8 +511,10 @@ cudaError_t launch_nb(const LinearParams& prm, const void* X, cudaStream_t strea
 cudaError_t launch_linear(const LinearParams& prm, const void* X, int nbits, cudaStream_t stream) {
     const bool small = prm.N * prm.K / 8 < ((int64_t)1 << 30);
     switch (nbits) {
+        case 1: return launch_nb<1, true>(prm, X, stream);
         case 2: return launch_nb<2, true>(prm, X, stream);
         case 4: return launch_nb<4, true>(prm, X, stream);
+        case 8: return launch_nb<8, true>(prm, X, stream);
         case 3:
             return small ? launch_nb<3, true>(prm, X, stream) : launch_nb<3, false>(prm, X, stream);
         default: return cudaErrorInvalidValue;

@@ -344,10 +344,21 @@ __device__ __forceinline__ void finalize_direct(const QuantParams& prm, const fl
         for (int b = 0; b < NB; ++b) {
             const int64_t unit = gi * (G / 8) + kl * NB + b;
             uint32_t word = 0;
+            if constexpr (NBITS == 8) {
+                uint2 bb;
+                bb.x = c[b][0] | (c[b][1] << 8) | (c[b][2] << 16) | (c[b][3] << 24);
+                bb.y = c[b][4] | (c[b][5] << 8) | (c[b][6] << 16) | (c[b][7] << 24);
+                reinterpret_cast<uint2*>(prm.packed)[unit] = bb;
+            } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) word |= c[b][i] << (NBITS * i);
-            if constexpr (NBITS == 4) reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
-            else reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)word;
+                for (int i = 0; i < 8; ++i) word |= c[b][i] << (NBITS * i);
+                if constexpr (NBITS == 4)
+                    reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
+                else if constexpr (NBITS == 2)
+                    reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)word;
+                else
+                    prm.packed[unit] = (uint8_t)word;
+            }
         }
     }
     if (kl == 0) {
@@ -360,8 +371,8 @@ __device__ __forceinline__ void finalize_direct(const QuantParams& prm, const fl
 }
 
 // Final codes of every group of a chunk (one uniform pass, phase-A layout),
-// from the staged weights and each group's (z_best, 1/s); 4 and 2 bit codes
-// are stored straight to HBM, 3 bit code bytes overwrite the front of the
+// from the staged weights and each group's (z_best, 1/s); 8, 4, 2 and 1 bit
+// codes are stored straight to HBM, 3 bit code bytes overwrite the front of the
 // chunk's weight buffer (round r writes bytes [512r, 512r+512), never ahead of
 // the weights still to be read) for word packing.  Scale, zero and the
 // diagnostics are written by each group's first lane.
@@ -417,6 +428,16 @@ __device__ __forceinline__ void final_pass(const QuantParams& prm, __half* s_w, 
 #pragma unroll
                 for (int i = 0; i < 8; ++i) h |= c[i] << (2 * i);
                 reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)h;
+            } else if constexpr (NBITS == 1) {
+                uint32_t h = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) h |= c[i] << i;
+                prm.packed[unit] = (uint8_t)h;
+            } else if constexpr (NBITS == 8) {
+                uint2 bb;
+                bb.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+                bb.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+                reinterpret_cast<uint2*>(prm.packed)[unit] = bb;
             } else {
                 uint2 bb;
                 bb.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
@@ -695,9 +716,11 @@ static cudaError_t launch_quantize_b(const QuantParams& prm, int group, cudaStre
 
 cudaError_t launch_quantize(const QuantParams& prm, int nbits, int group, cudaStream_t stream) {
     switch (nbits) {
+        case 1: return launch_quantize_b<1>(prm, group, stream);
         case 2: return launch_quantize_b<2>(prm, group, stream);
         case 3: return launch_quantize_b<3>(prm, group, stream);
         case 4: return launch_quantize_b<4>(prm, group, stream);
+        case 8: return launch_quantize_b<8>(prm, group, stream);
         default: return cudaErrorInvalidValue;
     }
 }

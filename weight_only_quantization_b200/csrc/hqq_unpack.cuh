@@ -67,7 +67,13 @@ __device__ __forceinline__ UnitRaw unit_fetch(const uint8_t* __restrict__ packed
     UnitRaw r;
     r.w1 = 0u;
     r.shift = 0u;
-    if constexpr (NBITS == 4) {
+    if constexpr (NBITS == 8) {                       // 8 bytes: w0 codes 0..3, w1 codes 4..7
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(packed) + u);
+        r.w0 = v.x;
+        r.w1 = v.y;
+    } else if constexpr (NBITS == 1) {
+        r.w0 = __ldg(packed + u);
+    } else if constexpr (NBITS == 4) {
         r.w0 = __ldg(reinterpret_cast<const uint32_t*>(packed) + u);
     } else if constexpr (NBITS == 2) {
         r.w0 = __ldg(reinterpret_cast<const uint16_t*>(packed) + u);
@@ -99,9 +105,39 @@ __device__ __forceinline__ uint32_t unit_merge(const UnitRaw& r) {
         return r.w0;
 }
 
+// Eight 8-bit codes (bytes of w0 then w1) -> fp16((c - z) s).  Byte i becomes
+// the mantissa of 2^23 by one byte permute; subtracting 2^23 is exact.
+__device__ __forceinline__ uint4 unit8_bytes(uint32_t w0, uint32_t w1, float z, float s) {
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t w = j < 2 ? w0 : w1;
+        const int b0 = 2 * (j & 1), b1 = b0 + 1;
+        // result bytes: (code, 0x00, 0x00, 0x4B) from (w, 0x4B000000)
+        const float2 f = make_float2(
+            __uint_as_float(__byte_perm(w, 0x4B000000u, (uint32_t)b0 | 0x7440u)),
+            __uint_as_float(__byte_perm(w, 0x4B000000u, (uint32_t)b1 | 0x7440u)));
+        const float2 c = __fadd2_rn(f, make_float2(-8388608.0f, -8388608.0f));
+        o[j] = dq2(c, z, s);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The eight weights of a fetched unit, for every width.
+template <int NBITS>
+__device__ __forceinline__ uint4 unit8_raw(const UnitRaw& r, float z, float s) {
+    if constexpr (NBITS == 8)
+        return unit8_bytes(r.w0, r.w1, z, s);
+    else
+        return unit8<NBITS>(unit_merge<NBITS>(r), z, s);
+}
+
 template <int NBITS, bool SMALL>
 __device__ __forceinline__ uint32_t unit_bits(const uint8_t* __restrict__ packed, int64_t u) {
-    if constexpr (NBITS == 4) {
+    static_assert(NBITS != 8, "8-bit units are 64 bits: use unit_fetch and unit8_raw");
+    if constexpr (NBITS == 1) {
+        return __ldg(packed + u);
+    } else if constexpr (NBITS == 4) {
         return __ldg(reinterpret_cast<const uint32_t*>(packed) + u);
     } else if constexpr (NBITS == 2) {
         return __ldg(reinterpret_cast<const uint16_t*>(packed) + u);
