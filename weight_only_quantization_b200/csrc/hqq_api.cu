@@ -11,16 +11,8 @@ namespace hqq {
 cudaError_t launch_quantize(const QuantParams& prm, int nbits, int group, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_group,
                               cudaStream_t stream);
-struct LinearParams {
-    const uint8_t* packed;
-    const __half* scale;
-    const __half* zero;
-    __half* Y;
-    int* status;
-    int64_t M, N, K;
-    int log2_group;
-};
 cudaError_t launch_linear(const LinearParams& prm, const void* X, int nbits, cudaStream_t stream);
+cudaError_t launch_gemv(const LinearParams& prm, const void* X, int nbits, cudaStream_t stream);
 cudaError_t launch_meta_quantize(const __half* x, int64_t n, int log2g, uint8_t* codes,
                                  __half* scale, __half* zero, cudaStream_t stream);
 cudaError_t launch_meta_dequantize(const uint8_t* codes, const __half* scale, const __half* zero,
@@ -318,6 +310,9 @@ extern "C" int hqq_linear(const void* X, int64_t M, const void* packed, const vo
     prm.N = rows;
     prm.K = cols;
     prm.log2_group = log2_of_group(group);
-    const cudaError_t err = launch_linear(prm, X, nbits, static_cast<cudaStream_t>(stream));
+    // up to 8 tokens: streaming kernel on the CUDA cores; more: tensor cores
+    const cudaError_t err = M <= 8
+        ? launch_gemv(prm, X, nbits, static_cast<cudaStream_t>(stream))
+        : launch_linear(prm, X, nbits, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }

@@ -58,6 +58,17 @@ struct Meta8 {
     int shift;
 };
 
+// Weight-only linear layer Y = X W_hat^T on a quantized [N, K] matrix.
+struct LinearParams {
+    const uint8_t* packed;
+    const __half* scale;
+    const __half* zero;
+    __half* Y;
+    int* status;             // optional: set to 1 if a wait inside a kernel ran out
+    int64_t M, N, K;         // tokens, output features, input features
+    int log2_group;
+};
+
 struct DequantParams {
     const uint8_t* packed;
     const __half* scale;   // fp16 scales, unless given in 8-bit form (sq)

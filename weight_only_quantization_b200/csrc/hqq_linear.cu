@@ -155,72 +155,124 @@ __device__ __forceinline__ void fence_after_sync() {
 
 }  // namespace
 
-struct LinearParams {
-    const uint8_t* packed;
-    const __half* scale;
-    const __half* zero;
-    __half* Y;
-    int* status;             // optional: set to 1 if a wait ran out
-    int64_t M, N, K;
-    int log2_group;
-};
 
 namespace {
 
 constexpr int kProducerWarps = 8;                     // warps 2..9
 constexpr int kProducers = kProducerWarps * 32;
-constexpr int kUnitsPerThread = kBM * (kBK / 8) / kProducers;   // 4
+constexpr int kUnitsPerThread = kBM * (kBK / 8) / kProducers;   // 4: one quad
+static_assert(kUnitsPerThread == 4, "one quad of units per producer thread and k-tile");
 constexpr int kMaxSplit = 4;                          // k-slices per cluster (decode shapes)
 
-// The units one producer thread writes per k-tile: unit column j = lane % 8 of
-// tile rows pw*16 + lane/8 + 4i (i < 4).  The 8 lanes of a row read that row's
-// codes for the k-tile as one contiguous run (24 bytes at 3 bits), so a warp
-// load touches 4 rows, not 32.
-template <int NBITS, bool SMALL>
-struct KTileCodes {
-    UnitRaw raw[kUnitsPerThread];                     // loaded words, merged at use
-    __half2 sz[kUnitsPerThread];                      // (s, z) of each unit's group
-    uint32_t present;                                 // bit i: unit i lies inside the matrix
+// The units one producer thread writes per k-tile: a quad of 4 consecutive
+// units (32 codes) of one row, units 4 (lane % 2) .. +3 of tile row
+// pw*16 + lane/2.  A quad's codes are one vector load (VEC: 4, 8, 16 or 32
+// bytes at 1, 2, 4 or 8 bits; four 32-bit words at 3 bits) and its group data
+// one (scale, zero) pair (two for groups of 16).
+template <int NBITS>
+struct QuadCodes {
+    static constexpr int NW = NBITS == 3 ? 4 : NBITS;     // 32-bit words of codes
+    uint32_t w[NW];
+    __half2 sz[2];                                     // (s, z) of units 0-1 and 2-3
+    uint32_t off;                                      // 3 bits: slot of code 0 in w[0]
+    uint32_t present;                                  // bit t: unit t inside the matrix
 };
 
-// Per-thread constants of the producer: the unit index (of the flat code
-// stream) and the group index of its four rows at k = 0.  Rows past N hold
-// no unit.
-struct ProducerRows {
-    int64_t u0[kUnitsPerThread];
-    int64_t g0[kUnitsPerThread];
-    uint32_t row_ok;                                  // bit i: row i inside the matrix
-};
-
-__device__ __forceinline__ void producer_rows(const LinearParams& p, int64_t row0, int j,
-                                              ProducerRows& pr) {
-    pr.row_ok = 0u;
+template <int NBITS, bool SMALL, bool VEC>
+__device__ __forceinline__ void load_quad(const LinearParams& p, int64_t fbase, bool row_ok,
+                                          int64_t kq, QuadCodes<NBITS>& c) {
+    // fbase: flat index of the row's first code; kq: k of the quad's first code
+    c.present = 0u;
+    c.off = 0u;
 #pragma unroll
-    for (int i = 0; i < kUnitsPerThread; ++i) {
-        const int64_t n = row0 + 4 * i;
-        pr.u0[i] = (n * p.K) / 8 + j;
-        pr.g0[i] = (n * p.K) >> p.log2_group;
-        if (n < p.N) pr.row_ok |= 1u << i;
+    for (int i = 0; i < QuadCodes<NBITS>::NW; ++i) c.w[i] = 0u;
+    c.sz[0] = c.sz[1] = __float2half2_rn(0.0f);
+    if (!row_ok || kq >= p.K) return;
+    const int64_t f = fbase + kq;
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+        if (kq + 8 * t < p.K) c.present |= 1u << t;
+    if constexpr (NBITS == 3) {
+        const int64_t u = f >> 3;
+        int64_t w0;
+        if (SMALL) {
+            const uint32_t u4 = 4u * (uint32_t)u;
+            w0 = __umulhi(u4, 0xCCCCCCCDu) >> 2;         // floor(f / 10)
+        } else {
+            w0 = (4 * u) / 5;
+        }
+        c.off = (uint32_t)(f - 10 * w0);
+        // slots off .. off + 8 * (present units) - 1 (< 40): only the words they
+        // touch are read, so a partial quad at the end stays inside the buffer
+        const uint32_t slots = c.off + 8u * (uint32_t)__popc(c.present);
+        const uint32_t* p32 = reinterpret_cast<const uint32_t*>(p.packed) + w0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (10u * i < slots) c.w[i] = __ldg(p32 + i);
+    } else if constexpr (VEC) {
+        const uint8_t* src = p.packed + (f >> 5) * (4 * NBITS);
+        if constexpr (NBITS == 8) {
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+            const uint4 b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+            c.w[0] = a.x; c.w[1] = a.y; c.w[2] = a.z; c.w[3] = a.w;
+            c.w[4] = b.x; c.w[5] = b.y; c.w[6] = b.z; c.w[7] = b.w;
+        } else if constexpr (NBITS == 4) {
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+            c.w[0] = a.x; c.w[1] = a.y; c.w[2] = a.z; c.w[3] = a.w;
+        } else if constexpr (NBITS == 2) {
+            const uint2 a = __ldg(reinterpret_cast<const uint2*>(src));
+            c.w[0] = a.x; c.w[1] = a.y;
+        } else {
+            c.w[0] = __ldg(reinterpret_cast<const uint32_t*>(src));
+        }
+    } else {                                           // unit by unit (any k alignment)
+        const int64_t u = f >> 3;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            if (!(c.present & (1u << t))) continue;
+            const UnitRaw r = unit_fetch<NBITS, SMALL>(p.packed, u + t);
+            if constexpr (NBITS == 8) {
+                c.w[2 * t] = r.w0;
+                c.w[2 * t + 1] = r.w1;
+            } else if constexpr (NBITS == 4) {
+                c.w[t] = r.w0;
+            } else if constexpr (NBITS == 2) {
+                c.w[t >> 1] |= r.w0 << (16 * (t & 1));
+            } else {
+                c.w[0] |= r.w0 << (8 * t);
+            }
+        }
     }
+    const int64_t g = f >> p.log2_group;
+    c.sz[0] = __halves2half2(__ldg(p.scale + g), __ldg(p.zero + g));
+    c.sz[1] = c.sz[0];
+    if (p.log2_group == 4 && (c.present & 4u))
+        c.sz[1] = __halves2half2(__ldg(p.scale + g + 1), __ldg(p.zero + g + 1));
 }
 
-template <int NBITS, bool SMALL>
-__device__ __forceinline__ void load_ktile(const LinearParams& p, const ProducerRows& pr, int j,
-                                           int kt, KTileCodes<NBITS, SMALL>& c) {
-    const int64_t kk = (int64_t)kt * kBK + 8 * j;
-    c.present = kk < p.K ? pr.row_ok : 0u;
-    const int64_t du = (int64_t)kt * (kBK / 8);
-    const int64_t dg = kk >> p.log2_group;
-#pragma unroll
-    for (int i = 0; i < kUnitsPerThread; ++i) {
-        if (c.present & (1u << i)) {
-            const int64_t g = pr.g0[i] + dg;
-            c.raw[i] = unit_fetch<NBITS, SMALL>(p.packed, pr.u0[i] + du);
-            c.sz[i] = __halves2half2(__ldg(p.scale + g), __ldg(p.zero + g));
-        } else {
-            c.raw[i].w0 = c.raw[i].w1 = c.raw[i].shift = 0u;
-            c.sz[i] = __float2half2_rn(0.0f);
-        }
+// Weights of unit t (0..3) of a loaded quad.
+template <int NBITS>
+__device__ __forceinline__ uint4 quad_unit(const QuadCodes<NBITS>& c, int t) {
+    const __half2 sz = c.sz[t >> 1];
+    const float s = __low2float(sz), z = __high2float(sz);
+    if constexpr (NBITS == 8) {
+        return unit8_bytes(c.w[2 * t], c.w[2 * t + 1], z, s);
+    } else if constexpr (NBITS == 4) {
+        return unit8<4>(c.w[t], z, s);
+    } else if constexpr (NBITS == 2) {
+        return unit8<2>((c.w[t >> 1] >> (16 * (t & 1))) & 0xFFFFu, z, s);
+    } else if constexpr (NBITS == 1) {
+        return unit8<1>((c.w[0] >> (8 * t)) & 0xFFu, z, s);
+    } else {
+        // the 30-bit fields of the four words as two 60-bit runs
+        const uint64_t A = (uint64_t)c.w[0] | ((uint64_t)c.w[1] << 30);
+        const uint64_t B = (uint64_t)c.w[2] | ((uint64_t)c.w[3] << 30);
+        const uint32_t pos = 3u * (c.off + 8u * (uint32_t)t);   // bit of code 8t
+        uint64_t v;
+        if (pos + 24u <= 60u) v = A >> pos;
+        else if (pos >= 60u) v = B >> (pos - 60u);
+        else v = (A >> pos) | (B << (60u - pos));
+        return unit8<3>((uint32_t)v & 0xFFFFFFu, z, s);
     }
 }
 
@@ -243,7 +295,7 @@ constexpr int kPrefetch = 2;                          // k-tiles of codes in fli
 // one output tile; each keeps its partial sums in its own tensor memory, the
 // others write theirs into rank 0's (then idle) stage buffers through
 // distributed shared memory, and rank 0 adds them and stores Y.
-template <int NBITS, bool SMALL, int BN>
+template <int NBITS, bool SMALL, bool VEC, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ LinearParams prm) {
     constexpr uint32_t kBBytes = BN * kBK * 2;
@@ -331,37 +383,40 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
             mma_commit(done);
         }
     } else {
-        // ---- producers of W_hat
-        const int pw = warp - 2, j = lane & 7;
-        const int rbase = pw * 16 + (lane >> 3);            // tile row of unit i: rbase + 4i
-        ProducerRows pr;
-        producer_rows(prm, n0 + rbase, j, pr);
-        // a ring of kPrefetch k-tiles of codes in registers (indices fixed by unrolling)
-        KTileCodes<NBITS, SMALL> ring[kPrefetch];
+        // ---- producers of W_hat: quads of 4 units, a ring of kPrefetch k-tiles
+        // of codes in registers (indices fixed by unrolling)
+        const int pw = warp - 2, j4 = lane & 1;
+        const int r = pw * 16 + (lane >> 1);
+        const int64_t n = n0 + r;
+        const bool row_ok = n < prm.N;
+        const int64_t fbase = n * prm.K;
+        QuadCodes<NBITS> ring[kPrefetch];
 #pragma unroll
         for (int u = 0; u < kPrefetch - 1; ++u)
-            if (u < nkt) load_ktile<NBITS, SMALL>(prm, pr, j, kt0 + u, ring[u]);
+            if (u < nkt)
+                load_quad<NBITS, SMALL, VEC>(prm, fbase, row_ok,
+                                             (int64_t)(kt0 + u) * kBK + 32 * j4, ring[u]);
         for (int kb = 0; kb < nkt; kb += kPrefetch) {
 #pragma unroll
             for (int u = 0; u < kPrefetch; ++u) {
                 const int kt = kb + u;
                 if (kt < nkt) {
                     if (kt + kPrefetch - 1 < nkt)
-                        load_ktile<NBITS, SMALL>(prm, pr, j, kt0 + kt + kPrefetch - 1,
-                                                 ring[(u + kPrefetch - 1) % kPrefetch]);
+                        load_quad<NBITS, SMALL, VEC>(
+                            prm, fbase, row_ok,
+                            (int64_t)(kt0 + kt + kPrefetch - 1) * kBK + 32 * j4,
+                            ring[(u + kPrefetch - 1) % kPrefetch]);
                     const int s = kt % kStages;
                     const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
                     mbar_wait(empty(s), ph ^ 1u, abrt, prm.status, false);
-                    uint8_t* a = a_st + s * kABytes;
-                    const KTileCodes<NBITS, SMALL>& cur = ring[u];
+                    uint8_t* arow = a_st + s * kABytes + r * 128;
+                    const QuadCodes<NBITS>& cur = ring[u];
 #pragma unroll
-                    for (int i = 0; i < kUnitsPerThread; ++i) {
-                        const int r = rbase + 4 * i;
+                    for (int t = 0; t < 4; ++t) {
+                        const int j = 4 * j4 + t;
                         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                        if (cur.present & (1u << i))
-                            v = unit8_raw<NBITS>(cur.raw[i], __high2float(cur.sz[i]),
-                                                 __low2float(cur.sz[i]));
-                        *reinterpret_cast<uint4*>(a + r * 128 + ((j ^ (r & 7)) << 4)) = v;
+                        if (cur.present & (1u << t)) v = quad_unit<NBITS>(cur, t);
+                        *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = v;
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     mbar_arrive(full_a(s));
@@ -453,7 +508,7 @@ constexpr size_t linear_smem() {
     return 1024 + (size_t)kStages * (kABytes + BN * kBK * 2) + (3 * kStages + 1) * 8 + 16;
 }
 
-template <int NBITS, bool SMALL, int BN>
+template <int NBITS, bool SMALL, bool VEC, int BN>
 cudaError_t launch_bn(const LinearParams& prm, const void* X, cudaStream_t stream) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
@@ -466,7 +521,7 @@ cudaError_t launch_bn(const LinearParams& prm, const void* X, cudaStream_t strea
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    auto kern = linear_kernel<NBITS, SMALL, BN>;
+    auto kern = linear_kernel<NBITS, SMALL, VEC, BN>;
     constexpr size_t smem = linear_smem<BN>();
     // split-k partials of up to kMaxSplit - 1 ranks fit in rank 0's stage buffers
     static_assert(BN > 32 || (size_t)(kMaxSplit - 1) * BN * kBM * 4 <= (size_t)kStages * kABytes,
@@ -497,13 +552,22 @@ cudaError_t launch_bn(const LinearParams& prm, const void* X, cudaStream_t strea
     return cudaLaunchKernelEx(&cfg, kern, map, prm);
 }
 
-template <int NBITS, bool SMALL>
+template <int NBITS, bool SMALL, bool VEC>
 cudaError_t launch_nb(const LinearParams& prm, const void* X, cudaStream_t stream) {
-    if (prm.M <= 16) return launch_bn<NBITS, SMALL, 16>(prm, X, stream);
-    if (prm.M <= 32) return launch_bn<NBITS, SMALL, 32>(prm, X, stream);
-    if (prm.M <= 64) return launch_bn<NBITS, SMALL, 64>(prm, X, stream);
-    if (prm.M <= 128) return launch_bn<NBITS, SMALL, 128>(prm, X, stream);
-    return launch_bn<NBITS, SMALL, 256>(prm, X, stream);
+    if (prm.M <= 16) return launch_bn<NBITS, SMALL, VEC, 16>(prm, X, stream);
+    if (prm.M <= 32) return launch_bn<NBITS, SMALL, VEC, 32>(prm, X, stream);
+    if (prm.M <= 64) return launch_bn<NBITS, SMALL, VEC, 64>(prm, X, stream);
+    if (prm.M <= 128) return launch_bn<NBITS, SMALL, VEC, 128>(prm, X, stream);
+    return launch_bn<NBITS, SMALL, VEC, 256>(prm, X, stream);
+}
+
+// Quads of codes load as one vector when every row starts on a quad (K % 32)
+// and the packed buffer is 16-byte aligned.
+template <int NBITS>
+cudaError_t launch_vec(const LinearParams& prm, const void* X, cudaStream_t stream) {
+    const bool vec = prm.K % 32 == 0 && (reinterpret_cast<uintptr_t>(prm.packed) & 15u) == 0;
+    return vec ? launch_nb<NBITS, true, true>(prm, X, stream)
+               : launch_nb<NBITS, true, false>(prm, X, stream);
 }
 
 }  // namespace
@@ -511,12 +575,13 @@ cudaError_t launch_nb(const LinearParams& prm, const void* X, cudaStream_t strea
 cudaError_t launch_linear(const LinearParams& prm, const void* X, int nbits, cudaStream_t stream) {
     const bool small = prm.N * prm.K / 8 < ((int64_t)1 << 30);
     switch (nbits) {
-        case 1: return launch_nb<1, true>(prm, X, stream);
-        case 2: return launch_nb<2, true>(prm, X, stream);
-        case 4: return launch_nb<4, true>(prm, X, stream);
-        case 8: return launch_nb<8, true>(prm, X, stream);
+        case 1: return launch_vec<1>(prm, X, stream);
+        case 2: return launch_vec<2>(prm, X, stream);
+        case 4: return launch_vec<4>(prm, X, stream);
+        case 8: return launch_vec<8>(prm, X, stream);
         case 3:
-            return small ? launch_nb<3, true>(prm, X, stream) : launch_nb<3, false>(prm, X, stream);
+            return small ? launch_nb<3, true, false>(prm, X, stream)
+                         : launch_nb<3, false, false>(prm, X, stream);
         default: return cudaErrorInvalidValue;
     }
 }
