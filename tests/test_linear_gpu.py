@@ -56,7 +56,7 @@ def _check(Y_gpu, X, Wh, label):
 
 @pytest.mark.parametrize("nbits,group", [(4, 64), (3, 64), (2, 32), (4, 128), (2, 16), (3, 256),
                                          (8, 128), (1, 64)])
-@pytest.mark.parametrize("M", [1, 16, 100, 256])
+@pytest.mark.parametrize("M", [1, 2, 3, 16, 100, 256])
 def test_linear_formats_and_token_counts(hqq, nbits, group, M):
     rows, cols = 256, 1024
     W = synth.student_t_host((rows, cols), seed=50, stream=nbits * 100 + group).astype(np.float16)
@@ -67,7 +67,8 @@ def test_linear_formats_and_token_counts(hqq, nbits, group, M):
     _check(Y.cpu().numpy(), X, Wh, f"{nbits}b g{group} M={M}")
 
 
-@pytest.mark.parametrize("rows,cols,M", [(128, 64, 1), (300, 192, 17), (129, 320, 33),
+@pytest.mark.parametrize("rows,cols,M", [(128, 64, 1), (300, 192, 17), (129, 320, 33), (77, 48, 2),
+                                         (130, 8208, 1),
                                          (1000, 2048, 300), (64, 4096, 513), (384, 16, 7),
                                          (200, 8208, 65)])
 def test_linear_ragged_shapes(hqq, rows, cols, M):

@@ -310,8 +310,8 @@ extern "C" int hqq_linear(const void* X, int64_t M, const void* packed, const vo
     prm.N = rows;
     prm.K = cols;
     prm.log2_group = log2_of_group(group);
-    // up to 8 tokens: streaming kernel on the CUDA cores; more: tensor cores
-    const cudaError_t err = M <= 8
+    // one or two tokens: streaming kernel on the CUDA cores; more: tensor cores
+    const cudaError_t err = M <= kGemvMaxTokens
         ? launch_gemv(prm, X, nbits, static_cast<cudaStream_t>(stream))
         : launch_linear(prm, X, nbits, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;

@@ -58,6 +58,11 @@ struct Meta8 {
     int shift;
 };
 
+// Token counts up to which the linear layer runs on the CUDA cores (measured:
+// from 3 tokens on, the tensor-core kernel is faster on the 8192 x 8192 and
+// 28672 x 8192 shapes).
+constexpr int64_t kGemvMaxTokens = 2;
+
 // Weight-only linear layer Y = X W_hat^T on a quantized [N, K] matrix.
 struct LinearParams {
     const uint8_t* packed;

@@ -160,4 +160,115 @@ __device__ __forceinline__ uint32_t unit_bits(const uint8_t* __restrict__ packed
     }
 }
 
+// A quad: 4 consecutive units (32 codes) of one row, the work item of the
+// linear-layer kernels.  Its codes are one vector load (VEC, when rows start
+// on a quad: 4, 8, 16 or 32 bytes at 1, 2, 4 or 8 bits; four 32-bit words at
+// 3 bits) and its group data one (scale, zero) pair (two for groups of 16).
+template <int NBITS>
+struct QuadCodes {
+    static constexpr int NW = NBITS == 3 ? 4 : NBITS;     // 32-bit words of codes
+    uint32_t w[NW];
+    __half2 sz[2];                                     // (s, z) of units 0-1 and 2-3
+    uint32_t off;                                      // 3 bits: slot of code 0 in w[0]
+    uint32_t present;                                  // bit t: unit t inside the matrix
+};
+
+template <int NBITS, bool SMALL, bool VEC>
+__device__ __forceinline__ void load_quad(const LinearParams& p, int64_t fbase, bool row_ok,
+                                          int64_t kq, QuadCodes<NBITS>& c) {
+    // fbase: flat index of the row's first code; kq: k of the quad's first code
+    c.present = 0u;
+    c.off = 0u;
+#pragma unroll
+    for (int i = 0; i < QuadCodes<NBITS>::NW; ++i) c.w[i] = 0u;
+    c.sz[0] = c.sz[1] = __float2half2_rn(0.0f);
+    if (!row_ok || kq >= p.K) return;
+    const int64_t f = fbase + kq;
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+        if (kq + 8 * t < p.K) c.present |= 1u << t;
+    if constexpr (NBITS == 3) {
+        const int64_t u = f >> 3;
+        int64_t w0;
+        if (SMALL) {
+            const uint32_t u4 = 4u * (uint32_t)u;
+            w0 = __umulhi(u4, 0xCCCCCCCDu) >> 2;         // floor(f / 10)
+        } else {
+            w0 = (4 * u) / 5;
+        }
+        c.off = (uint32_t)(f - 10 * w0);
+        // slots off .. off + 8 * (present units) - 1 (< 40): only the words they
+        // touch are read, so a partial quad at the end stays inside the buffer
+        const uint32_t slots = c.off + 8u * (uint32_t)__popc(c.present);
+        const uint32_t* p32 = reinterpret_cast<const uint32_t*>(p.packed) + w0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (10u * i < slots) c.w[i] = __ldg(p32 + i);
+    } else if constexpr (VEC) {
+        const uint8_t* src = p.packed + (f >> 5) * (4 * NBITS);
+        if constexpr (NBITS == 8) {
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+            const uint4 b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+            c.w[0] = a.x; c.w[1] = a.y; c.w[2] = a.z; c.w[3] = a.w;
+            c.w[4] = b.x; c.w[5] = b.y; c.w[6] = b.z; c.w[7] = b.w;
+        } else if constexpr (NBITS == 4) {
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+            c.w[0] = a.x; c.w[1] = a.y; c.w[2] = a.z; c.w[3] = a.w;
+        } else if constexpr (NBITS == 2) {
+            const uint2 a = __ldg(reinterpret_cast<const uint2*>(src));
+            c.w[0] = a.x; c.w[1] = a.y;
+        } else {
+            c.w[0] = __ldg(reinterpret_cast<const uint32_t*>(src));
+        }
+    } else {                                           // unit by unit (any k alignment)
+        const int64_t u = f >> 3;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            if (!(c.present & (1u << t))) continue;
+            const UnitRaw r = unit_fetch<NBITS, SMALL>(p.packed, u + t);
+            if constexpr (NBITS == 8) {
+                c.w[2 * t] = r.w0;
+                c.w[2 * t + 1] = r.w1;
+            } else if constexpr (NBITS == 4) {
+                c.w[t] = r.w0;
+            } else if constexpr (NBITS == 2) {
+                c.w[t >> 1] |= r.w0 << (16 * (t & 1));
+            } else {
+                c.w[0] |= r.w0 << (8 * t);
+            }
+        }
+    }
+    const int64_t g = f >> p.log2_group;
+    c.sz[0] = __halves2half2(__ldg(p.scale + g), __ldg(p.zero + g));
+    c.sz[1] = c.sz[0];
+    if (p.log2_group == 4 && (c.present & 4u))
+        c.sz[1] = __halves2half2(__ldg(p.scale + g + 1), __ldg(p.zero + g + 1));
+}
+
+// Weights of unit t (0..3) of a loaded quad.
+template <int NBITS>
+__device__ __forceinline__ uint4 quad_unit(const QuadCodes<NBITS>& c, int t) {
+    const __half2 sz = c.sz[t >> 1];
+    const float s = __low2float(sz), z = __high2float(sz);
+    if constexpr (NBITS == 8) {
+        return unit8_bytes(c.w[2 * t], c.w[2 * t + 1], z, s);
+    } else if constexpr (NBITS == 4) {
+        return unit8<4>(c.w[t], z, s);
+    } else if constexpr (NBITS == 2) {
+        return unit8<2>((c.w[t >> 1] >> (16 * (t & 1))) & 0xFFFFu, z, s);
+    } else if constexpr (NBITS == 1) {
+        return unit8<1>((c.w[0] >> (8 * t)) & 0xFFu, z, s);
+    } else {
+        // the 30-bit fields of the four words as two 60-bit runs
+        const uint64_t A = (uint64_t)c.w[0] | ((uint64_t)c.w[1] << 30);
+        const uint64_t B = (uint64_t)c.w[2] | ((uint64_t)c.w[3] << 30);
+        const uint32_t pos = 3u * (c.off + 8u * (uint32_t)t);   // bit of code 8t
+        uint64_t v;
+        if (pos + 24u <= 60u) v = A >> pos;
+        else if (pos >= 60u) v = B >> (pos - 60u);
+        else v = (A >> pos) | (B << (60u - pos));
+        return unit8<3>((uint32_t)v & 0xFFFFFFu, z, s);
+    }
+}
+
 }  // namespace hqq
