@@ -68,7 +68,7 @@ def test_linear_formats_and_token_counts(hqq, nbits, group, M):
 
 
 @pytest.mark.parametrize("rows,cols,M", [(128, 64, 1), (300, 192, 17), (129, 320, 33), (77, 48, 2),
-                                         (130, 8208, 1),
+                                         (130, 8208, 1), (200, 512, 1030), (256, 1024, 2048),
                                          (1000, 2048, 300), (64, 4096, 513), (384, 16, 7),
                                          (200, 8208, 65)])
 def test_linear_ragged_shapes(hqq, rows, cols, M):
@@ -116,7 +116,7 @@ def test_linear_exact_on_integer_data(hqq):
     assert np.array_equal(Y.cpu().numpy(), ref["y"])
 
 
-@pytest.mark.parametrize("M", [1, 16, 256])
+@pytest.mark.parametrize("M", [1, 16, 256, 2048])
 def test_linear_full_size_70b_gate_sampled(hqq, M):
     """The 28672 x 8192 3-bit g64 gate matrix quantized on the GPU; sampled
     output features checked against the oracle's own quantization of those

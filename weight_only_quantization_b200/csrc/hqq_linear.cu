@@ -44,6 +44,9 @@ namespace {
 constexpr int kBM = 128;                 // features per CTA (MMA M)
 constexpr int kBK = 64;                  // k per stage: one 128-byte swizzle row
 constexpr int kStages = 4;
+
+// Stage count: 4, except 2 for 512-token tiles (80 KiB per stage).
+__host__ __device__ constexpr int stages_of(int bn) { return bn > 256 ? 2 : kStages; }
 constexpr int kThreads = 320;            // 10 warps
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s per wait
@@ -163,6 +166,9 @@ constexpr int kProducers = kProducerWarps * 32;
 constexpr int kUnitsPerThread = kBM * (kBK / 8) / kProducers;   // 4: one quad
 static_assert(kUnitsPerThread == 4, "one quad of units per producer thread and k-tile");
 constexpr int kMaxSplit = 4;                          // k-slices per cluster (decode shapes)
+// From this many tokens a CTA takes 512 (both 256-column halves of tensor
+// memory): each dequantized weight tile then serves twice the tokens.
+constexpr int64_t kLargeTileTokens = 1024;
 
 // The units one producer thread writes per k-tile: a quad of 4 consecutive
 // units (32 codes) of one row, units 4 (lane % 2) .. +3 of tile row
@@ -190,15 +196,18 @@ constexpr int kPrefetch = 2;                          // k-tiles of codes in fli
 template <int NBITS, bool SMALL, bool VEC, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ LinearParams prm) {
+    constexpr int S = stages_of(BN);
     constexpr uint32_t kBBytes = BN * kBK * 2;
     constexpr int kTmemCols = BN < 32 ? 32 : BN;
+    constexpr int kMmaN = BN > 256 ? 256 : BN;             // N of one MMA (and TMA box rows)
+    constexpr int kParts = BN / kMmaN;                     // accumulators side by side
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* a_st = smem;                                  // kStages x 16 KB
-    uint8_t* b_st = smem + kStages * kABytes;              // kStages x BN*128 B
-    uint64_t* bars = reinterpret_cast<uint64_t*>(b_st + kStages * kBBytes);
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
+    uint8_t* a_st = smem;                                  // S x 16 KB
+    uint8_t* b_st = smem + S * kABytes;              // S x BN*128 B
+    uint64_t* bars = reinterpret_cast<uint64_t*>(b_st + S * kBBytes);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * S + 1);
     float* red = reinterpret_cast<float*>(smem);           // split-k partials (rank 0)
     __shared__ int abort_flag;
 
@@ -212,13 +221,13 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
     const uint32_t bar0 = smem_u32(bars);
     // full_a[s] = bar0 + 8s, full_b[s] = bar0 + 8(S+s), empty[s] = bar0 + 8(2S+s), done
     auto full_a = [&](int s) { return bar0 + 8u * s; };
-    auto full_b = [&](int s) { return bar0 + 8u * (kStages + s); };
-    auto empty = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
-    const uint32_t done = bar0 + 8u * (3 * kStages);
+    auto full_b = [&](int s) { return bar0 + 8u * (S + s); };
+    auto empty = [&](int s) { return bar0 + 8u * (2 * S + s); };
+    const uint32_t done = bar0 + 8u * (3 * S);
 
     if (threadIdx.x == 0) {
         abort_flag = 0;
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(full_a(s), kProducers);
             mbar_init(full_b(s), 1);
             mbar_init(empty(s), 1);
@@ -244,32 +253,37 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
     if (warp == 0) {
         if (lane == 0) {                                    // X tiles by TMA
             for (int kt = 0; kt < nkt; ++kt) {
-                const int s = kt % kStages;
-                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                const int s = kt % S;
+                const uint32_t ph = (uint32_t)(kt / S) & 1u;
                 mbar_wait(empty(s), ph ^ 1u, abrt, prm.status, false);
                 mbar_expect_tx(full_b(s), kBBytes);
-                tma_load_2d(smem_u32(b_st + s * kBBytes), &xmap, full_b(s), (kt0 + kt) * kBK,
-                            (int)m0);
+#pragma unroll
+                for (int h = 0; h < kParts; ++h)
+                    tma_load_2d(smem_u32(b_st + s * kBBytes + h * kMmaN * kBK * 2), &xmap,
+                                full_b(s), (kt0 + kt) * kBK, (int)m0 + h * kMmaN);
             }
-            for (int kt = nkt > kStages ? nkt - kStages : 0; kt < nkt; ++kt)  // own loads landed
-                mbar_wait(full_b(kt % kStages), (uint32_t)(kt / kStages) & 1u, abrt, prm.status,
+            for (int kt = nkt > S ? nkt - S : 0; kt < nkt; ++kt)  // own loads landed
+                mbar_wait(full_b(kt % S), (uint32_t)(kt / S) & 1u, abrt, prm.status,
                           true);
         }
     } else if (warp == 1) {
         if (lane == 0) {                                    // MMA issue
-            const uint32_t idesc = f16_idesc<BN>();
+            const uint32_t idesc = f16_idesc<kMmaN>();
             for (int kt = 0; kt < nkt; ++kt) {
-                const int s = kt % kStages;
-                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                const int s = kt % S;
+                const uint32_t ph = (uint32_t)(kt / S) & 1u;
                 mbar_wait(full_b(s), ph, abrt, prm.status, false);
                 mbar_wait(full_a(s), ph, abrt, prm.status, false);
                 fence_after_sync();
                 const uint32_t a0 = smem_u32(a_st + s * kABytes);
                 const uint32_t b0 = smem_u32(b_st + s * kBBytes);
 #pragma unroll
-                for (int k4 = 0; k4 < kBK / 16; ++k4)
-                    mma_f16(tmem, sw128_desc(a0 + 32u * k4), sw128_desc(b0 + 32u * k4), idesc,
-                            (kt | k4) != 0 ? 1u : 0u);
+                for (int h = 0; h < kParts; ++h)            // columns [h kMmaN, (h+1) kMmaN)
+#pragma unroll
+                    for (int k4 = 0; k4 < kBK / 16; ++k4)
+                        mma_f16(tmem + (uint32_t)(h * kMmaN), sw128_desc(a0 + 32u * k4),
+                                sw128_desc(b0 + (uint32_t)(h * kMmaN * kBK * 2) + 32u * k4),
+                                idesc, (kt | k4) != 0 ? 1u : 0u);
                 mma_commit(empty(s));                       // stage free once these MMAs end
             }
             mma_commit(done);
@@ -298,8 +312,8 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
                             prm, fbase, row_ok,
                             (int64_t)(kt0 + kt + kPrefetch - 1) * kBK + 32 * j4,
                             ring[(u + kPrefetch - 1) % kPrefetch]);
-                    const int s = kt % kStages;
-                    const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                    const int s = kt % S;
+                    const uint32_t ph = (uint32_t)(kt / S) & 1u;
                     mbar_wait(empty(s), ph ^ 1u, abrt, prm.status, false);
                     uint8_t* arow = a_st + s * kABytes + r * 128;
                     const QuadCodes<NBITS>& cur = ring[u];
@@ -397,7 +411,8 @@ EncodeTiledFn encode_fn() {
 
 template <int BN>
 constexpr size_t linear_smem() {
-    return 1024 + (size_t)kStages * (kABytes + BN * kBK * 2) + (3 * kStages + 1) * 8 + 16;
+    return 1024 + (size_t)stages_of(BN) * (kABytes + BN * kBK * 2) + (3 * stages_of(BN) + 1) * 8 +
+           16;
 }
 
 template <int NBITS, bool SMALL, bool VEC, int BN>
@@ -407,7 +422,7 @@ cudaError_t launch_bn(const LinearParams& prm, const void* X, cudaStream_t strea
     CUtensorMap map;
     const cuuint64_t dims[2] = {(cuuint64_t)prm.K, (cuuint64_t)prm.M};
     const cuuint64_t strides[1] = {(cuuint64_t)prm.K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BN};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)(BN > 256 ? 256 : BN)};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(X), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -450,7 +465,8 @@ cudaError_t launch_nb(const LinearParams& prm, const void* X, cudaStream_t strea
     if (prm.M <= 32) return launch_bn<NBITS, SMALL, VEC, 32>(prm, X, stream);
     if (prm.M <= 64) return launch_bn<NBITS, SMALL, VEC, 64>(prm, X, stream);
     if (prm.M <= 128) return launch_bn<NBITS, SMALL, VEC, 128>(prm, X, stream);
-    return launch_bn<NBITS, SMALL, VEC, 256>(prm, X, stream);
+    if (prm.M < kLargeTileTokens) return launch_bn<NBITS, SMALL, VEC, 256>(prm, X, stream);
+    return launch_bn<NBITS, SMALL, VEC, 512>(prm, X, stream);
 }
 
 // Quads of codes load as one vector when every row starts on a quad (K % 32)
