@@ -5,7 +5,7 @@
 #include <cstring>
 
 #include "../../include/hqq.h"
-#include "hqq_common.cuh"
+#include "hqq_params.cuh"
 
 namespace hqq {
 cudaError_t launch_quantize(const QuantParams& prm, int nbits, int group, cudaStream_t stream);

@@ -1,4 +1,5 @@
-// hqq_common.cuh -- types and device helpers shared by libhqq's kernels.
+// hqq_common.cuh -- the quantize kernel's types and device helpers, and the
+// arithmetic contract every libhqq kernel follows.
 //
 // Arithmetic contract of the solver (binary32, round-to-nearest-even, every
 // rounding explicit): products and sums that the method writes separately are
@@ -47,41 +48,6 @@ struct QuantParams {
     PowTable tp;           // exponent p     (l_p error)
     PowTable tq;           // exponent p - 1 (generalised shrink)
     float shrink_thr[kMaxIters];  // |r| <= thr[t] guarantees W_e == 0 at step t
-};
-
-// 8-bit form of a meta tensor (zero points or scales): codes, the fp16 s and z
-// of each second-level group, and log2 of that group (62: one group).
-struct Meta8 {
-    const uint8_t* codes;
-    const __half* scale;
-    const __half* zero;
-    int shift;
-};
-
-// Token counts up to which the linear layer runs on the CUDA cores (measured:
-// from 3 tokens on, the tensor-core kernel is faster on the 8192 x 8192 and
-// 28672 x 8192 shapes).
-constexpr int64_t kGemvMaxTokens = 2;
-
-// Weight-only linear layer Y = X W_hat^T on a quantized [N, K] matrix.
-struct LinearParams {
-    const uint8_t* packed;
-    const __half* scale;
-    const __half* zero;
-    __half* Y;
-    int* status;             // optional: set to 1 if a wait inside a kernel ran out
-    int64_t M, N, K;         // tokens, output features, input features
-    int log2_group;
-};
-
-struct DequantParams {
-    const uint8_t* packed;
-    const __half* scale;   // fp16 scales, unless given in 8-bit form (sq)
-    const __half* zero;    // fp16 zero points, unless given in 8-bit form (zq)
-    __half* out;
-    int64_t n_units;       // n_elems / 8
-    int group;
-    Meta8 zq, sq;
 };
 
 // Shared-memory image of one PowTable (separate arrays, so that the two values

@@ -23,7 +23,7 @@
 //  - meta_dequant_kernel: 8 codes (one 8-byte load) -> one 16-byte store.
 #include <cooperative_groups.h>
 
-#include "hqq_common.cuh"
+#include "hqq_params.cuh"
 
 namespace hqq {
 

@@ -13,7 +13,7 @@
 // for fp16 z, so the only roundings are the product with s and the conversion
 // to fp16, as the definition requires.
 #pragma once
-#include "hqq_common.cuh"
+#include "hqq_params.cuh"
 
 namespace hqq {
 
