@@ -219,7 +219,8 @@ int hqq_dequantize_meta(const void* packed, const hqq_meta8* zero_q, const void*
  *
  *   X      [in]  fp16 [M, cols] row-major (tokens x input features),
  *                16-byte aligned.
- *   M      [in]  number of tokens, 0 <= M <= 65535*256 (M == 0: no-op).
+ *   M      [in]  number of tokens, 0 <= M <= 2^31 - 1024 (M == 0: no-op);
+ *                rows at most 65535*128.
  *   packed, scale, zero, rows, cols, nbits, group [in]  the quantized
  *                [rows, cols] matrix as hqq_quantize writes it (alignment as
  *                for hqq_dequantize).

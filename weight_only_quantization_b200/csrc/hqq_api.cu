@@ -292,8 +292,10 @@ extern "C" int hqq_linear(const void* X, int64_t M, const void* packed, const vo
                           void* Y, int* status, void* stream) {
     int st = validate_common(rows, cols, nbits, group);
     if (st != HQQ_OK) return st;
-    // one launch covers 65535 CTA rows of 256 tokens
-    if (M < 0 || M > (int64_t)65535 * 256) return HQQ_ERR_SHAPE;
+    // the grid holds 65535 feature tiles of 128; token coordinates of the
+    // 512-token tiles stay below 2^31
+    if (M < 0 || M > (((int64_t)1 << 31) - 1024)) return HQQ_ERR_SHAPE;
+    if (rows > (int64_t)65535 * 128) return HQQ_ERR_SHAPE;
     if (M == 0 || rows == 0 || cols == 0) return HQQ_OK;
     if (!X || !packed || !scale || !zero || !Y) return HQQ_ERR_NULL;
     if (!aligned(X, 16) || !aligned(packed, packed_align(nbits)) || !aligned(scale, 2) ||

@@ -212,8 +212,10 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n0 = (int64_t)blockIdx.x * kBM;
-    const int64_t m0 = (int64_t)blockIdx.y * BN;
+    // token tiles of one feature tile are adjacent in the grid (x), so a
+    // feature tile's codes come from HBM once and from L2 for the others
+    const int64_t n0 = (int64_t)blockIdx.y * kBM;
+    const int64_t m0 = (int64_t)blockIdx.x * BN;
     const int ks = (int)gridDim.z, rank = (int)blockIdx.z;
     const int KT = (int)((prm.K + kBK - 1) / kBK);
     const int kt0 = (int)((int64_t)KT * rank / ks);
@@ -450,7 +452,7 @@ cudaError_t launch_bn(const LinearParams& prm, const void* X, cudaStream_t strea
     attr.val.clusterDim.x = 1;
     attr.val.clusterDim.y = 1;
     attr.val.clusterDim.z = (unsigned)ks;
-    cfg.gridDim = dim3((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)ks);
+    cfg.gridDim = dim3((unsigned)tiles_m, (unsigned)tiles_n, (unsigned)ks);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
