@@ -118,8 +118,104 @@ gemv_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams p
     }
 }
 
+// Persistent form: X staged once per CTA in shared memory (fp16), each warp
+// owns whole output features (rows), its lanes take quads l, l+32, ... of the
+// row with kPvUnroll quads' loads issued before any use, and a warp shuffle
+// sums the row.  No cross-warp reduction, no token reloads per row.
+constexpr int kPvUnroll = 4;
+
+template <int NBITS, bool SMALL, bool VEC, int MT>
+__global__ void __launch_bounds__(kGvThreads)
+gemv_rows_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams p) {
+    extern __shared__ __align__(16) uint8_t gv_smem[];
+    __half* xs = reinterpret_cast<__half*>(gv_smem);            // [MT][K], rows past M zero
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    {
+        const int64_t nv = (int64_t)MT * p.K / 8;                  // 16-byte vectors
+        for (int64_t v = threadIdx.x; v < nv; v += kGvThreads) {
+            const int64_t m = v * 8 / p.K;
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (m < p.M) val = __ldg(reinterpret_cast<const uint4*>(X) + v);
+            reinterpret_cast<uint4*>(xs)[v] = val;
+        }
+    }
+    __syncthreads();
+    const int64_t nq = (p.K + 31) >> 5;
+    for (int64_t n = (int64_t)blockIdx.x * kGvWarps + warp; n < p.N;
+         n += (int64_t)gridDim.x * kGvWarps) {
+        float2 acc[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[m] = make_float2(0.0f, 0.0f);
+        for (int64_t qb = 0; qb < nq; qb += 32 * kPvUnroll) {
+            QuadCodes<NBITS> qc[kPvUnroll];
+#pragma unroll
+            for (int i = 0; i < kPvUnroll; ++i) {
+                const int64_t q = qb + 32 * i + lane;
+                load_quad<NBITS, SMALL, VEC>(p, n * p.K, q < nq, q * 32, qc[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < kPvUnroll; ++i) {
+                const int64_t q = qb + 32 * i + lane;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    if (!(qc[i].present & (1u << t))) continue;
+                    const uint4 wv = quad_unit<NBITS>(qc[i], t);
+                    const float2 w0 = __half22float2(*reinterpret_cast<const __half2*>(&wv.x));
+                    const float2 w1 = __half22float2(*reinterpret_cast<const __half2*>(&wv.y));
+                    const float2 w2 = __half22float2(*reinterpret_cast<const __half2*>(&wv.z));
+                    const float2 w3 = __half22float2(*reinterpret_cast<const __half2*>(&wv.w));
+                    const int64_t k = q * 32 + 8 * t;
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        const uint4 xv = *reinterpret_cast<const uint4*>(xs + m * p.K + k);
+                        float2 a = acc[m];
+                        a = __ffma2_rn(w0, __half22float2(*reinterpret_cast<const __half2*>(&xv.x)), a);
+                        a = __ffma2_rn(w1, __half22float2(*reinterpret_cast<const __half2*>(&xv.y)), a);
+                        a = __ffma2_rn(w2, __half22float2(*reinterpret_cast<const __half2*>(&xv.z)), a);
+                        a = __ffma2_rn(w3, __half22float2(*reinterpret_cast<const __half2*>(&xv.w)), a);
+                        acc[m] = a;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            float v = __fadd_rn(acc[m].x, acc[m].y);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == 0 && m < p.M) p.Y[(int64_t)m * p.N + n] = __float2half_rn(v);
+        }
+    }
+}
+
+// Shared memory of the persistent form: the token rows in fp16.
+constexpr int64_t kPvMaxSmem = 160 * 1024;
+
+template <int NBITS, bool SMALL, bool VEC, int MT>
+cudaError_t launch_rows(const LinearParams& p, const void* X, cudaStream_t stream) {
+    auto kern = gemv_rows_kernel<NBITS, SMALL, VEC, MT>;
+    const size_t smem = (size_t)MT * p.K * 2;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGvThreads, smem);
+    if (per_sm < 1) per_sm = 1;
+    int64_t blocks = (int64_t)sms * per_sm;
+    const int64_t need = (p.N + kGvWarps - 1) / kGvWarps;
+    if (blocks > need) blocks = need;
+    kern<<<(unsigned)blocks, kGvThreads, smem, stream>>>(static_cast<const __half*>(X), p);
+    return cudaGetLastError();
+}
+
 template <int NBITS, bool SMALL, bool VEC, int MT>
 cudaError_t launch_m(const LinearParams& p, const void* X, cudaStream_t stream) {
+    // measured: the persistent form is faster at 3 bits (gate 28672x8192: 0.129
+    // vs 0.141 ms for one token), slower at 4 bits (8192^2: 0.053 vs 0.041 ms)
+    if (NBITS == 3 && (int64_t)MT * p.K * 2 <= kPvMaxSmem)
+        return launch_rows<NBITS, SMALL, VEC, MT>(p, X, stream);
     constexpr int R = MT <= 2 ? 2 : 1;
     const int64_t blocks = (p.N + R - 1) / R;
     gemv_kernel<NBITS, SMALL, VEC, MT, R><<<(unsigned)blocks, kGvThreads, 0, stream>>>(
