@@ -164,6 +164,17 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+def tensor_peak():
+    """Dense fp16/bf16 tensor-core peak in TFLOP/s: the measured cuBLAS bf16 burst
+    figure (fp16 runs at the same rate), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        return 1590.0
+
+
 def profiled_traffic(kernel: str, fmt: str):
     """DRAM bytes per weight of `kernel` from the committed ncu summary, or None
     when the kernel's sources changed since the counters were taken."""
@@ -186,6 +197,17 @@ def profiled_traffic(kernel: str, fmt: str):
         if kv.get("source_sha256_16") == cur and "traffic_bytes_per_param" in kv:
             return float(kv["traffic_bytes_per_param"]), os.path.relpath(path, ROOT)
     return None, None
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def cpu_cores():
@@ -283,7 +305,8 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_dict(args.workload, mats, args.gpus),
             "cpu_baseline": {"value": value, "unit": "Gparam/s", "cores": cores,
-                             "kind": "oracle", "sample": desc + f"; {n} params per step"},
+                             "kind": "oracle", "cpu_model": cpu_model(),
+                             "sample": desc + f"; {n} params per step"},
             "e2e": {"value": value, "unit": "Gparam/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -477,9 +500,17 @@ def run_gpu(args):
             "gpu_launches": 2 * len(views) * args.steps,
             "clocks": clk}
 
+    # ---- weight-only linear layer on the quantized matrices
+    if not args.no_linear:
+        line["linear"] = run_linear(args, views, hqq, dev, hbm_peak, tensor_peak(), pg)
+
     # ---- 8-bit meta data (zero points: one group; scales: groups of 128)
     if not args.no_meta:
         line["meta8"] = run_meta8(args, views, hqq, dev, hbm_peak, pg)
+
+    # ---- memory-side calibration: round-to-nearest quantize pass (HBM-bound;
+    # runs after the sections above, which use the HQQ codes)
+    line["rtn"] = run_rtn(views, hqq, dev, hbm_peak, qbytes, pg)
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     if ws == 1 and not args.no_cpu_baseline:
@@ -494,7 +525,8 @@ def run_gpu(args):
             n, dt, reps = n + n1, dt + dt1, reps + 1
         desc += f"; repeated {reps}x"
         line["cpu_baseline"] = {"value": n / dt / 1e9, "unit": "Gparam/s", "cores": cores,
-                                "kind": "oracle", "sample": desc + f"; {n} params, {dt:.1f} s"}
+                                "kind": "oracle", "cpu_model": cpu_model(),
+                                "sample": desc + f"; {n} params, {dt:.1f} s"}
 
     # ---- model-shaped sets: one streamed pass, each layer's weights generated
     # on the device into one reused buffer and then quantized (wall time)
@@ -593,6 +625,128 @@ def run_meta8(args, views, hqq, dev, hbm_peak, pg):
                                 "hbm_frac": dq_gbs / hbm_peak,
                                 "gparam_s": params / (dq_ms / 1e3) / 1e9,
                                 "bytes_per_param": dq_bytes / params}}
+
+
+def run_rtn(views, hqq, dev, hbm_peak, qbytes, pg):
+    """The memory-side calibration point: the same quantize pass with zero
+    solver iterations (min-max round-to-nearest + packing), HBM-bound."""
+    import torch
+    stream = torch.cuda.current_stream()
+
+    def rtn_all():
+        for W, q, _ in views:
+            hqq.hqq_quantize(W, q.nbits, q.group, iters=0, packed=q.packed, scale=q.scale,
+                             zero=q.zero)
+
+    rtn_all()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        rtn_all()
+    for _ in range(3):
+        g.replay()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    reps = 3
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(reps):
+        g.replay()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps], pg, dev)[0]
+    del g
+    gbs = qbytes / (ms / 1e3) / 1e9
+    return {"what": "quantize pass with iters = 0 (min-max round-to-nearest + packing)",
+            "ms_per_pass": ms, "gbs": gbs, "hbm_frac": gbs / hbm_peak}
+
+
+def run_linear(args, views, hqq, dev, hbm_peak, tensor_peak, pg):
+    """Times the weight-only linear layer Y = X W_hat^T (dequantization fused
+    into the tensor-core product) on the workload's quantized matrices:
+    decode steps (M = 1 and 16 tokens through every matrix, as CUDA graphs) and
+    a prefill of M = 2048 tokens through the first seven matrices (one layer of
+    the model-shaped sets).  Beside it, torch's fp16 matmul on the dequantized
+    weights of those seven matrices, for context."""
+    import torch
+    stream = torch.cuda.current_stream()
+    maxk = max(q.cols for _, q, _ in views)
+    maxn = max(q.rows for _, q, _ in views)
+
+    def timed(fn, reps=3):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(2):
+            g.replay()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for _ in range(reps):
+            g.replay()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / reps
+        del g
+        return ms
+
+    out = {"what": "Y = X W_hat^T, W_hat dequantized inside the tensor-core kernel (fp16 X and Y, "
+                   "fp32 accumulation)"}
+    for M in (1, 16):
+        X = torch.randn(M * maxk, device=dev).half()
+        Y = torch.empty(M * maxn, dtype=torch.float16, device=dev)
+
+        def dec():
+            for _, q, _ in views:
+                hqq.hqq_linear(X[:M * q.cols].view(M, q.cols), q,
+                               out=Y[:M * q.rows].view(M, q.rows))
+        ms = max_over_ranks([timed(dec)], pg, dev)[0]
+        wbytes = sum(q.packed.numel() + 4 * q.scale.numel() for _, q, _ in views)
+        iobytes = sum(2 * M * (q.cols + q.rows) for _, q, _ in views)
+        gbs = (wbytes + iobytes) / (ms / 1e3) / 1e9
+        flops = sum(2.0 * M * q.rows * q.cols for _, q, _ in views)
+        out[f"decode_m{M}"] = {"matrices": len(views), "ms_per_pass": ms,
+                               "tokens_per_s": M / (ms / 1e3),
+                               "gbs": gbs, "hbm_frac": gbs / hbm_peak,
+                               "tflops": flops / (ms / 1e3) / 1e12,
+                               "bytes_per_pass": wbytes + iobytes}
+        del X, Y
+    sub = views[:7]
+    M = 2048
+    X = torch.randn(M * maxk, device=dev).half()
+    Y = torch.empty(M * maxn, dtype=torch.float16, device=dev)
+
+    def pre():
+        for _, q, _ in sub:
+            hqq.hqq_linear(X[:M * q.cols].view(M, q.cols), q, out=Y[:M * q.rows].view(M, q.rows))
+    ms = max_over_ranks([timed(pre)], pg, dev)[0]
+    flops = sum(2.0 * M * q.rows * q.cols for _, q, _ in sub)
+    tf = flops / (ms / 1e3) / 1e12
+    Wd = [hqq.hqq_dequantize(q) for _, q, _ in sub]
+
+    def ref():
+        for (_, q, _), w in zip(sub, Wd):
+            torch.matmul(X[:M * q.cols].view(M, q.cols), w.t(),
+                         out=Y[:M * q.rows].view(M, q.rows))
+    ms_t = max_over_ranks([timed(ref)], pg, dev)[0]
+
+    def ref1():
+        for (_, q, _), w in zip(sub, Wd):
+            torch.matmul(X[:q.cols].view(1, q.cols), w.t(), out=Y[:q.rows].view(1, q.rows))
+    ms_t1 = max_over_ranks([timed(ref1)], pg, dev)[0]
+
+    def dec1():
+        for _, q, _ in sub:
+            hqq.hqq_linear(X[:q.cols].view(1, q.cols), q, out=Y[:q.rows].view(1, q.rows))
+    ms_1 = max_over_ranks([timed(dec1)], pg, dev)[0]
+    out["prefill_m2048"] = {"matrices": len(sub), "ms_per_pass": ms, "tflops": tf,
+                            "tensor_frac": tf / tensor_peak,
+                            "torch_fp16_dequantized_ms": ms_t,
+                            "torch_fp16_tflops": flops / (ms_t / 1e3) / 1e12}
+    out["decode_m1_first7"] = {"ms_per_pass": ms_1, "torch_fp16_dequantized_ms": ms_t1}
+    del X, Y, Wd
+    return out
 
 
 def run_stream_pass(mats, hqq, dev, views):
@@ -708,6 +862,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
     ap.add_argument("--no-stream", action="store_true", help="skip the streamed generate+quantize pass")
     ap.add_argument("--no-meta", action="store_true", help="skip the 8-bit meta-data timing")
+    ap.add_argument("--no-linear", action="store_true", help="skip the linear-layer timing")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every library call from Python each pass instead of replaying "
                          "CUDA graphs of the passes")
