@@ -259,3 +259,33 @@ def test_multi_chunk_per_warp(hqq, nbits, group):
 def test_multi_chunk_shrink_active(hqq, group):
     W, Wn = _dev_weights((2048, 8192), seed=31, stream=group, std=1.0)
     _check(hqq, W, Wn, 4, group, f"multi-chunk std 1 4b g{group}")
+
+
+# --------------------------------------- iters = 0: the round-to-nearest kernel
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("group", [16, 32, 64, 128, 256])
+def test_rtn_all_formats_ragged(hqq, nbits, group):
+    # 41 rows x 17 groups: several 2560-weight tiles and a ragged last one
+    W, Wn = _dev_weights((41, 17 * group), seed=40, stream=nbits * 1000 + group)
+    _, _, st = _check(hqq, W, Wn, nbits, group, f"rtn {nbits}b g{group}", iters=0)
+    assert st["code_match"] == 1.0
+
+
+@pytest.mark.parametrize("nbits,group", [(3, 64), (4, 64), (2, 32)])
+def test_rtn_full_size_sampled_rows(hqq, nbits, group):
+    rows, cols = 28672, 8192
+    W = synth.student_t_device((rows, cols), seed=5, stream=4)
+    q = gpu_quantize(W, nbits, group, iters=0)
+    rng = np.random.default_rng(41)
+    sample = np.sort(rng.choice(rows, 48, replace=False))
+    Wn = W[torch.from_numpy(sample).cuda()].cpu().numpy()
+    ref = oracle.quantize(Wn, nbits, group, iters=0)
+    gs = cols // group
+    sc = q.scale.view(-1).cpu().numpy().reshape(rows, gs)[sample].reshape(-1)
+    zf = q.zero_f32.view(-1).cpu().numpy().reshape(rows, gs)[sample].reshape(-1)
+    assert np.array_equal(sc.view(np.uint16), ref["scale"].view(np.uint16))
+    assert np.max(np.abs(zf - ref["zero_f32"])) <= ZERO_TOL
+    g_idx = (sample[:, None] * gs + np.arange(gs)[None, :]).reshape(-1)
+    codes = group_codes(q.packed.cpu().numpy(), nbits, group, g_idx).reshape(-1)
+    assert np.array_equal(codes, ref["codes"])
+    assert np.all(q.iters.view(-1).cpu().numpy() == 0)

@@ -9,6 +9,17 @@
 
 namespace hqq {
 cudaError_t launch_quantize(const QuantParams& prm, int nbits, int group, cudaStream_t stream);
+struct RtnParams {
+    const __half* W;
+    uint8_t* packed;
+    __half* scale;
+    __half* zero;
+    float* zero_f32;
+    float* err_out;
+    uint8_t* iters_out;
+    int64_t n_elems;
+};
+cudaError_t launch_rtn(const RtnParams& p, int nbits, int group, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_group,
                               cudaStream_t stream);
 cudaError_t launch_linear(const LinearParams& prm, const void* X, int nbits, cudaStream_t stream);
@@ -136,6 +147,20 @@ extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nb
         !aligned(zero, 2) || (zero_f32 && !aligned(zero_f32, 4)) ||
         (err_out && !aligned(err_out, 4)))
         return HQQ_ERR_ALIGN;
+
+    if (iters == 0) {                  // min-max round-to-nearest: the streaming kernel
+        RtnParams rp;
+        rp.W = static_cast<const __half*>(W);
+        rp.packed = static_cast<uint8_t*>(packed);
+        rp.scale = static_cast<__half*>(scale);
+        rp.zero = static_cast<__half*>(zero);
+        rp.zero_f32 = zero_f32;
+        rp.err_out = err_out;
+        rp.iters_out = iters_out;
+        rp.n_elems = n;
+        const cudaError_t err = launch_rtn(rp, nbits, group, static_cast<cudaStream_t>(stream));
+        return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+    }
 
     QuantParams prm;
     std::memset(&prm, 0, sizeof prm);
