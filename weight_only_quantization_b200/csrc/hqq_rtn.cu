@@ -8,9 +8,12 @@
 // and group data.  Each warp takes tiles of 2560 weights (a multiple of every
 // group size and of the ten codes of a 3-bit word): all ten 16-byte loads of a
 // lane are issued first (unit l + 32 r of the tile in round r), a group's
-// min/max meets over its segment of G/8 lanes, and each lane writes its unit's
-// packed codes (3-bit codes go through shared memory and leave as whole
-// words).  The arithmetic is the solver kernel's, op for op: s = (max-min)/L
+// min/max meets over its segment of G/8 lanes, the group constants s, 1/s, z
+// are formed with one group per lane (gathered by shuffles, so the correctly
+// rounded division and reciprocal run ceil(2560/G/32) times per lane and tile,
+// not 10) and fetched back per round, and each lane writes its unit's packed
+// codes (3-bit units go through shared memory as 24-bit values and leave as
+// whole words, each a funnel shift of two units).  The arithmetic is the solver kernel's, op for op: s = (max-min)/L
 // and 1/s correctly rounded (s = 1/s = 1 for a constant group),
 // z = -(min * 1/s), code = round(clamp(fma(w, 1/s, z), 0, L)) by the 1.5*2^23
 // shift; the solver's error output is +inf and its iteration count 0.
@@ -41,12 +44,16 @@ template <int NBITS, int G>
 __global__ void __launch_bounds__(kRtWarps * 32)
 rtn_kernel(const __grid_constant__ RtnParams p) {
     constexpr int SEG = G / 8;                // lanes of one group in a round
+    constexpr int GPR = 32 / SEG;             // groups per round
+    constexpr int GT = kRtTile / G;           // groups per tile (10 GPR)
+    constexpr int kRtJ = (GT + 31) / 32;      // group constants per lane
     constexpr float L = (float)((1 << NBITS) - 1);
-    __shared__ __align__(16) uint8_t codes_s[NBITS == 3 ? kRtWarps * kRtTile : 16];
+    // 3 bits: one 32-bit slot (24 code bits) per unit of each warp's tile
+    __shared__ __align__(16) uint8_t codes_s[NBITS == 3 ? kRtWarps * kRtUnits * 4 : 16];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nunits = p.n_elems >> 3;
     const int64_t ntiles = (p.n_elems + kRtTile - 1) / kRtTile;
-    uint8_t* my_codes = codes_s + (NBITS == 3 ? warp * kRtTile : 0);
+    uint8_t* my_codes = codes_s + (NBITS == 3 ? warp * kRtUnits * 4 : 0);
 
     for (int64_t tile = (int64_t)blockIdx.x * kRtWarps + warp; tile < ntiles;
          tile += (int64_t)gridDim.x * kRtWarps) {
@@ -58,10 +65,10 @@ rtn_kernel(const __grid_constant__ RtnParams p) {
             raw[r] = u < nunits ? __ldg(reinterpret_cast<const uint4*>(p.W) + u)
                                 : make_uint4(0u, 0u, 0u, 0u);
         }
+        // 1. exact min/max of every group (all lanes of a segment hold them)
+        float mnr[kRtRounds], mxr[kRtRounds];
 #pragma unroll
         for (int r = 0; r < kRtRounds; ++r) {
-            const int64_t u = u0 + 32 * r + lane;
-            const bool valid = u < nunits;            // whole groups: n_elems % G == 0
             const uint32_t wv[4] = {raw[r].x, raw[r].y, raw[r].z, raw[r].w};
             __half2 hmn = *reinterpret_cast<const __half2*>(&wv[0]), hmx = hmn;
 #pragma unroll
@@ -77,20 +84,60 @@ rtn_kernel(const __grid_constant__ RtnParams p) {
                 mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             }
-            const float rng = __fsub_rn(mx, mn);
-            float s = 1.0f, inv = 1.0f;
-            if (rng != 0.0f) {
-                s = __fdiv_rn(rng, L);
-                inv = __frcp_rn(s);
+            mnr[r] = mn;
+            mxr[r] = mx;
+        }
+        // 2. one lane per group (group 32 j + lane of the tile): gather its
+        // min/max from the round and segment that hold it, then s, 1/s and z
+        // (the correctly rounded division and reciprocal once per group)
+        float sj[kRtJ], invj[kRtJ], zj[kRtJ];
+#pragma unroll
+        for (int j = 0; j < kRtJ; ++j) {
+            const int gl = 32 * j + lane;
+            const int r_mine = gl / GPR;                  // round holding the group
+            const int src = (gl % GPR) * SEG;             // its segment's first lane
+            float mn = 0.0f, mx = 0.0f;
+#pragma unroll
+            for (int rr = 0; rr < kRtRounds; ++rr) {
+                if (rr < (32 * j) / GPR || rr > (32 * j + 31) / GPR) continue;   // compile-time
+                const float a = __shfl_sync(0xffffffffu, mnr[rr], src);
+                const float bmx = __shfl_sync(0xffffffffu, mxr[rr], src);
+                if (rr == r_mine) {
+                    mn = a;
+                    mx = bmx;
+                }
             }
-            const float z = -__fmul_rn(mn, inv);
+            const float rng = __fsub_rn(mx, mn);
+            float sv = 1.0f, inv = 1.0f;
+            if (rng != 0.0f) {
+                sv = __fdiv_rn(rng, L);
+                inv = __frcp_rn(sv);
+            }
+            sj[j] = sv;
+            invj[j] = inv;
+            zj[j] = -__fmul_rn(mn, inv);
+        }
+        // 3. codes and outputs (each lane's group constants fetched back)
+#pragma unroll
+        for (int r = 0; r < kRtRounds; ++r) {
+            const int64_t u = u0 + 32 * r + lane;
+            const bool valid = u < nunits;            // whole groups: n_elems % G == 0
+            const int src = ((32 * r + lane) / SEG) % 32; // lane holding this unit's group
+            const float s = __shfl_sync(0xffffffffu, sj[r / SEG], src);
+            const float inv = __shfl_sync(0xffffffffu, invj[r / SEG], src);
+            const float z = __shfl_sync(0xffffffffu, zj[r / SEG], src);
+            const uint32_t wv[4] = {raw[r].x, raw[r].y, raw[r].z, raw[r].w};
+            // No clamp is needed: with z = -fl(min (1/s)), fma(w, 1/s, z) lies
+            // within [-2^-5, L + 2^-5] for every w of the group (a finite fp16
+            // group has max - min >= 2^-11 |min|, so |min (1/s)| <= L 2^11 <=
+            // 2^19 and z is off by at most 2^-5; fma is monotone in w), so
+            // round-to-nearest already gives 0..L and the clamp of the
+            // definition is the identity here.
             uint32_t c[8];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[j]));
-                float2 v = __ffma2_rn(f, make_float2(inv, inv), make_float2(z, z));
-                v.x = fminf(fmaxf(v.x, 0.0f), L);
-                v.y = fminf(fmaxf(v.y, 0.0f), L);
+                const float2 v = __ffma2_rn(f, make_float2(inv, inv), make_float2(z, z));
                 const float2 t = __fadd2_rn(v, make_float2(kRoundShift, kRoundShift));
                 c[2 * j] = __float_as_uint(t.x) & 0xFFu;
                 c[2 * j + 1] = __float_as_uint(t.y) & 0xFFu;
@@ -101,11 +148,11 @@ rtn_kernel(const __grid_constant__ RtnParams p) {
                     b.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
                     b.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
                     reinterpret_cast<uint2*>(p.packed)[u] = b;
-                } else if constexpr (NBITS == 3) {
-                    uint2 b;
-                    b.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-                    b.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-                    *reinterpret_cast<uint2*>(my_codes + (32 * r + lane) * 8) = b;
+                } else if constexpr (NBITS == 3) {            // the unit's 24 code bits
+                    uint32_t b = 0u;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) b |= c[i] << (3 * i);
+                    reinterpret_cast<uint32_t*>(my_codes)[32 * r + lane] = b;
                 } else {
                     uint32_t word = 0u;
 #pragma unroll
@@ -129,11 +176,16 @@ rtn_kernel(const __grid_constant__ RtnParams p) {
             const int64_t e0 = tile * kRtTile;        // first weight of the tile
             const int64_t left = p.n_elems - e0;
             const int nw = (int)((left < kRtTile ? left : kRtTile) + 9) / 10;
+            // word w = code bits [30 w, 30 w + 30) of the tile: a funnel shift
+            // of the two units (24 bits each) that hold them; codes past the
+            // end of the matrix are zero
+            const uint32_t* ub = reinterpret_cast<const uint32_t*>(my_codes);
+            const int nu = (int)((left < kRtTile ? left : kRtTile) >> 3);   // units in the tile
             for (int w = lane; w < nw; w += 32) {
-                uint32_t word = 0u;
-#pragma unroll
-                for (int i = 0; i < 10; ++i)
-                    if (10 * w + i < left) word |= (uint32_t)my_codes[10 * w + i] << (3 * i);
+                const int a = (30 * w) / 24, sh = (30 * w) % 24;
+                const uint64_t lo = ub[a];
+                const uint64_t hi = a + 1 < nu ? ub[a + 1] : 0u;
+                const uint32_t word = (uint32_t)(((lo | (hi << 24)) >> sh) & 0x3FFFFFFFu);
                 reinterpret_cast<uint32_t*>(p.packed)[tile * kRtWords + w] = word;
             }
             __syncwarp();
