@@ -6,7 +6,8 @@
 // one 16-byte output, always inside one group (8 divides every group size).
 // Lane l of a block takes units base + r*256 + l, so every warp load is a
 // contiguous run of packed codes and every warp store writes 512 contiguous
-// bytes; all loads of a thread's units are issued before any store.  No shared
+// bytes (streaming stores: the output is written once and not re-read by this
+// kernel); all loads of a thread's units are issued before any store.  No shared
 // memory, so occupancy is limited only by registers (staging the output tile
 // in shared memory for TMA bulk stores measured slower: it cost occupancy).
 // The code-to-weight arithmetic is in hqq_unpack.cuh.
@@ -58,7 +59,7 @@ dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
                 o = unit8_raw<8>(x8[r], zf[r], sf[r]);
             else
                 o = unit8<NBITS>(x[r], zf[r], sf[r]);
-            if (u < prm.n_units) reinterpret_cast<uint4*>(prm.out)[u] = o;
+            if (u < prm.n_units) __stcs(reinterpret_cast<uint4*>(prm.out) + u, o);   // written once: evict first
         }
     }
 }
