@@ -227,6 +227,7 @@ extern "C" int hqq_dequantize(const void* packed, const void* scale, const void*
     prm.zero = static_cast<const __half*>(zero);
     prm.out = static_cast<__half*>(W_out);
     prm.n_units = n / 8;
+    prm.n_words = (uint32_t)((n + 9) / 10 < ((int64_t)1 << 32) ? (n + 9) / 10 : 0);
     prm.group = group;
     const cudaError_t err = launch_dequantize(prm, nbits, log2_of_group(group),
                                               static_cast<cudaStream_t>(stream));
@@ -306,6 +307,7 @@ extern "C" int hqq_dequantize_meta(const void* packed, const hqq_meta8* zero_q, 
     prm.scale = static_cast<const __half*>(scale);
     prm.out = static_cast<__half*>(W_out);
     prm.n_units = n / 8;
+    prm.n_words = (uint32_t)((n + 9) / 10 < ((int64_t)1 << 32) ? (n + 9) / 10 : 0);
     prm.group = group;
     const cudaError_t err = launch_dequantize(prm, nbits, log2_of_group(group),
                                               static_cast<cudaStream_t>(stream));

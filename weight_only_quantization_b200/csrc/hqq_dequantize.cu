@@ -35,7 +35,11 @@ __global__ void __launch_bounds__(kDqThreads)
 dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
     for (int64_t base = (int64_t)blockIdx.x * kDqTile; base < prm.n_units;
          base += (int64_t)gridDim.x * kDqTile) {
-        // 8-bit units are 64 bits (fetched raw); narrower ones one word
+        // 8-bit units are 64 bits (fetched raw); narrower ones one word; 3 bits
+        // (word indices < 2^32): the warp's 32 consecutive units span at most
+        // 27 words, so lane l loads word l of the span and each unit takes its
+        // two words from their lanes by shuffle
+        constexpr bool kWarp3 = NBITS == 3 && SMALL;
         uint32_t x[kDqUnits];
         UnitRaw x8[NBITS == 8 ? kDqUnits : 1];
         float sf[kDqUnits], zf[kDqUnits];
@@ -46,19 +50,37 @@ dequantize_kernel(const __grid_constant__ DequantParams prm, int log2_group) {
             const int64_t g = (u * 8) >> log2_group;
             sf[r] = (META & 2) ? restore_meta(prm.sq, g) : __half2float(__ldg(prm.scale + g));
             zf[r] = (META & 1) ? restore_meta(prm.zq, g) : __half2float(__ldg(prm.zero + g));
-            if constexpr (NBITS == 8)
+            if constexpr (NBITS == 8) {
                 x8[r] = unit_fetch<8, SMALL>(prm.packed, u);
-            else
+            } else if constexpr (kWarp3) {
+                const uint32_t u0 = (uint32_t)(base + r * kDqThreads + (threadIdx.x & ~31u));
+                const uint32_t wfirst = __umulhi(4u * u0, 0xCCCCCCCDu) >> 2;   // floor(8 u0 / 10)
+                const uint32_t wi = wfirst + (threadIdx.x & 31u);
+                x[r] = wi < prm.n_words ? __ldg(reinterpret_cast<const uint32_t*>(prm.packed) + wi)
+                                        : 0u;
+            } else {
                 x[r] = unit_bits<NBITS, SMALL>(prm.packed, u);
+            }
         }
 #pragma unroll
         for (int r = 0; r < kDqUnits; ++r) {
             const int64_t u = base + r * kDqThreads + threadIdx.x;
             uint4 o;
-            if constexpr (NBITS == 8)
+            if constexpr (NBITS == 8) {
                 o = unit8_raw<8>(x8[r], zf[r], sf[r]);
-            else
+            } else if constexpr (kWarp3) {
+                const uint32_t u0 = (uint32_t)(base + r * kDqThreads + (threadIdx.x & ~31u));
+                const uint32_t wfirst = __umulhi(4u * u0, 0xCCCCCCCDu) >> 2;
+                const uint32_t u4 = 4u * (u0 + (threadIdx.x & 31u));
+                const uint32_t a = __umulhi(u4, 0xCCCCCCCDu) >> 2;             // floor(8u / 10)
+                const uint32_t k0 = 2u * (u4 - 5u * a);                         // 8u mod 10
+                const uint32_t lo = __shfl_sync(0xffffffffu, x[r], (int)(a - wfirst));
+                const uint32_t hi = __shfl_sync(0xffffffffu, x[r], (int)(a - wfirst + 1u));
+                const uint32_t bits = (uint32_t)(((uint64_t)lo | ((uint64_t)hi << 30)) >> (3u * k0));
+                o = unit8<3>(bits, zf[r], sf[r]);
+            } else {
                 o = unit8<NBITS>(x[r], zf[r], sf[r]);
+            }
             if (u < prm.n_units) __stcs(reinterpret_cast<uint4*>(prm.out) + u, o);   // written once: evict first
         }
     }

@@ -36,6 +36,7 @@ struct DequantParams {
     const __half* zero;    // fp16 zero points, unless given in 8-bit form (zq)
     __half* out;
     int64_t n_units;       // n_elems / 8
+    uint32_t n_words;      // 3 bits: 32-bit words of packed codes (when < 2^32)
     int group;
     Meta8 zq, sq;
 };
