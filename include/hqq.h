@@ -237,6 +237,22 @@ int hqq_linear(const void* X, int64_t M, const void* packed, const void* scale,
                const void* zero, int64_t rows, int64_t cols, int nbits, int group,
                void* Y, int* status, void* stream);
 
+/*
+ * hqq_linear_meta -- hqq_linear for a matrix whose zero points (and,
+ * optionally, scales) are kept in their 8-bit form (hqq_meta_quantize): each
+ * group's z' = fp16((c_z - z_z) * s_z) (and s' likewise) is restored inside the
+ * kernel, then Y = X W_hat^T with W_hat = fp16((code - z') * s').  The result is
+ * that of hqq_meta_dequantize followed by hqq_linear (same tolerance).
+ *   zero_q  [in]  HOST pointer to the zero points' 8-bit form (required).
+ *   scale   [in]  fp16 scales, or NULL when scale_q is given.
+ *   scale_q [in]  HOST pointer to the scales' 8-bit form, or NULL.
+ *                 Exactly one of scale and scale_q must be non-NULL.
+ *   other arguments as for hqq_linear.
+ */
+int hqq_linear_meta(const void* X, int64_t M, const void* packed, const hqq_meta8* zero_q,
+                    const void* scale, const hqq_meta8* scale_q, int64_t rows, int64_t cols,
+                    int nbits, int group, void* Y, int* status, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* hqq_status_string(int status);
 

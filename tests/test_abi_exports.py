@@ -149,3 +149,14 @@ def test_meta_host_validation_without_gpu(lib):
     assert L.hqq_dequantize_meta(P(256), r(good), P(256), None, 64, 256, 5, 64, P(256),
                                  None) == 3
     assert L.hqq_dequantize_meta(None, None, None, None, 0, 256, 4, 64, None, None) == 0
+    # linear layer with 8-bit meta data: argument checks before any launch
+    assert L.hqq_linear_meta(P(256), 4, P(256), r(good), P(256), r(good), 64, 256, 4, 64,
+                             P(256), None, None) == 4
+    assert L.hqq_linear_meta(P(256), 4, P(256), None, P(256), None, 64, 256, 4, 64, P(256),
+                             None, None) == 1
+    assert L.hqq_linear_meta(P(256), 4, P(256), r(bad_group), P(256), None, 64, 256, 4, 64,
+                             P(256), None, None) == 3
+    assert L.hqq_linear_meta(P(264), 4, P(256), r(good), P(256), None, 64, 256, 4, 64,
+                             P(256), None, None) == 5
+    assert L.hqq_linear_meta(None, 0, None, None, None, None, 64, 256, 4, 64, None, None,
+                             None) == 0

@@ -162,3 +162,29 @@ def test_linear_bad_arguments(hqq):
     st = L.hqq_linear(P(Xd.data_ptr()), -1, P(q.packed.data_ptr()), P(q.scale.data_ptr()),
                       P(q.zero.data_ptr()), rows, cols, 4, 64, P(Yd.data_ptr()), None, None)
     assert st == 2
+
+
+@pytest.mark.parametrize("nbits,group", [(3, 64), (4, 64), (2, 16), (8, 128)])
+@pytest.mark.parametrize("M", [1, 3, 100, 1030])
+@pytest.mark.parametrize("scale_8bit", [False, True])
+def test_linear_with_8bit_meta(hqq, nbits, group, M, scale_8bit):
+    """Zero points (one group) and optionally scales (groups of 128) in their
+    8-bit form, restored inside the kernel: against the oracle's restore, Q^-1
+    and fp64 product (all inputs quantized by the oracle)."""
+    rows, cols = 200, 8 * group
+    W = synth.student_t_host((rows, cols), seed=60, stream=nbits * 10 + group).astype(np.float16)
+    q, _, r = _quantized(hqq, W, nbits, group)
+    zq = oracle.meta_quantize(r["zero"], 0)
+    sq = oracle.meta_quantize(r["scale"], 128) if scale_8bit else None
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    zq8 = hqq.Meta8(dev(zq["codes"]), dev(zq["scale"]), dev(zq["zero"]), 0)
+    sq8 = hqq.Meta8(dev(sq["codes"]), dev(sq["scale"]), dev(sq["zero"]), 128) if scale_8bit else None
+    X = _tokens(M, cols, seed=M + 5)
+    Y = hqq.hqq_linear_meta(torch.from_numpy(X).cuda(), q.packed, zq8, rows, cols, nbits, group,
+                            scale=None if scale_8bit else q.scale, scale_q=sq8)
+    torch.cuda.synchronize()
+    if scale_8bit:
+        Wh = oracle.dequantize_meta(r["codes"], group, zq, 0, scale_q=sq, scale_group=128)
+    else:
+        Wh = oracle.dequantize_meta(r["codes"], group, zq, 0, scale=r["scale"])
+    _check(Y.cpu().numpy(), X, Wh.reshape(rows, cols), f"meta {nbits}b g{group} M={M}")

@@ -15,7 +15,7 @@ from dataclasses import dataclass
 __all__ = ["HQQError", "hqq_quantize", "hqq_quantize_ex", "hqq_dequantize",
            "hqq_packed_bytes", "hqq_status_string", "QuantizedMatrix", "LIB_PATH",
            "Meta8", "hqq_meta_groups", "hqq_meta_quantize", "hqq_meta_dequantize",
-           "hqq_dequantize_meta", "hqq_linear",
+           "hqq_dequantize_meta", "hqq_linear", "hqq_linear_meta",
            "DEFAULT_P", "DEFAULT_BETA", "DEFAULT_KAPPA", "DEFAULT_ITERS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -58,6 +58,9 @@ _lib.hqq_dequantize_meta.argtypes = [_P, ctypes.POINTER(_CMeta8), _P, ctypes.POI
 _lib.hqq_dequantize_meta.restype = _I
 _lib.hqq_linear.argtypes = [_P, _I64, _P, _P, _P, _I64, _I64, _I, _I, _P, _P, _P]
 _lib.hqq_linear.restype = _I
+_lib.hqq_linear_meta.argtypes = [_P, _I64, _P, ctypes.POINTER(_CMeta8), _P,
+                                 ctypes.POINTER(_CMeta8), _I64, _I64, _I, _I, _P, _P, _P]
+_lib.hqq_linear_meta.restype = _I
 
 
 class HQQError(RuntimeError):
@@ -274,4 +277,26 @@ def hqq_linear(X, q: QuantizedMatrix, out=None, status=None, stream=None):
     _check(_lib.hqq_linear(_ptr(X), X.shape[0], _ptr(q.packed), _ptr(q.scale), _ptr(q.zero),
                            q.rows, q.cols, q.nbits, q.group, _ptr(out), _ptr(status),
                            _stream(stream)))
+    return out
+
+
+def hqq_linear_meta(X, packed, zero_q: Meta8, rows: int, cols: int, nbits: int, group: int,
+                    scale=None, scale_q: Meta8 | None = None, out=None, status=None,
+                    stream=None):
+    """hqq_linear for a matrix whose zero points (and optionally scales) are
+    kept in 8-bit form; they are restored inside the kernel (see include/hqq.h)."""
+    import torch
+    if X.dtype != torch.float16 or X.dim() != 2 or X.shape[1] != cols:
+        raise ValueError("X must be a float16 [M, cols] tensor")
+    for t, nm in ((X, "X"), (packed, "packed"), (scale, "scale"), (out, "out"),
+                  (status, "status")):
+        _check_tensor(t, nm)
+    if out is None:
+        out = torch.empty((X.shape[0], rows), dtype=torch.float16, device=X.device)
+    zc = zero_q._c()
+    sc = scale_q._c() if scale_q is not None else None
+    _check(_lib.hqq_linear_meta(_ptr(X), X.shape[0], _ptr(packed), ctypes.byref(zc),
+                                _ptr(scale), ctypes.byref(sc) if sc is not None else None,
+                                rows, cols, nbits, group, _ptr(out), _ptr(status),
+                                _stream(stream)))
     return out

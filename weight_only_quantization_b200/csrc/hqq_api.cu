@@ -314,9 +314,13 @@ extern "C" int hqq_dequantize_meta(const void* packed, const hqq_meta8* zero_q, 
     return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }
 
-extern "C" int hqq_linear(const void* X, int64_t M, const void* packed, const void* scale,
-                          const void* zero, int64_t rows, int64_t cols, int nbits, int group,
-                          void* Y, int* status, void* stream) {
+namespace {
+// Shared body of hqq_linear and hqq_linear_meta: zero_q / scale_q (host
+// structs, nullable) replace zero / scale by their 8-bit forms.
+int linear_common(const void* X, int64_t M, const void* packed, const void* scale,
+                  const void* zero, const hqq_meta8* zero_q, const hqq_meta8* scale_q,
+                  int64_t rows, int64_t cols, int nbits, int group, void* Y, int* status,
+                  void* stream) {
     int st = validate_common(rows, cols, nbits, group);
     if (st != HQQ_OK) return st;
     // the grid holds 65535 feature tiles of 128; token coordinates of the
@@ -324,12 +328,15 @@ extern "C" int hqq_linear(const void* X, int64_t M, const void* packed, const vo
     if (M < 0 || M > (((int64_t)1 << 31) - 1024)) return HQQ_ERR_SHAPE;
     if (rows > (int64_t)65535 * 128) return HQQ_ERR_SHAPE;
     if (M == 0 || rows == 0 || cols == 0) return HQQ_OK;
-    if (!X || !packed || !scale || !zero || !Y) return HQQ_ERR_NULL;
-    if (!aligned(X, 16) || !aligned(packed, packed_align(nbits)) || !aligned(scale, 2) ||
-        !aligned(zero, 2) || !aligned(Y, 2) || (status && !aligned(status, 4)))
-        return HQQ_ERR_ALIGN;
+    if (!X || !packed || !Y || (!scale && !scale_q) || (!zero && !zero_q)) return HQQ_ERR_NULL;
     LinearParams prm;
     std::memset(&prm, 0, sizeof prm);
+    if (zero_q && (st = meta8_image(zero_q, prm.zq)) != HQQ_OK) return st;
+    if (scale_q && (st = meta8_image(scale_q, prm.sq)) != HQQ_OK) return st;
+    if (!aligned(X, 16) || !aligned(packed, packed_align(nbits)) ||
+        (scale && !aligned(scale, 2)) || (zero && !aligned(zero, 2)) || !aligned(Y, 2) ||
+        (status && !aligned(status, 4)))
+        return HQQ_ERR_ALIGN;
     prm.packed = static_cast<const uint8_t*>(packed);
     prm.scale = static_cast<const __half*>(scale);
     prm.zero = static_cast<const __half*>(zero);
@@ -344,4 +351,26 @@ extern "C" int hqq_linear(const void* X, int64_t M, const void* packed, const vo
         ? launch_gemv(prm, X, nbits, static_cast<cudaStream_t>(stream))
         : launch_linear(prm, X, nbits, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" int hqq_linear(const void* X, int64_t M, const void* packed, const void* scale,
+                          const void* zero, int64_t rows, int64_t cols, int nbits, int group,
+                          void* Y, int* status, void* stream) {
+    if (M > 0 && rows > 0 && cols > 0 && (!scale || !zero)) {
+        const int st = validate_common(rows, cols, nbits, group);
+        return st != HQQ_OK ? st : HQQ_ERR_NULL;
+    }
+    return linear_common(X, M, packed, scale, zero, nullptr, nullptr, rows, cols, nbits, group, Y,
+                         status, stream);
+}
+
+extern "C" int hqq_linear_meta(const void* X, int64_t M, const void* packed,
+                               const hqq_meta8* zero_q, const void* scale,
+                               const hqq_meta8* scale_q, int64_t rows, int64_t cols, int nbits,
+                               int group, void* Y, int* status, void* stream) {
+    if (scale && scale_q) return HQQ_ERR_PARAM;
+    if (M > 0 && rows > 0 && cols > 0 && !zero_q) return HQQ_ERR_NULL;
+    return linear_common(X, M, packed, scale, nullptr, zero_q, scale_q, rows, cols, nbits, group,
+                         Y, status, stream);
 }

@@ -19,16 +19,6 @@ constexpr int kDqThreads = 256;
 constexpr int kDqUnits = 4;                          // units per thread per pass
 constexpr int kDqTile = kDqThreads * kDqUnits;
 
-// Zero point or scale of group g restored from its 8-bit form (method section
-// 4.1's 8-bit meta data): fp16((c - z2) s2) with the second-level fp16 s2, z2.
-__device__ __forceinline__ float restore_meta(const Meta8& m, int64_t g) {
-    const int64_t k = g >> m.shift;
-    const float c = (float)__ldg(m.codes + g);
-    const float v = __fmul_rn(__fsub_rn(c, __half2float(__ldg(m.zero + k))),
-                              __half2float(__ldg(m.scale + k)));
-    return __half2float(__float2half_rn(v));
-}
-
 // META bit 0: zero points in 8-bit form; bit 1: scales in 8-bit form.
 template <int NBITS, bool SMALL, int META>
 __global__ void __launch_bounds__(kDqThreads)

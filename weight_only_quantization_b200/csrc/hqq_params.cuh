@@ -28,6 +28,7 @@ struct LinearParams {
     int* status;             // optional: set to 1 if a wait inside a kernel ran out
     int64_t M, N, K;         // tokens, output features, input features
     int log2_group;
+    Meta8 zq, sq;            // 8-bit zero points / scales (codes NULL: use zero / scale)
 };
 
 struct DequantParams {

@@ -105,6 +105,23 @@ __device__ __forceinline__ uint32_t unit_merge(const UnitRaw& r) {
         return r.w0;
 }
 
+// Zero point or scale of group g restored from its 8-bit form (method section
+// 4.1's 8-bit meta data): fp16((c - z2) s2) with the second-level fp16 s2, z2.
+__device__ __forceinline__ float restore_meta(const Meta8& m, int64_t g) {
+    const int64_t k = g >> m.shift;
+    const float c = (float)__ldg(m.codes + g);
+    const float v = __fmul_rn(__fsub_rn(c, __half2float(__ldg(m.zero + k))),
+                              __half2float(__ldg(m.scale + k)));
+    return __half2float(__float2half_rn(v));
+}
+
+__device__ __forceinline__ __half restore_meta_h(const Meta8& m, int64_t g) {
+    const int64_t k = g >> m.shift;
+    const float c = (float)__ldg(m.codes + g);
+    return __float2half_rn(__fmul_rn(__fsub_rn(c, __half2float(__ldg(m.zero + k))),
+                                     __half2float(__ldg(m.scale + k))));
+}
+
 // Eight 8-bit codes (bytes of w0 then w1) -> fp16((c - z) s).  Byte i becomes
 // the mantissa of 2^23 by one byte permute; subtracting 2^23 is exact.
 __device__ __forceinline__ uint4 unit8_bytes(uint32_t w0, uint32_t w1, float z, float s) {
@@ -173,6 +190,14 @@ struct QuadCodes {
     uint32_t present;                                  // bit t: unit t inside the matrix
 };
 
+// (s, z) of group g: the stored fp16 values, or restored from their 8-bit
+// form when the layer was given one (a launch-uniform branch).
+__device__ __forceinline__ __half2 group_sz(const LinearParams& p, int64_t g) {
+    const __half s = p.sq.codes ? restore_meta_h(p.sq, g) : __ldg(p.scale + g);
+    const __half z = p.zq.codes ? restore_meta_h(p.zq, g) : __ldg(p.zero + g);
+    return __halves2half2(s, z);
+}
+
 template <int NBITS, bool SMALL, bool VEC>
 __device__ __forceinline__ void load_quad(const LinearParams& p, int64_t fbase, bool row_ok,
                                           int64_t kq, QuadCodes<NBITS>& c) {
@@ -239,10 +264,9 @@ __device__ __forceinline__ void load_quad(const LinearParams& p, int64_t fbase, 
         }
     }
     const int64_t g = f >> p.log2_group;
-    c.sz[0] = __halves2half2(__ldg(p.scale + g), __ldg(p.zero + g));
+    c.sz[0] = group_sz(p, g);
     c.sz[1] = c.sz[0];
-    if (p.log2_group == 4 && (c.present & 4u))
-        c.sz[1] = __halves2half2(__ldg(p.scale + g + 1), __ldg(p.zero + g + 1));
+    if (p.log2_group == 4 && (c.present & 4u)) c.sz[1] = group_sz(p, g + 1);
 }
 
 // Weights of unit t (0..3) of a loaded quad.
