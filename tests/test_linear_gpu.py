@@ -99,9 +99,12 @@ def test_linear_status_and_empty(hqq):
     assert E.shape == (0, rows)
 
 
-def test_linear_exact_on_integer_data(hqq):
+@pytest.mark.parametrize("M", [1, 8, 32, 96])
+def test_linear_exact_on_integer_data(hqq, M):
     """Small integers keep every product and partial sum exact in fp32, so the
-    result must equal the exact one rounded to fp16, whatever the order."""
+    result must equal the exact one rounded to fp16, whatever the order (the
+    few-token kernel's 8-token blocks at 1, 8 and 32 tokens; tensor-memory
+    tiles at 96)."""
     rows, cols, group = 256, 512, 64
     rng = np.random.default_rng(9)
     W = rng.integers(-8, 8, (rows, cols)).astype(np.float16)
@@ -109,11 +112,49 @@ def test_linear_exact_on_integer_data(hqq):
     W[:, 1::group] = 7
     q, Wh, r = _quantized(hqq, W, 4, group, iters=0)
     assert np.array_equal(Wh.astype(np.float32), W.astype(np.float32))
-    X = rng.integers(-4, 5, (96, cols)).astype(np.float16)
+    X = rng.integers(-4, 5, (M, cols)).astype(np.float16)
     Y = hqq.hqq_linear(torch.from_numpy(X).cuda(), q)
     torch.cuda.synchronize()
     ref = oracle.linear(X, Wh)
     assert np.array_equal(Y.cpu().numpy(), ref["y"])
+
+
+@pytest.mark.parametrize("nbits,group", [(3, 64), (4, 64), (2, 16), (8, 32), (1, 128)])
+@pytest.mark.parametrize("M", [4, 8, 9, 15, 24, 32, 33])
+def test_linear_decode_token_blocks(hqq, nbits, group, M):
+    """Token counts inside and at the edges of the few-token kernel's 8-token
+    MMA column blocks (1, 2 and 4 blocks) and the first count past them."""
+    rows, cols = 200, 1024
+    W = synth.student_t_host((rows, cols), seed=53, stream=nbits * 1000 + M).astype(np.float16)
+    q, Wh, _ = _quantized(hqq, W, nbits, group)
+    X = _tokens(M, cols, seed=M + 7)
+    Y = hqq.hqq_linear(torch.from_numpy(X).cuda(), q)
+    torch.cuda.synchronize()
+    _check(Y.cpu().numpy(), X, Wh, f"{nbits}b g{group} M={M}")
+
+
+@pytest.mark.parametrize("nbits,group,rows,cols", [(3, 64, 130, 1088), (4, 16, 48, 16384),
+                                                   (1, 32, 77, 96), (8, 64, 33, 512)])
+@pytest.mark.parametrize("M", [1, 5])
+def test_linear_decode_packed_alignment(hqq, nbits, group, rows, cols, M):
+    """A packed buffer that is 4-byte but not 16-byte aligned takes the
+    few-token kernel's direct-load form; it must give the same bits as the
+    staged form on an aligned copy (same products, same summation order)."""
+    W = synth.student_t_host((rows, cols), seed=54, stream=rows + nbits).astype(np.float16)
+    q, Wh, r = _quantized(hqq, W, nbits, group)
+    shift = 8 if nbits == 8 else 4
+    raw = torch.zeros(q.packed.numel() + 16, dtype=torch.uint8, device="cuda")
+    base = (16 - raw.data_ptr() % 16) % 16
+    un = raw[base + shift: base + shift + q.packed.numel()]
+    un.copy_(q.packed)
+    assert un.data_ptr() % 16 == shift
+    qu = hqq.QuantizedMatrix(un, q.scale, q.zero, rows, cols, nbits, group)
+    X = torch.from_numpy(_tokens(M, cols, seed=rows + M)).cuda()
+    Ya = hqq.hqq_linear(X, q)
+    Yu = hqq.hqq_linear(X, qu)
+    torch.cuda.synchronize()
+    assert torch.equal(Ya, Yu)
+    _check(Yu.cpu().numpy(), X.cpu().numpy(), Wh, f"unaligned {nbits}b M={M}")
 
 
 @pytest.mark.parametrize("M", [1, 16, 256, 2048])

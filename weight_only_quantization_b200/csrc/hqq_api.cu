@@ -23,7 +23,8 @@ cudaError_t launch_rtn(const RtnParams& p, int nbits, int group, cudaStream_t st
 cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_group,
                               cudaStream_t stream);
 cudaError_t launch_linear(const LinearParams& prm, const void* X, int nbits, cudaStream_t stream);
-cudaError_t launch_gemv(const LinearParams& prm, const void* X, int nbits, cudaStream_t stream);
+cudaError_t launch_decode(const LinearParams& prm, const void* X, int nbits, int64_t packed_bytes,
+                          cudaStream_t stream);
 cudaError_t launch_meta_quantize(const __half* x, int64_t n, int log2g, uint8_t* codes,
                                  __half* scale, __half* zero, cudaStream_t stream);
 cudaError_t launch_meta_dequantize(const uint8_t* codes, const __half* scale, const __half* zero,
@@ -346,9 +347,10 @@ int linear_common(const void* X, int64_t M, const void* packed, const void* scal
     prm.N = rows;
     prm.K = cols;
     prm.log2_group = log2_of_group(group);
-    // one or two tokens: streaming kernel on the CUDA cores; more: tensor cores
-    const cudaError_t err = M <= kGemvMaxTokens
-        ? launch_gemv(prm, X, nbits, static_cast<cudaStream_t>(stream))
+    // few tokens: warp-level MMAs fed from registers; more: tensor-memory tiles
+    const cudaError_t err = M <= decode_max_tokens(nbits)
+        ? launch_decode(prm, X, nbits, hqq_packed_bytes(rows, cols, nbits),
+                        static_cast<cudaStream_t>(stream))
         : launch_linear(prm, X, nbits, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }

@@ -14,10 +14,12 @@ struct Meta8 {
     int shift;
 };
 
-// Token counts up to which the linear layer runs on the CUDA cores (measured:
-// from 3 tokens on, the tensor-core kernel is faster on the 8192 x 8192 and
-// 28672 x 8192 shapes).
-constexpr int64_t kGemvMaxTokens = 2;
+// Token counts up to which the linear layer runs as warp-level MMAs fed from
+// registers (one or two 8-token m16n8k16 column blocks share each decoded
+// weight); above it, the tensor-memory kernel.  Measured on the 28672 x 8192
+// and 8192 x 28672 3-bit and 8192 x 8192 4-bit shapes: the second block pays
+// at 3 bits (16 tokens: 0.17 vs 0.23 ms), not at 4 bits.
+__host__ __device__ constexpr int64_t decode_max_tokens(int nbits) { return nbits == 3 ? 16 : 8; }
 
 // Weight-only linear layer Y = X W_hat^T on a quantized [N, K] matrix.
 struct LinearParams {
