@@ -252,6 +252,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
                  : "memory");
 }
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -339,22 +342,37 @@ decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams
             b00 = n0 * p.K * NBITS >> 5;
             b10 = n1 * p.K * NBITS >> 5;
         }
+        // copy the chunk's granules of features r and r + 8: whole 16-byte
+        // copies while a feature's slot lies inside the buffer, else clamped
+        // (zero-filled) ones
         auto fill = [&](int64_t c, int stage) {
             if (c < nchunk) {
                 const uint32_t kc = (uint32_t)(4 * S * c);
                 const Loc<NBITS, S> l0(b00, b01, kc, 0), l1(b10, b11, kc, 0);
-                const uint32_t d0 = ring_s + 4u * (uint32_t)(stage * G::STAGE + r * G::RS);
+                const uint32_t d0 = ring_s + 4u * (uint32_t)(stage * G::STAGE + r * G::RS) + 16u * j;
                 const uint32_t d1 = d0 + 4u * 8u * G::RS;
+                const uint8_t* src0 = p.packed + 16 * (l0.g + j);
+                const uint8_t* src1 = p.packed + 16 * (l1.g + j);
+                // (feature r + 8 valid and inside the buffer: so is feature r)
+                if (ok1 && 16 * (l1.g + G::GR) <= packed_bytes) {
 #pragma unroll
-                for (int t = 0; t < G::GPL; ++t) {
-                    const int gi = j + 4 * t;
-                    if (gi < G::GR) {
-                        const int64_t s0 = 16 * (l0.g + gi), s1 = 16 * (l1.g + gi);
-                        const int64_t r0 = ok0 ? packed_bytes - s0 : 0, r1 = ok1 ? packed_bytes - s1 : 0;
-                        const uint32_t c0 = r0 <= 0 ? 0u : r0 >= 16 ? 16u : (uint32_t)r0;
-                        const uint32_t c1 = r1 <= 0 ? 0u : r1 >= 16 ? 16u : (uint32_t)r1;
-                        cp_async16(d0 + 16u * gi, p.packed + (c0 ? s0 : 0), c0);
-                        cp_async16(d1 + 16u * gi, p.packed + (c1 ? s1 : 0), c1);
+                    for (int t = 0; t < G::GPL; ++t)
+                        if (j + 4 * t < G::GR) {
+                            cp_async16(d0 + 64u * t, src0 + 64 * t);
+                            cp_async16(d1 + 64u * t, src1 + 64 * t);
+                        }
+                } else {
+#pragma unroll
+                    for (int t = 0; t < G::GPL; ++t) {
+                        const int gi = j + 4 * t;
+                        if (gi < G::GR) {
+                            const int64_t s0 = 16 * (l0.g + gi), s1 = 16 * (l1.g + gi);
+                            const int64_t r0 = ok0 ? packed_bytes - s0 : 0, r1 = ok1 ? packed_bytes - s1 : 0;
+                            const uint32_t c0 = r0 <= 0 ? 0u : r0 >= 16 ? 16u : (uint32_t)r0;
+                            const uint32_t c1 = r1 <= 0 ? 0u : r1 >= 16 ? 16u : (uint32_t)r1;
+                            cp_async16(d0 + 64u * t, p.packed + (c0 ? s0 : 0), c0);
+                            cp_async16(d1 + 64u * t, p.packed + (c1 ? s1 : 0), c1);
+                        }
                     }
                 }
             }
@@ -474,6 +492,17 @@ cudaError_t launch_s(const LinearParams& p, const void* X, int64_t packed_bytes,
     const int64_t nchunk = (p.K / S + 3) / 4;
     int split = 1;
     while (split < kDcMaxSplit && tiles * split < 2 * sms && nchunk >= 2 * split * kDcWarps)
+        split *= 2;
+    // long rows: halve the chunks per CTA while each warp keeps >= 6 of them
+    // and the tiles fill the last round of resident CTAs badly
+    int per_sm = 1;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDcThreads, smem);
+    const int64_t slots = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+    auto fill_frac = [&](int64_t units) {
+        return (double)units / (double)(((units + slots - 1) / slots) * slots);
+    };
+    while (split < kDcMaxSplit && nchunk >= (int64_t)12 * split * kDcWarps &&
+           fill_frac(tiles * split * 2) > fill_frac(tiles * split) + 0.1)
         split *= 2;
     const __half* xp = static_cast<const __half*>(X);
     if (split == 1) {
