@@ -662,7 +662,7 @@ def run_rtn(views, hqq, dev, hbm_peak, qbytes, pg):
 
 def run_linear(args, views, hqq, dev, hbm_peak, tensor_peak, pg):
     """Times the weight-only linear layer Y = X W_hat^T (dequantization fused
-    into the tensor-core product) on the workload's quantized matrices:
+    into the product kernels) on the workload's quantized matrices:
     decode steps (M = 1 and 16 tokens through every matrix, as CUDA graphs) and
     a prefill of M = 2048 tokens through the first seven matrices (one layer of
     the model-shaped sets).  Beside it, torch's fp16 matmul on the dequantized
@@ -691,8 +691,9 @@ def run_linear(args, views, hqq, dev, hbm_peak, tensor_peak, pg):
         del g
         return ms
 
-    out = {"what": "Y = X W_hat^T, W_hat dequantized inside the tensor-core kernel (fp16 X and Y, "
-                   "fp32 accumulation)"}
+    out = {"what": "Y = X W_hat^T, W_hat dequantized inside the product kernels (warp-level MMAs "
+                   "fed from registers up to 16 tokens at 3 bits, tcgen05 tiles above; fp16 X and "
+                   "Y, fp32 accumulation)"}
     for M in (1, 16):
         X = torch.randn(M * maxk, device=dev).half()
         Y = torch.empty(M * maxn, dtype=torch.float16, device=dev)
