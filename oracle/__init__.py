@@ -293,6 +293,27 @@ def linear(X, W_hat) -> dict:
     return dict(y=Y64.astype(np.float16), y64=Y64, absum=absum)
 
 
+def quant_error(W, codes, scale, zero, group: int) -> np.ndarray:
+    """Delta W = W - W_hat in fp64 (exact: both are fp16), W_hat from ``dequantize``."""
+    W64 = np.asarray(W, dtype=np.float16).astype(np.float64)
+    Wh = dequantize(codes, scale, zero, group).astype(np.float64).reshape(W64.shape)
+    return W64 - Wh
+
+
+def lowrank(dW, rank: int) -> dict:
+    """Rank-r residual of the quantization error by plain SVD ("Boost 2-bit LLM
+    accuracy with EoRA", the section on finding adapters in the feature space:
+    Delta W = U Sigma V^T, B = U_r Sigma_r, A = V_r^T; the Eckart-Young optimum
+    in the Frobenius norm).  Library SVD in fp64 on the exact Delta W.
+
+    Returns B [N, r], A [r, K], the r leading singular values and all of them.
+    The factors are unique up to the signs of matching columns of B and rows of
+    A when sigma_r > sigma_{r+1}; B @ A is then unique."""
+    dW = np.asarray(dW, dtype=np.float64)
+    U, S, Vt = np.linalg.svd(dW, full_matrices=False)
+    return dict(B=U[:, :rank] * S[:rank], A=Vt[:rank].copy(), sigma=S[:rank].copy(), sigma_all=S)
+
+
 def f32_to_f16(x) -> np.ndarray:
     lib = _load()
     x = np.ascontiguousarray(x, dtype=np.float32)

@@ -509,3 +509,62 @@ def test_linear_is_x_times_w_transposed():
             assert abs(acc - out["y64"][m, n]) <= 1e-12 * out["absum"][m, n]
             assert out["y"][m, n] == np.float16(out["y64"][m, n])
     assert np.all(out["absum"] >= np.abs(out["y64"]))
+
+
+# ------------------------------------------------- low-rank residual (plain SVD)
+def _planted(n, m, s0, seed):
+    rng = np.random.default_rng(seed)
+    U0, _ = np.linalg.qr(rng.standard_normal((n, len(s0))))
+    V0, _ = np.linalg.qr(rng.standard_normal((m, len(s0))))
+    return U0, V0, U0 @ np.diag(s0) @ V0.T
+
+
+def test_lowrank_recovers_a_planted_spectrum():
+    """Delta W built from orthonormal U0, V0 and known singular values: the
+    rank-r factors must give back those values, the product U0_r S0_r V0_r^T,
+    orthonormal rows of A and B^T B = S_r^2; the residual is the Eckart-Young
+    optimum sum_{i>r} s_i^2 (computed from the planted values, not an SVD)."""
+    s0 = np.array([5.0, 3.5, 2.0, 1.25, 0.5, 0.25, 0.125, 0.0625])
+    U0, V0, dW = _planted(40, 56, s0, seed=60)
+    for r in (1, 3, 5, 8):
+        out = oracle.lowrank(dW, r)
+        assert np.allclose(out["sigma"], s0[:r], rtol=1e-12, atol=0)
+        want = U0[:, :r] @ np.diag(s0[:r]) @ V0[:, :r].T
+        assert np.abs(out["B"] @ out["A"] - want).max() <= 1e-12
+        assert np.abs(out["A"] @ out["A"].T - np.eye(r)).max() <= 1e-12
+        assert np.abs(out["B"].T @ out["B"] - np.diag(s0[:r] ** 2)).max() <= 1e-11
+        resid = np.sum((dW - out["B"] @ out["A"]) ** 2)
+        assert abs(resid - np.sum(s0[r:] ** 2)) <= 1e-12 * np.sum(s0 ** 2)
+
+
+def test_lowrank_rank_one_and_zero():
+    """A rank-one error u v^T has sigma_1 = |u| |v| and nothing else; a zero
+    error gives zero factors."""
+    rng = np.random.default_rng(61)
+    u, v = rng.standard_normal(30), rng.standard_normal(20)
+    out = oracle.lowrank(np.outer(u, v), 2)
+    assert abs(out["sigma"][0] - np.linalg.norm(u) * np.linalg.norm(v)) <= 1e-12 * out["sigma"][0]
+    assert out["sigma"][1] <= 1e-12 * out["sigma"][0]
+    assert np.abs(out["B"][:, :1] @ out["A"][:1] - np.outer(u, v)).max() <= 1e-12 * np.abs(np.outer(u, v)).max()
+    z = oracle.lowrank(np.zeros((12, 9)), 3)
+    assert np.all(z["sigma"] == 0) and np.all(z["B"] @ z["A"] == 0)
+
+
+def test_quant_error_is_w_minus_w_hat_and_within_half_a_step():
+    """Delta W is W - W_hat exactly; for min-max round-to-nearest (no solver
+    iterations) every error is at most half a code step s/2, plus what the fp16
+    storage of s and z adds (L half-spacings of s, half a spacing of z times s)
+    and the fp16 rounding of W_hat (half a spacing of |W_hat|)."""
+    N, K, g = 16, 256, 64
+    W = synth.student_t_host((N, K), seed=62, stream=0).astype(np.float16)
+    r = oracle.quantize(W, 3, g, iters=0)
+    dW = oracle.quant_error(W, r["codes"], r["scale"], r["zero"], g)
+    Wh = oracle.dequantize(r["codes"], r["scale"], r["zero"], g).reshape(N, K)
+    assert np.array_equal(dW, W.astype(np.float64) - Wh.astype(np.float64))
+    rep = lambda a: np.repeat(a.reshape(N, K // g), g, axis=1)
+    s16, z16 = rep(r["scale"]), rep(r["zero"])
+    s = s16.astype(np.float64)
+    sp = lambda a: np.spacing(np.abs(a).astype(np.float16)).astype(np.float64)
+    bound = s / 2 + 7 * sp(s16) / 2 + sp(z16) / 2 * s + sp(Wh) / 2
+    assert np.all(np.abs(dW) <= bound)
+    assert np.count_nonzero(oracle.quant_error(Wh, r["codes"], r["scale"], r["zero"], g)) == 0
