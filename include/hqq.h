@@ -256,6 +256,55 @@ int hqq_linear_meta(const void* X, int64_t M, const void* packed, const hqq_meta
 /* Human-readable name of a status code (static string, never NULL). */
 const char* hqq_status_string(int status);
 
+/*
+ * Low-rank residual of the quantization error ("Boost 2-bit LLM accuracy with
+ * EoRA", the section on finding adapters in the feature space: Delta W =
+ * W - W_hat = U Sigma V^T, B = U_r Sigma_r, A = V_r^T, the best rank-r
+ * approximation in the Frobenius norm).  Computed on the GPU by randomized
+ * subspace iteration (Halko, Martinsson and Tropp 2011, Algorithms 4.4 and
+ * 5.1) with shifted CholeskyQR3 orthonormalization and a Jacobi eigensolver
+ * for the sketch-sized problem; Delta W is formed inside every product from W
+ * and the packed codes and is never stored.  The result approximates the
+ * truncated SVD: the closer sigma_r / sigma_{r+1} is to 1, the more power
+ * iterations it needs; with a clear gap it matches the SVD to fp32 accuracy.
+ *
+ * hqq_lowrank_workspace_bytes -- device workspace bytes hqq_lowrank needs for
+ * a rows x cols matrix and a sketch of 16, 32 or 64 columns; -1 for a bad
+ * argument.
+ */
+int64_t hqq_lowrank_workspace_bytes(int64_t rows, int64_t cols, int sketch);
+
+/*
+ * hqq_lowrank -- B and A of the rank-`rank` residual and its singular values.
+ *   W        [in]  fp16 [rows, cols] row-major, 16-byte aligned: the weights
+ *                  that packed/scale/zero quantize.
+ *   packed, scale, zero, rows, cols, nbits, group [in]  as for hqq_dequantize.
+ *   rank     [in]  1 <= rank <= sketch.
+ *   sketch   [in]  16, 32 or 64 columns of the random sketch; rows and cols
+ *                  must be at least sketch, cols below 2^30.
+ *   power_iters [in] 0..16 subspace iterations (each adds two products with
+ *                  Delta W; 2 suits the nearly flat spectra of quantization
+ *                  errors).
+ *   omega    [in]  fp32 [cols, sketch] row-major, 16-byte aligned: the
+ *                  Gaussian test matrix, drawn by the caller (any seeded
+ *                  standard normal source).
+ *   B        [out] fp32 [rows, rank] row-major; A [out] fp32 [rank, cols].
+ *   sigma    [out] fp32 [rank] decreasing, or NULL.  A singular value below
+ *                  1e-7 sigma_1 gives a zero row of A (and its B column is
+ *                  sigma times the basis vector, i.e. near zero).
+ *   workspace [in] device memory, 256-byte aligned, at least
+ *                  hqq_lowrank_workspace_bytes() bytes (workspace_bytes); its
+ *                  contents on return are unspecified.
+ *   stream   [in]  cudaStream_t or NULL; asynchronous.
+ * Errors: HQQ_ERR_UNSUPPORTED (sketch), HQQ_ERR_PARAM (rank, power_iters,
+ * workspace too small), HQQ_ERR_SHAPE (rows or cols below sketch),
+ * HQQ_ERR_NULL, HQQ_ERR_ALIGN, plus those of hqq_dequantize.
+ */
+int hqq_lowrank(const void* W, const void* packed, const void* scale, const void* zero,
+                int64_t rows, int64_t cols, int nbits, int group, int rank, int sketch,
+                int power_iters, const float* omega, float* B, float* A, float* sigma,
+                void* workspace, int64_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

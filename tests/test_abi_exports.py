@@ -160,3 +160,41 @@ def test_meta_host_validation_without_gpu(lib):
                              P(256), None, None) == 5
     assert L.hqq_linear_meta(None, 0, None, None, None, None, 64, 256, 4, 64, None, None,
                              None) == 0
+
+
+def test_lowrank_host_validation_without_gpu(lib):
+    L = lib._lib
+    P = lambda v: ctypes.c_void_p(v)
+    ws = L.hqq_lowrank_workspace_bytes(256, 512, 32)
+    assert ws > 0 and ws % 256 == 0
+    assert L.hqq_lowrank_workspace_bytes(256, 512, 24) == -1
+    assert L.hqq_lowrank_workspace_bytes(-1, 512, 32) == -1
+    assert L.hqq_lowrank_workspace_bytes(256, 512, 64) > ws
+
+    def call(rows=256, cols=512, nbits=4, group=64, rank=8, sketch=32, iters=2, omega=256,
+             W=256, B=256, A=256, sigma=None, wsp=256, wsb=ws):
+        if wsb == ws:
+            wsb = L.hqq_lowrank_workspace_bytes(max(rows, 0), max(cols, 0), sketch) \
+                if sketch in (16, 32, 64) and rows >= 0 and cols >= 0 else ws
+        return L.hqq_lowrank(P(W) if W else None, P(256), P(256), P(256), rows, cols, nbits,
+                             group, rank, sketch, iters, P(omega) if omega else None,
+                             P(B) if B else None, P(A) if A else None,
+                             P(sigma) if sigma else None, P(wsp) if wsp else None, wsb, None)
+    assert call(sketch=24) == 3
+    assert call(nbits=5) == 3
+    assert call(rank=0) == 4
+    assert call(rank=33) == 4
+    assert call(iters=-1) == 4
+    assert call(iters=17) == 4
+    assert call(rows=16) == 2
+    assert call(cols=16, group=16) == 2
+    assert call(cols=500) == 2
+    assert call(W=0) == 1
+    assert call(omega=0) == 1
+    assert call(wsp=0) == 1
+    assert call(wsb=ws - 1) == 4
+    assert call(W=264) == 5
+    assert call(omega=260) == 5
+    assert call(B=258) == 5
+    assert call(sigma=258) == 5
+    assert call(wsp=384) == 5

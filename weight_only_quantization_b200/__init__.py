@@ -61,6 +61,11 @@ _lib.hqq_linear.restype = _I
 _lib.hqq_linear_meta.argtypes = [_P, _I64, _P, ctypes.POINTER(_CMeta8), _P,
                                  ctypes.POINTER(_CMeta8), _I64, _I64, _I, _I, _P, _P, _P]
 _lib.hqq_linear_meta.restype = _I
+_lib.hqq_lowrank_workspace_bytes.argtypes = [_I64, _I64, _I]
+_lib.hqq_lowrank_workspace_bytes.restype = _I64
+_lib.hqq_lowrank.argtypes = [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                             _I64, _P]
+_lib.hqq_lowrank.restype = _I
 
 
 class HQQError(RuntimeError):
@@ -300,3 +305,32 @@ def hqq_linear_meta(X, packed, zero_q: Meta8, rows: int, cols: int, nbits: int, 
                                 rows, cols, nbits, group, _ptr(out), _ptr(status),
                                 _stream(stream)))
     return out
+
+
+def hqq_lowrank(W, q: QuantizedMatrix, rank: int, omega, power_iters: int = 2, workspace=None,
+                stream=None):
+    """Rank-r residual B [rows, rank], A [rank, cols] (fp32) of the quantization
+    error W - W_hat, with the r leading singular values (see include/hqq.h).
+    ``omega`` is the fp32 [cols, sketch] Gaussian test matrix (sketch 16, 32 or
+    64), drawn by the caller; the workspace is allocated here unless given."""
+    import torch
+    if W.dtype != torch.float16 or tuple(W.shape) != (q.rows, q.cols):
+        raise ValueError("W must be the float16 [rows, cols] matrix that q quantizes")
+    if omega.dtype != torch.float32 or omega.dim() != 2 or omega.shape[0] != q.cols:
+        raise ValueError("omega must be a float32 [cols, sketch] tensor")
+    for t, nm in ((W, "W"), (omega, "omega"), (workspace, "workspace")):
+        _check_tensor(t, nm)
+    sketch = omega.shape[1]
+    need = _lib.hqq_lowrank_workspace_bytes(q.rows, q.cols, sketch)
+    if need < 0:
+        raise ValueError("sketch must be 16, 32 or 64")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    B = torch.empty((q.rows, rank), dtype=torch.float32, device=W.device)
+    A = torch.empty((rank, q.cols), dtype=torch.float32, device=W.device)
+    sigma = torch.empty(rank, dtype=torch.float32, device=W.device)
+    _check(_lib.hqq_lowrank(_ptr(W), _ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols,
+                            q.nbits, q.group, rank, sketch, power_iters, _ptr(omega), _ptr(B),
+                            _ptr(A), _ptr(sigma), _ptr(workspace), workspace.numel(),
+                            _stream(stream)))
+    return B, A, sigma

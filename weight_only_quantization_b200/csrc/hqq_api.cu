@@ -25,6 +25,11 @@ cudaError_t launch_dequantize(const DequantParams& prm, int nbits, int log2_grou
 cudaError_t launch_linear(const LinearParams& prm, const void* X, int nbits, cudaStream_t stream);
 cudaError_t launch_decode(const LinearParams& prm, const void* X, int nbits, int64_t packed_bytes,
                           cudaStream_t stream);
+int64_t lowrank_workspace_bytes(int64_t N, int64_t K, int sketch);
+cudaError_t launch_lowrank(const void* W, const uint8_t* packed, const __half* scale,
+                           const __half* zero, int64_t N, int64_t K, int nbits, int log2_group,
+                           int rank, int sketch, int power_iters, const float* omega, float* B,
+                           float* A, float* sigma, void* ws, cudaStream_t st);
 cudaError_t launch_meta_quantize(const __half* x, int64_t n, int log2g, uint8_t* codes,
                                  __half* scale, __half* zero, cudaStream_t stream);
 cudaError_t launch_meta_dequantize(const uint8_t* codes, const __half* scale, const __half* zero,
@@ -375,4 +380,38 @@ extern "C" int hqq_linear_meta(const void* X, int64_t M, const void* packed,
     if (M > 0 && rows > 0 && cols > 0 && !zero_q) return HQQ_ERR_NULL;
     return linear_common(X, M, packed, scale, nullptr, zero_q, scale_q, rows, cols, nbits, group,
                          Y, status, stream);
+}
+
+extern "C" int64_t hqq_lowrank_workspace_bytes(int64_t rows, int64_t cols, int sketch) {
+    if (rows < 0 || cols < 0 || (sketch != 16 && sketch != 32 && sketch != 64)) return -1;
+    return lowrank_workspace_bytes(rows, cols, sketch);
+}
+
+extern "C" int hqq_lowrank(const void* W, const void* packed, const void* scale, const void* zero,
+                           int64_t rows, int64_t cols, int nbits, int group, int rank, int sketch,
+                           int power_iters, const float* omega, float* B, float* A, float* sigma,
+                           void* workspace, int64_t workspace_bytes, void* stream) {
+    int st = validate_common(rows, cols, nbits, group);
+    if (st != HQQ_OK) return st;
+    if (sketch != 16 && sketch != 32 && sketch != 64) return HQQ_ERR_UNSUPPORTED;
+    if (rank < 1 || rank > sketch || power_iters < 0 || power_iters > 16) return HQQ_ERR_PARAM;
+    if (rows < sketch || cols < sketch || cols >= ((int64_t)1 << 30)) return HQQ_ERR_SHAPE;
+    if (!W || !packed || !scale || !zero || !omega || !B || !A || !workspace) return HQQ_ERR_NULL;
+    if (workspace_bytes < lowrank_workspace_bytes(rows, cols, sketch)) return HQQ_ERR_PARAM;
+    if (!aligned(W, 16) || !aligned(packed, packed_align(nbits)) || !aligned(scale, 2) ||
+        !aligned(zero, 2) || !aligned(omega, 16) || !aligned(B, 4) || !aligned(A, 4) ||
+        (sigma && !aligned(sigma, 4)) || !aligned(workspace, 256))
+        return HQQ_ERR_ALIGN;
+    float* sg = sigma;
+    float* scratch_sigma = nullptr;
+    if (!sg) {                          // the solver always writes sigma: use workspace slack
+        scratch_sigma = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                 lowrank_workspace_bytes(rows, cols, sketch) - 256);
+        sg = scratch_sigma;
+    }
+    const cudaError_t err = launch_lowrank(
+        W, static_cast<const uint8_t*>(packed), static_cast<const __half*>(scale),
+        static_cast<const __half*>(zero), rows, cols, nbits, log2_of_group(group), rank, sketch,
+        power_iters, omega, B, A, sg, workspace, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }

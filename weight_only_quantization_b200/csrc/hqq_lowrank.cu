@@ -1,0 +1,529 @@
+// hqq_lowrank.cu -- rank-r residual of the quantization error: Delta W =
+// W - W_hat ~ B A with B = U_r Sigma_r, A = V_r^T, the plain-SVD compensation
+// of "Boost 2-bit LLM accuracy with EoRA" (section on finding adapters in the
+// feature space).  Delta W is never stored: every product forms it tile by
+// tile from the fp16 W and the packed codes (W_hat exactly as hqq_dequantize
+// restores it, the difference in fp32).
+//
+// The truncated SVD is computed by randomized subspace iteration (Halko,
+// Martinsson and Tropp, "Finding structure with randomness", SIAM Review 2011:
+// Algorithm 4.4 for the range, Algorithm 5.1 for the factorization) with a
+// sketch of l = 16, 32 or 64 columns and a Gaussian test matrix given by the
+// caller:
+//   Y = orth(dW Omega); q times { Z = orth(dW^T Y); Y = orth(dW Z) };
+//   Z = dW^T Y (so Z^T = Q^T dW, l x K); Z^T Z = U_s Lambda U_s^T (Jacobi);
+//   sigma = sqrt(Lambda); B = Y U_s,r Sigma_r; A = (Z U_s,r Sigma_r^-1)^T.
+// orth() is shifted CholeskyQR3 (Fukaya, Kannan, Nakatsukasa, Yamamoto and
+// Yanagisawa, SIAM J. Sci. Comput. 2020): three passes of Gram matrix (fp64),
+// Cholesky factor R and X <- X R^-1, the first with a small diagonal shift.
+// The l x l eigenproblem is solved by cyclic Jacobi in fp64 (Golub and Van
+// Loan, "Matrix Computations", the symmetric Schur rotation), L/2 disjoint
+// rotations at a time in round-robin order.
+#include "hqq_unpack.cuh"
+
+namespace hqq {
+
+namespace {
+
+constexpr int kLrThreads = 256;
+
+struct LrParams {
+    const __half* W;
+    const uint8_t* packed;
+    const __half* scale;
+    const __half* zero;
+    int64_t N, K;
+    int log2_group;
+};
+
+// Delta W of the 8 weights at flat index f (f % 8 == 0) in fp32.
+template <int NBITS>
+__device__ __forceinline__ void unit_delta(const LrParams& p, int64_t f, float (&d)[8]) {
+    const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.W + f));
+    const UnitRaw ur = unit_fetch<NBITS, false>(p.packed, f >> 3);
+    const int64_t g = f >> p.log2_group;
+    const uint4 hv =
+        unit8_raw<NBITS>(ur, __half2float(__ldg(p.zero + g)), __half2float(__ldg(p.scale + g)));
+    const __half2* w2 = reinterpret_cast<const __half2*>(&wv);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&hv);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 a = __half22float2(w2[i]), b = __half22float2(h2[i]);
+        d[2 * i] = __fsub_rn(a.x, b.x);
+        d[2 * i + 1] = __fsub_rn(a.y, b.y);
+    }
+}
+
+// Y[N, L] = dW[N, K] M[K, L].  CTA: 32 rows x L; per 32-wide k-tile, threads
+// 0..127 form the dW tile (one unit each), 128..255 stage M; thread t then
+// owns row t/8 and L/8 consecutive columns.
+template <int NBITS, int L>
+__global__ void __launch_bounds__(kLrThreads)
+lr_right_kernel(const __grid_constant__ LrParams p, const float* __restrict__ M,
+                float* __restrict__ Y) {
+    constexpr int CPT = L / 8;
+    __shared__ float As[32][33];                          // [k][row]
+    __shared__ __align__(16) float Bs[32][L];             // [k][column]
+    const int t = threadIdx.x;
+    const int64_t n0 = (int64_t)blockIdx.x * 32;
+    const int row = t >> 3, c0 = (t & 7) * CPT;
+    float acc[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[c] = 0.0f;
+    for (int64_t k0 = 0; k0 < p.K; k0 += 32) {
+        if (t < 128) {
+            const int r = t >> 2, u = t & 3;
+            const int64_t n = n0 + r, k = k0 + 8 * u;
+            float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (n < p.N && k < p.K) unit_delta<NBITS>(p, n * p.K + k, d);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) As[8 * u + i][r] = d[i];
+        } else {
+            for (int idx = t - 128; idx < 32 * L / 4; idx += 128) {
+                const int kk = idx / (L / 4), c4 = idx % (L / 4);
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (k0 + kk < p.K) v = __ldg(reinterpret_cast<const float4*>(M + (k0 + kk) * L) + c4);
+                *reinterpret_cast<float4*>(&Bs[kk][4 * c4]) = v;
+            }
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {
+            const float a = As[kk][row];
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) acc[c] = __fmaf_rn(a, Bs[kk][c0 + c], acc[c]);
+        }
+        __syncthreads();
+    }
+    if (n0 + row < p.N) {
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) Y[(n0 + row) * L + c0 + c] = acc[c];
+    }
+}
+
+// Zp[split, K, L] = sum over the split's rows of dW[row, k] Y[row, :].  CTA:
+// 32 columns k x L, rows [blockIdx.y * rps, +rps) in 32-row tiles.
+template <int NBITS, int L>
+__global__ void __launch_bounds__(kLrThreads)
+lr_left_kernel(const __grid_constant__ LrParams p, const float* __restrict__ Y,
+               float* __restrict__ Zp, int64_t rps) {
+    constexpr int CPT = L / 8;
+    __shared__ float As[32][33];                          // [row][k]
+    __shared__ __align__(16) float Bs[32][L];             // [row][column]
+    const int t = threadIdx.x;
+    const int64_t k0 = (int64_t)blockIdx.x * 32;
+    const int64_t rb = (int64_t)blockIdx.y * rps;
+    const int64_t re = rb + rps < p.N ? rb + rps : p.N;
+    const int kk = t >> 3, c0 = (t & 7) * CPT;
+    float acc[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[c] = 0.0f;
+    for (int64_t r0 = rb; r0 < re; r0 += 32) {
+        if (t < 128) {
+            const int r = t >> 2, u = t & 3;
+            const int64_t n = r0 + r, k = k0 + 8 * u;
+            float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (n < re && k < p.K) unit_delta<NBITS>(p, n * p.K + k, d);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) As[r][8 * u + i] = d[i];
+        } else {
+            for (int idx = t - 128; idx < 32 * L / 4; idx += 128) {
+                const int r = idx / (L / 4), c4 = idx % (L / 4);
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (r0 + r < re) v = __ldg(reinterpret_cast<const float4*>(Y + (r0 + r) * L) + c4);
+                *reinterpret_cast<float4*>(&Bs[r][4 * c4]) = v;
+            }
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int r = 0; r < 32; ++r) {
+            const float a = As[r][kk];
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) acc[c] = __fmaf_rn(a, Bs[r][c0 + c], acc[c]);
+        }
+        __syncthreads();
+    }
+    if (k0 + kk < p.K) {
+        float* z = Zp + ((int64_t)blockIdx.y * p.K + k0 + kk) * L + c0;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) z[c] = acc[c];
+    }
+}
+
+// Z[i] = sum_s Zp[s * n + i].
+__global__ void __launch_bounds__(kLrThreads)
+lr_reduce_kernel(const float* __restrict__ Zp, int splits, int64_t n, float* __restrict__ Z) {
+    for (int64_t i = (int64_t)blockIdx.x * kLrThreads + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * kLrThreads) {
+        float s = Zp[i];
+        for (int k = 1; k < splits; ++k) s = __fadd_rn(s, Zp[k * n + i]);
+        Z[i] = s;
+    }
+}
+
+// GP[block] = X[rows of the block]^T X[rows of the block] in fp64 (L x L).
+template <int L>
+__global__ void __launch_bounds__(kLrThreads)
+lr_gram_kernel(const float* __restrict__ X, int64_t n, int64_t rpb, double* __restrict__ GP) {
+    constexpr int EPT = L * L / kLrThreads;
+    __shared__ float Xs[32][L + 1];
+    const int t = threadIdx.x;
+    const int e0 = t * EPT, i = e0 / L, j0 = e0 % L;
+    double acc[EPT];
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) acc[e] = 0.0;
+    const int64_t rb = (int64_t)blockIdx.x * rpb;
+    const int64_t re = rb + rpb < n ? rb + rpb : n;
+    for (int64_t r0 = rb; r0 < re; r0 += 32) {
+        for (int idx = t; idx < 32 * L; idx += kLrThreads) {
+            const int r = idx / L, c = idx % L;
+            Xs[r][c] = r0 + r < re ? X[(r0 + r) * L + c] : 0.0f;
+        }
+        __syncthreads();
+        for (int r = 0; r < 32; ++r) {
+            const double a = (double)Xs[r][i];
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) acc[e] = fma(a, (double)Xs[r][j0 + e], acc[e]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) GP[(int64_t)blockIdx.x * L * L + e0 + e] = acc[e];
+}
+
+// One CTA: G = sum of the nparts Gram blocks (+ shift * trace / L on the
+// diagonal when shift > 0), G = R^T R (upper R), Rinv = R^-1 (fp32 out).  A
+// pivot at most 1e-20 of G's largest diagonal (a column with no norm left)
+// becomes 1 with a zero row of R: that column of X R^-1 stays as it is (near
+// zero) instead of being blown up.
+template <int L>
+__global__ void __launch_bounds__(kLrThreads)
+lr_chol_kernel(const double* __restrict__ GP, int nparts, double shift, float* __restrict__ Rinv) {
+    extern __shared__ double lr_dsm[];                    // G, R, Ri: L x (L + 1) each
+    auto G = reinterpret_cast<double(*)[L + 1]>(lr_dsm);
+    auto R = reinterpret_cast<double(*)[L + 1]>(lr_dsm + L * (L + 1));
+    auto Ri = reinterpret_cast<double(*)[L + 1]>(lr_dsm + 2 * L * (L + 1));
+    const int t = threadIdx.x;
+    for (int e = t; e < L * L; e += kLrThreads) {
+        double s = 0.0;
+        for (int q = 0; q < nparts; ++q) s += GP[(int64_t)q * L * L + e];
+        G[e / L][e % L] = s;
+        R[e / L][e % L] = 0.0;
+    }
+    __syncthreads();
+    __shared__ double thr;
+    __shared__ int live;
+    if (t == 0) {
+        double tr = 0.0, dmax = 0.0;
+        for (int i = 0; i < L; ++i) {
+            tr += G[i][i];
+            dmax = G[i][i] > dmax ? G[i][i] : dmax;
+        }
+        const double sh = shift * tr / L;
+        for (int i = 0; i < L; ++i) G[i][i] += sh;
+        thr = 1e-20 * dmax + 1e-300;
+    }
+    __syncthreads();
+    for (int k = 0; k < L; ++k) {
+        if (t == 0) {
+            const double d = G[k][k];
+            live = d > thr;
+            R[k][k] = live ? sqrt(d) : 1.0;
+        }
+        __syncthreads();
+        for (int j = k + 1 + t; j < L; j += kLrThreads) R[k][j] = live ? G[k][j] / R[k][k] : 0.0;
+        __syncthreads();
+        for (int e = t; e < L * L; e += kLrThreads) {
+            const int i = e / L, j = e % L;
+            if (i > k && j >= i) G[i][j] -= R[k][i] * R[k][j];
+        }
+        __syncthreads();
+    }
+    for (int j = t; j < L; j += kLrThreads) {      // column j of the upper inverse
+        for (int i = L - 1; i > j; --i) Ri[i][j] = 0.0;
+        for (int i = j; i >= 0; --i) {
+            double s = i == j ? 1.0 : 0.0;
+            for (int k = i + 1; k <= j; ++k) s -= R[i][k] * Ri[k][j];
+            Ri[i][j] = s / R[i][i];
+        }
+    }
+    __syncthreads();
+    for (int e = t; e < L * L; e += kLrThreads) Rinv[e] = (float)Ri[e / L][e % L];
+}
+
+// out = X[n, L] Rm[L, L] restricted to the first ncols columns; one row per
+// thread (in place when out == X: the row is read before it is written).
+// trans: out[j * ostride + row], else out[row * ostride + j].
+template <int L>
+__global__ void __launch_bounds__(kLrThreads)
+lr_apply_kernel(const float* X, int64_t n, const float* __restrict__ Rm, int ncols, float* out,
+                int64_t ostride, int trans) {
+    __shared__ float Rs[L][L];
+    for (int e = threadIdx.x; e < L * L; e += kLrThreads) Rs[e / L][e % L] = Rm[e];
+    __syncthreads();
+    const int64_t row = (int64_t)blockIdx.x * kLrThreads + threadIdx.x;
+    if (row >= n) return;
+    float x[L];
+#pragma unroll
+    for (int c = 0; c < L; c += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(X + row * L + c);
+        x[c] = v.x;
+        x[c + 1] = v.y;
+        x[c + 2] = v.z;
+        x[c + 3] = v.w;
+    }
+    constexpr int JB = L < 16 ? L : 16;
+    for (int j0 = 0; j0 < ncols; j0 += JB) {
+        float o[JB];
+#pragma unroll
+        for (int jj = 0; jj < JB; ++jj) o[jj] = 0.0f;
+#pragma unroll 8
+        for (int c = 0; c < L; ++c)
+#pragma unroll
+            for (int jj = 0; jj < JB; ++jj)
+                if (j0 + jj < L) o[jj] = __fmaf_rn(x[c], Rs[c][j0 + jj], o[jj]);
+#pragma unroll
+        for (int jj = 0; jj < JB; ++jj) {
+            const int j = j0 + jj;
+            if (j < ncols) {
+                if (trans) out[(int64_t)j * ostride + row] = o[jj];
+                else out[row * ostride + j] = o[jj];
+            }
+        }
+    }
+}
+
+// One CTA: S = sum of the Gram blocks (symmetric L x L), cyclic Jacobi until
+// the off-diagonal mass is below 1e-28 of the total (at most 40 sweeps);
+// eigenvalues sorted decreasing, sigma = sqrt(max(lambda, 0)).  Writes
+// Mr = U_s,r Sigma_r and Mi = U_s,r Sigma_r^-1 (L x L, columns >= rank zero;
+// a column whose sigma is at most 1e-7 sigma_1 is zero in Mi) and sigma[rank].
+template <int L>
+__global__ void __launch_bounds__(kLrThreads)
+lr_jacobi_kernel(const double* __restrict__ GP, int nparts, int rank, float* __restrict__ Mr,
+                 float* __restrict__ Mi, float* __restrict__ sigma) {
+    extern __shared__ double lr_dsm[];                    // A, V: L x (L + 1) each
+    auto A = reinterpret_cast<double(*)[L + 1]>(lr_dsm);
+    auto V = reinterpret_cast<double(*)[L + 1]>(lr_dsm + L * (L + 1));
+    __shared__ double rc[L / 2], rs[L / 2];
+    __shared__ int rp[L / 2], rq[L / 2];
+    __shared__ double off_rel;
+    __shared__ int perm[L];
+    __shared__ double sg[L];
+    const int t = threadIdx.x;
+    for (int e = t; e < L * L; e += kLrThreads) {
+        double s = 0.0;
+        for (int q = 0; q < nparts; ++q) s += GP[(int64_t)q * L * L + e];
+        A[e / L][e % L] = s;
+        V[e / L][e % L] = (e / L == e % L) ? 1.0 : 0.0;
+    }
+    __syncthreads();
+    for (int sweep = 0; sweep < 40; ++sweep) {
+        if (t == 0) {
+            double off = 0.0, tot = 0.0;
+            for (int i = 0; i < L; ++i)
+                for (int j = 0; j < L; ++j) {
+                    const double a2 = A[i][j] * A[i][j];
+                    tot += a2;
+                    if (i != j) off += a2;
+                }
+            off_rel = tot > 0.0 ? off / tot : 0.0;
+        }
+        __syncthreads();
+        if (off_rel < 1e-28) break;
+        for (int step = 0; step < L - 1; ++step) {
+            if (t < L / 2) {                       // round-robin pairs (circle method)
+                const int p = t == 0 ? 0 : ((t - 1 + step) % (L - 1)) + 1;
+                const int q = ((L - 2 - t + step) % (L - 1)) + 1;
+                const double apq = A[p][q];
+                double c = 1.0, s = 0.0;
+                if (fabs(apq) > 1e-300) {
+                    const double tau = (A[q][q] - A[p][p]) / (2.0 * apq);
+                    const double tt = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+                    c = 1.0 / sqrt(1.0 + tt * tt);
+                    s = tt * c;
+                }
+                rp[t] = p;
+                rq[t] = q;
+                rc[t] = c;
+                rs[t] = s;
+            }
+            __syncthreads();
+            for (int e = t; e < (L / 2) * L; e += kLrThreads) {      // rows: A <- J^T A
+                const int k = e / L, j = e % L, p = rp[k], q = rq[k];
+                const double ap = A[p][j], aq = A[q][j];
+                A[p][j] = rc[k] * ap - rs[k] * aq;
+                A[q][j] = rs[k] * ap + rc[k] * aq;
+            }
+            __syncthreads();
+            for (int e = t; e < (L / 2) * L; e += kLrThreads) {      // columns: A <- A J, V <- V J
+                const int k = e / L, j = e % L, p = rp[k], q = rq[k];
+                const double ap = A[j][p], aq = A[j][q];
+                A[j][p] = rc[k] * ap - rs[k] * aq;
+                A[j][q] = rs[k] * ap + rc[k] * aq;
+                const double vp = V[j][p], vq = V[j][q];
+                V[j][p] = rc[k] * vp - rs[k] * vq;
+                V[j][q] = rs[k] * vp + rc[k] * vq;
+            }
+            __syncthreads();
+        }
+    }
+    if (t == 0) {
+        for (int i = 0; i < L; ++i) perm[i] = i;
+        for (int i = 0; i < L; ++i) {              // selection sort, decreasing eigenvalue
+            int b = i;
+            for (int j = i + 1; j < L; ++j)
+                if (A[perm[j]][perm[j]] > A[perm[b]][perm[b]]) b = j;
+            const int tmp = perm[i];
+            perm[i] = perm[b];
+            perm[b] = tmp;
+        }
+        for (int i = 0; i < L; ++i) {
+            const double lam = A[perm[i]][perm[i]];
+            sg[i] = lam > 0.0 ? sqrt(lam) : 0.0;
+        }
+    }
+    __syncthreads();
+    const double floor_sg = 1e-7 * sg[0];
+    for (int e = t; e < L * L; e += kLrThreads) {
+        const int c = e / L, j = e % L;
+        const bool live = j < rank;
+        const double u = V[c][perm[j]];
+        Mr[e] = live ? (float)(u * sg[j]) : 0.0f;
+        Mi[e] = live && sg[j] > floor_sg && sg[j] > 0.0 ? (float)(u / sg[j]) : 0.0f;
+    }
+    if (t < rank) sigma[t] = (float)sg[t];
+}
+
+constexpr int64_t kGramRows = 1024;                // rows per Gram block
+
+int64_t align256(int64_t b) { return (b + 255) & ~(int64_t)255; }
+
+int64_t left_splits(int64_t K) {
+    const int64_t tiles = (K + 31) / 32;
+    int64_t s = (512 + tiles - 1) / tiles;
+    return s < 1 ? 1 : s > 16 ? 16 : s;
+}
+
+struct LrWorkspace {
+    float *Y, *Z, *Zp, *R, *Mr, *Mi;
+    double* GP;
+};
+
+LrWorkspace carve(void* ws, int64_t N, int64_t K, int L) {
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    LrWorkspace w;
+    w.Y = reinterpret_cast<float*>(b);
+    b += align256(N * L * 4);
+    w.Z = reinterpret_cast<float*>(b);
+    b += align256(K * L * 4);
+    w.Zp = reinterpret_cast<float*>(b);
+    b += align256(left_splits(K) * K * L * 4);
+    w.GP = reinterpret_cast<double*>(b);
+    const int64_t parts = ((N > K ? N : K) + kGramRows - 1) / kGramRows;
+    b += align256(parts * (int64_t)L * L * 8);
+    w.R = reinterpret_cast<float*>(b);
+    b += align256((int64_t)L * L * 4);
+    w.Mr = reinterpret_cast<float*>(b);
+    b += align256((int64_t)L * L * 4);
+    w.Mi = reinterpret_cast<float*>(b);
+    return w;
+}
+
+template <int NBITS, int L>
+cudaError_t run(const LrParams& p, int rank, int power_iters, const float* omega, float* B,
+                float* A, float* sigma, void* ws, cudaStream_t st) {
+    const LrWorkspace w = carve(ws, p.N, p.K, L);
+    constexpr int kCholSmem = 3 * L * (L + 1) * 8, kJacobiSmem = 2 * L * (L + 1) * 8;
+    cudaError_t e = cudaFuncSetAttribute(lr_chol_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kCholSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(lr_jacobi_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kJacobiSmem);
+    if (e != cudaSuccess) return e;
+    const int64_t S = left_splits(p.K);
+    const int64_t rps = ((p.N + S - 1) / S + 31) / 32 * 32;
+    auto right = [&](const float* M) {
+        lr_right_kernel<NBITS, L><<<(unsigned)((p.N + 31) / 32), kLrThreads, 0, st>>>(p, M, w.Y);
+    };
+    auto left = [&]() {
+        lr_left_kernel<NBITS, L><<<dim3((unsigned)((p.K + 31) / 32), (unsigned)S), kLrThreads, 0, st>>>(
+            p, w.Y, w.Zp, rps);
+        lr_reduce_kernel<<<592, kLrThreads, 0, st>>>(w.Zp, (int)S, p.K * L, w.Z);
+    };
+    auto gram = [&](const float* X, int64_t n) {
+        const int64_t parts = (n + kGramRows - 1) / kGramRows;
+        lr_gram_kernel<L><<<(unsigned)parts, kLrThreads, 0, st>>>(X, n, kGramRows, w.GP);
+        return (int)parts;
+    };
+    auto orth = [&](float* X, int64_t n) {
+        for (int pass = 0; pass < 3; ++pass) {
+            const int parts = gram(X, n);
+            lr_chol_kernel<L><<<1, kLrThreads, kCholSmem, st>>>(w.GP, parts, pass == 0 ? 1e-9 : 0.0, w.R);
+            lr_apply_kernel<L><<<(unsigned)((n + kLrThreads - 1) / kLrThreads), kLrThreads, 0, st>>>(
+                X, n, w.R, L, X, L, 0);
+        }
+    };
+    right(omega);
+    orth(w.Y, p.N);
+    for (int it = 0; it < power_iters; ++it) {
+        left();
+        orth(w.Z, p.K);
+        right(w.Z);
+        orth(w.Y, p.N);
+    }
+    left();
+    const int parts = gram(w.Z, p.K);
+    lr_jacobi_kernel<L><<<1, kLrThreads, kJacobiSmem, st>>>(w.GP, parts, rank, w.Mr, w.Mi, sigma);
+    lr_apply_kernel<L><<<(unsigned)((p.N + kLrThreads - 1) / kLrThreads), kLrThreads, 0, st>>>(
+        w.Y, p.N, w.Mr, rank, B, rank, 0);
+    lr_apply_kernel<L><<<(unsigned)((p.K + kLrThreads - 1) / kLrThreads), kLrThreads, 0, st>>>(
+        w.Z, p.K, w.Mi, rank, A, p.K, 1);
+    return cudaGetLastError();
+}
+
+template <int NBITS>
+cudaError_t run_l(const LrParams& p, int rank, int sketch, int power_iters, const float* omega,
+                  float* B, float* A, float* sigma, void* ws, cudaStream_t st) {
+    switch (sketch) {
+        case 16: return run<NBITS, 16>(p, rank, power_iters, omega, B, A, sigma, ws, st);
+        case 32: return run<NBITS, 32>(p, rank, power_iters, omega, B, A, sigma, ws, st);
+        case 64: return run<NBITS, 64>(p, rank, power_iters, omega, B, A, sigma, ws, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+// Bytes of workspace the low-rank residual needs for an N x K matrix and a
+// sketch of l columns (the last 256 bytes hold sigma when the caller gives none).
+int64_t lowrank_workspace_bytes(int64_t N, int64_t K, int sketch) {
+    const int64_t L = sketch;
+    const int64_t parts = ((N > K ? N : K) + kGramRows - 1) / kGramRows;
+    return align256(N * L * 4) + align256(K * L * 4) + align256(left_splits(K) * K * L * 4) +
+           align256(parts * L * L * 8) + 3 * align256(L * L * 4) + 256;   // + sigma slot
+}
+
+cudaError_t launch_lowrank(const void* W, const uint8_t* packed, const __half* scale,
+                           const __half* zero, int64_t N, int64_t K, int nbits, int log2_group,
+                           int rank, int sketch, int power_iters, const float* omega, float* B,
+                           float* A, float* sigma, void* ws, cudaStream_t st) {
+    LrParams p;
+    p.W = static_cast<const __half*>(W);
+    p.packed = packed;
+    p.scale = scale;
+    p.zero = zero;
+    p.N = N;
+    p.K = K;
+    p.log2_group = log2_group;
+    switch (nbits) {
+        case 1: return run_l<1>(p, rank, sketch, power_iters, omega, B, A, sigma, ws, st);
+        case 2: return run_l<2>(p, rank, sketch, power_iters, omega, B, A, sigma, ws, st);
+        case 3: return run_l<3>(p, rank, sketch, power_iters, omega, B, A, sigma, ws, st);
+        case 4: return run_l<4>(p, rank, sketch, power_iters, omega, B, A, sigma, ws, st);
+        case 8: return run_l<8>(p, rank, sketch, power_iters, omega, B, A, sigma, ws, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace hqq
