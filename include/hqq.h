@@ -46,7 +46,9 @@ typedef enum hqq_status {
     HQQ_ERR_ALIGN = 5,       /* W / W_out / X not 16-byte aligned; packed not
                                 4-byte (8-byte at 8 bits); zero_f32 or err_out
                                 not 4-byte; scale/zero not 2-byte                */
-    HQQ_ERR_CUDA = 6         /* the kernel launch failed                         */
+    HQQ_ERR_CUDA = 6,        /* the kernel launch failed                         */
+    HQQ_ERR_SCRATCH = 7      /* hqq_lowrank_noalloc: the problem's workspace is
+                                larger than its fixed scratch array              */
 } hqq_status;
 
 /* Solver defaults of the method's section 4.1. */
@@ -304,6 +306,35 @@ int hqq_lowrank(const void* W, const void* packed, const void* scale, const void
                 int64_t rows, int64_t cols, int nbits, int group, int rank, int sketch,
                 int power_iters, const float* omega, float* B, float* A, float* sigma,
                 void* workspace, int64_t workspace_bytes, void* stream);
+
+/*
+ * hqq_lowrank_noalloc -- hqq_lowrank for callers that cannot allocate device
+ * memory: code that runs where cudaMalloc is not available or not allowed
+ * (a host whose allocator is owned by another framework, a plugin loaded into
+ * a process that forbids extra allocations after start-up, a real-time loop
+ * that must not allocate).  The paper has no counterpart of this entry point;
+ * it is a service of this library.
+ *
+ * Same arguments and results as hqq_lowrank without workspace and
+ * workspace_bytes: the workspace is a fixed scratch array inside the library
+ * (hqq_lowrank_noalloc_max_bytes() bytes, 16 MiB, present on every GPU that
+ * loads the library until the process exits).  A matrix whose
+ * hqq_lowrank_workspace_bytes() exceeds it returns HQQ_ERR_SCRATCH (at a
+ * 32-column sketch every Llama-2-70B matrix fits).  No call allocates device
+ * or host memory.
+ * The first call on each device looks up the array's device address with that
+ * device current and keeps it; make that first call before any stream
+ * capture.  All calls share the one array: calls whose work overlaps on the
+ * GPU (other streams, other host threads) race and give wrong results, so the
+ * caller orders them.  Nothing in the array needs to start at zero.
+ */
+int hqq_lowrank_noalloc(const void* W, const void* packed, const void* scale, const void* zero,
+                        int64_t rows, int64_t cols, int nbits, int group, int rank, int sketch,
+                        int power_iters, const float* omega, float* B, float* A, float* sigma,
+                        void* stream);
+
+/* Bytes of the fixed scratch array of hqq_lowrank_noalloc. */
+int64_t hqq_lowrank_noalloc_max_bytes(void);
 
 #ifdef __cplusplus
 }

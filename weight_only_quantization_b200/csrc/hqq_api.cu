@@ -26,6 +26,8 @@ cudaError_t launch_linear(const LinearParams& prm, const void* X, int nbits, cud
 cudaError_t launch_decode(const LinearParams& prm, const void* X, int nbits, int64_t packed_bytes,
                           cudaStream_t stream);
 int64_t lowrank_workspace_bytes(int64_t N, int64_t K, int sketch);
+int64_t lowrank_scratch_bytes();
+cudaError_t lowrank_scratch(void** ptr);
 cudaError_t launch_lowrank(const void* W, const uint8_t* packed, const __half* scale,
                            const __half* zero, int64_t N, int64_t K, int nbits, int log2_group,
                            int rank, int sketch, int power_iters, const float* omega, float* B,
@@ -132,6 +134,7 @@ extern "C" const char* hqq_status_string(int status) {
         case HQQ_ERR_PARAM: return "HQQ_ERR_PARAM: need 0<p<=1, beta>0, kappa>0 (finite), 0<=iters<=255";
         case HQQ_ERR_ALIGN: return "HQQ_ERR_ALIGN: W/W_out/X/meta x/meta out need 16-byte, meta codes and 8-bit packed 8-byte, packed/zero_f32 4-byte, scale/zero 2-byte alignment";
         case HQQ_ERR_CUDA: return "HQQ_ERR_CUDA: kernel launch failed (see cudaGetLastError)";
+        case HQQ_ERR_SCRATCH: return "HQQ_ERR_SCRATCH: the problem needs more scratch than the fixed array of hqq_lowrank_noalloc holds (hqq_lowrank_noalloc_max_bytes)";
         default: return "HQQ: unknown status";
     }
 }
@@ -414,4 +417,27 @@ extern "C" int hqq_lowrank(const void* W, const void* packed, const void* scale,
         static_cast<const __half*>(zero), rows, cols, nbits, log2_of_group(group), rank, sketch,
         power_iters, omega, B, A, sg, workspace, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
+extern "C" int64_t hqq_lowrank_noalloc_max_bytes(void) { return lowrank_scratch_bytes(); }
+
+extern "C" int hqq_lowrank_noalloc(const void* W, const void* packed, const void* scale,
+                                   const void* zero, int64_t rows, int64_t cols, int nbits,
+                                   int group, int rank, int sketch, int power_iters,
+                                   const float* omega, float* B, float* A, float* sigma,
+                                   void* stream) {
+    // the argument checks of hqq_lowrank that come before its workspace, so
+    // that a bad call is reported as such before any device lookup
+    const int st = validate_common(rows, cols, nbits, group);
+    if (st != HQQ_OK) return st;
+    if (sketch != 16 && sketch != 32 && sketch != 64) return HQQ_ERR_UNSUPPORTED;
+    if (rank < 1 || rank > sketch || power_iters < 0 || power_iters > 16) return HQQ_ERR_PARAM;
+    if (rows < sketch || cols < sketch || cols >= ((int64_t)1 << 30)) return HQQ_ERR_SHAPE;
+    if (lowrank_workspace_bytes(rows, cols, sketch) > lowrank_scratch_bytes())
+        return HQQ_ERR_SCRATCH;
+    if (!W || !packed || !scale || !zero || !omega || !B || !A) return HQQ_ERR_NULL;
+    void* scratch = nullptr;
+    if (lowrank_scratch(&scratch) != cudaSuccess) return HQQ_ERR_CUDA;
+    return hqq_lowrank(W, packed, scale, zero, rows, cols, nbits, group, rank, sketch,
+                       power_iters, omega, B, A, sigma, scratch, lowrank_scratch_bytes(), stream);
 }

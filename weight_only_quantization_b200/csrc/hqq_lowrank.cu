@@ -19,6 +19,8 @@
 // The l x l eigenproblem is solved by cyclic Jacobi in fp64 (Golub and Van
 // Loan, "Matrix Computations", the symmetric Schur rotation), L/2 disjoint
 // rotations at a time in round-robin order.
+#include <mutex>
+
 #include "hqq_unpack.cuh"
 
 namespace hqq {
@@ -524,6 +526,37 @@ cudaError_t launch_lowrank(const void* W, const uint8_t* packed, const __half* s
         case 8: return run_l<8>(p, rank, sketch, power_iters, omega, B, A, sigma, ws, st);
         default: return cudaErrorInvalidValue;
     }
+}
+
+// Fixed device scratch for callers that cannot allocate device memory (see
+// hqq_lowrank_noalloc in hqq.h): 16 MiB in every GPU's copy of this module,
+// held until the process exits.  Nothing in it needs to start at zero (every
+// part is written before it is read), and every call shares it.
+constexpr int64_t kLowrankScratchBytes = (int64_t)16 << 20;
+static __device__ __align__(256) uint8_t g_lowrank_scratch[kLowrankScratchBytes];
+
+int64_t lowrank_scratch_bytes() { return kLowrankScratchBytes; }
+
+// The device address of this GPU's scratch array, looked up once per device
+// (with that device current) and cached; host code can only name the array's
+// host-side stand-in, which is not a device address.
+cudaError_t lowrank_scratch(void** ptr) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* cached[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cached[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_lowrank_scratch);
+        if (e != cudaSuccess) return e;
+        cached[dev] = p;
+    }
+    *ptr = cached[dev];
+    return cudaSuccess;
 }
 
 }  // namespace hqq
