@@ -508,6 +508,11 @@ def run_gpu(args):
     if not args.no_meta:
         line["meta8"] = run_meta8(args, views, hqq, dev, hbm_peak, pg)
 
+    # ---- low-rank residual of the quantization error (before the RTN pass,
+    # which overwrites the HQQ codes)
+    if not args.no_lowrank:
+        line["lowrank"] = run_lowrank(views, hqq, dev, alu_peak, pg)
+
     # ---- memory-side calibration: round-to-nearest quantize pass (HBM-bound;
     # runs after the sections above, which use the HQQ codes)
     line["rtn"] = run_rtn(views, hqq, dev, hbm_peak, qbytes, pg)
@@ -750,6 +755,43 @@ def run_linear(args, views, hqq, dev, hbm_peak, tensor_peak, pg):
     return out
 
 
+def run_lowrank(views, hqq, dev, fma_peak, pg):
+    """Times the low-rank residual B A of the quantization error W - W_hat
+    (rank 16 from a 32-column Gaussian sketch, 2 power iterations) on the first
+    seven matrices (one layer of the model-shaped sets).  The products with
+    Delta W, (2 * iters + 2) * rows * cols * sketch fp32 FMAs per matrix, are
+    reported against the fp32 FMA lane peak."""
+    import torch
+    sub = views[:7]
+    rank, sketch, iters = 16, 32, 2
+    wsb = max(hqq._lib.hqq_lowrank_workspace_bytes(q.rows, q.cols, sketch) for _, q, _ in sub)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20)
+    oms = [torch.randn(q.cols, sketch, generator=gen, device=dev) for _, q, _ in sub]
+
+    def one():
+        for (W, q, _), om in zip(sub, oms):
+            hqq.hqq_lowrank(W, q, rank, om, power_iters=iters, workspace=ws)
+    one()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    reps = 3
+    ev[0].record()
+    for _ in range(reps):
+        one()
+    ev[1].record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps], pg, dev)[0]
+    fmas = sum((2 * iters + 2) * q.rows * q.cols * sketch for _, q, _ in sub)
+    return {"what": "rank-16 residual of W - W_hat by randomized subspace iteration (32-column "
+                    "sketch, 2 power iterations), Delta W formed inside the fp32 products",
+            "matrices": len(sub), "ms_per_pass": ms,
+            "products_tfma_s": fmas / (ms / 1e3) / 1e12,
+            "fma_frac": fmas / (ms / 1e3) / 1e12 / fma_peak,
+            "fma_peak_t": fma_peak}
+
+
 def run_stream_pass(mats, hqq, dev, views):
     """Generate + quantize layer by layer through one reused weight buffer
     (outputs stay resident); CUDA-event wall time of the whole pass."""
@@ -864,6 +906,7 @@ def main():
     ap.add_argument("--no-stream", action="store_true", help="skip the streamed generate+quantize pass")
     ap.add_argument("--no-meta", action="store_true", help="skip the 8-bit meta-data timing")
     ap.add_argument("--no-linear", action="store_true", help="skip the linear-layer timing")
+    ap.add_argument("--no-lowrank", action="store_true", help="skip the low-rank residual timing")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every library call from Python each pass instead of replaying "
                          "CUDA graphs of the passes")

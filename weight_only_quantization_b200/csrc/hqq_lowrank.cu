@@ -38,15 +38,37 @@ struct LrParams {
     int log2_group;
 };
 
-// Delta W of the 8 weights at flat index f (f % 8 == 0) in fp32.
+// One unit (8 consecutive weights of a row, flat index f, f % 8 == 0) in
+// flight: its fp16 weights, raw code words and group constants, so that the
+// loads of the next tile overlap the current tile's FMAs.
+struct UnitLoad {
+    uint4 w;
+    UnitRaw r;
+    __half s, z;
+};
+
 template <int NBITS>
-__device__ __forceinline__ void unit_delta(const LrParams& p, int64_t f, float (&d)[8]) {
-    const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.W + f));
-    const UnitRaw ur = unit_fetch<NBITS, false>(p.packed, f >> 3);
-    const int64_t g = f >> p.log2_group;
-    const uint4 hv =
-        unit8_raw<NBITS>(ur, __half2float(__ldg(p.zero + g)), __half2float(__ldg(p.scale + g)));
-    const __half2* w2 = reinterpret_cast<const __half2*>(&wv);
+__device__ __forceinline__ UnitLoad unit_load(const LrParams& p, int64_t f, bool ok) {
+    UnitLoad u;
+    if (ok) {
+        u.w = __ldg(reinterpret_cast<const uint4*>(p.W + f));
+        u.r = unit_fetch<NBITS, false>(p.packed, f >> 3);
+        const int64_t g = f >> p.log2_group;
+        u.s = __ldg(p.scale + g);
+        u.z = __ldg(p.zero + g);
+    } else {                                   // W = W_hat = 0: Delta W = 0
+        u.w = make_uint4(0u, 0u, 0u, 0u);
+        u.r.w0 = u.r.w1 = u.r.shift = 0u;
+        u.s = u.z = __float2half(0.0f);
+    }
+    return u;
+}
+
+// Delta W = W - W_hat of the unit in fp32 (W_hat exactly as hqq_dequantize).
+template <int NBITS>
+__device__ __forceinline__ void unit_delta(const UnitLoad& u, float (&d)[8]) {
+    const uint4 hv = unit8_raw<NBITS>(u.r, __half2float(u.z), __half2float(u.s));
+    const __half2* w2 = reinterpret_cast<const __half2*>(&u.w);
     const __half2* h2 = reinterpret_cast<const __half2*>(&hv);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -56,100 +78,164 @@ __device__ __forceinline__ void unit_delta(const LrParams& p, int64_t f, float (
     }
 }
 
-// Y[N, L] = dW[N, K] M[K, L].  CTA: 32 rows x L; per 32-wide k-tile, threads
-// 0..127 form the dW tile (one unit each), 128..255 stage M; thread t then
-// owns row t/8 and L/8 consecutive columns.
+// Y[N, L] = dW[N, K] M[K, L] over the k-tiles of split blockIdx.y (out: Y, or
+// the split's partial block when gridDim.y > 1).  CTA: 64 rows x L, k-tiles
+// of 32; thread t forms one unit of the dW tile (row t/4, k 8(t%4)) and owns
+// RPT = L/16 consecutive rows x 4 columns of the result (two vector shared
+// loads per k for 4 RPT FMAs).  The next tile's loads are issued before the
+// current tile's FMAs.
 template <int NBITS, int L>
 __global__ void __launch_bounds__(kLrThreads)
 lr_right_kernel(const __grid_constant__ LrParams p, const float* __restrict__ M,
-                float* __restrict__ Y) {
-    constexpr int CPT = L / 8;
-    __shared__ float As[32][33];                          // [k][row]
-    __shared__ __align__(16) float Bs[32][L];             // [k][column]
+                float* __restrict__ out, int64_t tiles_per_split) {
+    constexpr int RPT = L / 16, CG = L / 4, MV = 32 * L / 4;       // float4s of an M tile
+    __shared__ __align__(16) float As[32][64 + 4];                 // [k][row]
+    __shared__ __align__(16) float Bs[32][L];                      // [k][column]
     const int t = threadIdx.x;
-    const int64_t n0 = (int64_t)blockIdx.x * 32;
-    const int row = t >> 3, c0 = (t & 7) * CPT;
-    float acc[CPT];
+    const int64_t n0 = (int64_t)blockIdx.x * 64;
+    const int64_t kt0 = (int64_t)blockIdx.y * tiles_per_split;
+    const int64_t ktiles = (p.K + 31) / 32;
+    const int64_t kt1 = kt0 + tiles_per_split < ktiles ? kt0 + tiles_per_split : ktiles;
+    const int ur = t >> 2, uk = 8 * (t & 3);                       // this thread's unit
+    const int tr = (t / CG) * RPT, tc = 4 * (t % CG);              // this thread's outputs
+    const bool row_ok = n0 + ur < p.N;
+    float acc[RPT][4];
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) acc[c] = 0.0f;
-    for (int64_t k0 = 0; k0 < p.K; k0 += 32) {
-        if (t < 128) {
-            const int r = t >> 2, u = t & 3;
-            const int64_t n = n0 + r, k = k0 + 8 * u;
-            float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (n < p.N && k < p.K) unit_delta<NBITS>(p, n * p.K + k, d);
+    for (int i = 0; i < RPT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+    auto load = [&](int64_t kt, UnitLoad& u, float4 (&mv)[(MV + kLrThreads - 1) / kLrThreads]) {
+        const int64_t k = kt * 32 + uk;
+        u = unit_load<NBITS>(p, (n0 + ur) * p.K + k, row_ok && k < p.K);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) As[8 * u + i][r] = d[i];
-        } else {
-            for (int idx = t - 128; idx < 32 * L / 4; idx += 128) {
-                const int kk = idx / (L / 4), c4 = idx % (L / 4);
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (k0 + kk < p.K) v = __ldg(reinterpret_cast<const float4*>(M + (k0 + kk) * L) + c4);
-                *reinterpret_cast<float4*>(&Bs[kk][4 * c4]) = v;
+        for (int v = 0; v < (MV + kLrThreads - 1) / kLrThreads; ++v) {
+            const int idx = t + v * kLrThreads;
+            const int kk = idx / CG, c4 = idx % CG;
+            mv[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (idx < MV && kt * 32 + kk < p.K)
+                mv[v] = __ldg(reinterpret_cast<const float4*>(M + (kt * 32 + kk) * L) + c4);
+        }
+    };
+    UnitLoad u;
+    float4 mv[(MV + kLrThreads - 1) / kLrThreads];
+    if (kt0 < kt1) load(kt0, u, mv);
+    for (int64_t kt = kt0; kt < kt1; ++kt) {
+        float d[8];
+        unit_delta<NBITS>(u, d);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) As[uk + i][ur] = d[i];
+#pragma unroll
+        for (int v = 0; v < (MV + kLrThreads - 1) / kLrThreads; ++v) {
+            const int idx = t + v * kLrThreads;
+            if (idx < MV) *reinterpret_cast<float4*>(&Bs[idx / CG][4 * (idx % CG)]) = mv[v];
+        }
+        __syncthreads();
+        if (kt + 1 < kt1) load(kt + 1, u, mv);
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {
+            const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tc]);
+            float a[RPT];
+            if constexpr (RPT == 4) {
+                const float4 a4 = *reinterpret_cast<const float4*>(&As[kk][tr]);
+                a[0] = a4.x; a[1] = a4.y; a[2] = a4.z; a[3] = a4.w;
+            } else if constexpr (RPT == 2) {
+                const float2 a2 = *reinterpret_cast<const float2*>(&As[kk][tr]);
+                a[0] = a2.x; a[1] = a2.y;
+            } else {
+                a[0] = As[kk][tr];
+            }
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                acc[i][0] = __fmaf_rn(a[i], b.x, acc[i][0]);
+                acc[i][1] = __fmaf_rn(a[i], b.y, acc[i][1]);
+                acc[i][2] = __fmaf_rn(a[i], b.z, acc[i][2]);
+                acc[i][3] = __fmaf_rn(a[i], b.w, acc[i][3]);
             }
         }
         __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < 32; ++kk) {
-            const float a = As[kk][row];
-#pragma unroll
-            for (int c = 0; c < CPT; ++c) acc[c] = __fmaf_rn(a, Bs[kk][c0 + c], acc[c]);
-        }
-        __syncthreads();
     }
-    if (n0 + row < p.N) {
+    float* o = out + (int64_t)blockIdx.y * p.N * L;
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) Y[(n0 + row) * L + c0 + c] = acc[c];
-    }
+    for (int i = 0; i < RPT; ++i)
+        if (n0 + tr + i < p.N)
+            *reinterpret_cast<float4*>(o + (n0 + tr + i) * L + tc) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
 }
 
-// Zp[split, K, L] = sum over the split's rows of dW[row, k] Y[row, :].  CTA:
-// 32 columns k x L, rows [blockIdx.y * rps, +rps) in 32-row tiles.
+// Z[K, L] = dW^T Y over the rows of split blockIdx.y (out: Z, or the split's
+// partial block).  CTA: 64 columns k x L, rows in tiles of 32; thread t forms
+// one unit (row t/8, k 8(t%8)) and owns RPT = L/16 consecutive k x 4 columns.
 template <int NBITS, int L>
 __global__ void __launch_bounds__(kLrThreads)
 lr_left_kernel(const __grid_constant__ LrParams p, const float* __restrict__ Y,
-               float* __restrict__ Zp, int64_t rps) {
-    constexpr int CPT = L / 8;
-    __shared__ float As[32][33];                          // [row][k]
-    __shared__ __align__(16) float Bs[32][L];             // [row][column]
+               float* __restrict__ out, int64_t rows_per_split) {
+    constexpr int RPT = L / 16, CG = L / 4, YV = 32 * L / 4;
+    __shared__ __align__(16) float As[32][64 + 4];                 // [row][k]
+    __shared__ __align__(16) float Bs[32][L];                      // [row][column]
     const int t = threadIdx.x;
-    const int64_t k0 = (int64_t)blockIdx.x * 32;
-    const int64_t rb = (int64_t)blockIdx.y * rps;
-    const int64_t re = rb + rps < p.N ? rb + rps : p.N;
-    const int kk = t >> 3, c0 = (t & 7) * CPT;
-    float acc[CPT];
+    const int64_t k0 = (int64_t)blockIdx.x * 64;
+    const int64_t rb = (int64_t)blockIdx.y * rows_per_split;
+    const int64_t re = rb + rows_per_split < p.N ? rb + rows_per_split : p.N;
+    const int ur = t >> 3, uk = 8 * (t & 7);
+    const int tk = (t / CG) * RPT, tc = 4 * (t % CG);
+    const bool col_ok = k0 + uk < p.K;
+    float acc[RPT][4];
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) acc[c] = 0.0f;
+    for (int i = 0; i < RPT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+    auto load = [&](int64_t r0, UnitLoad& u, float4 (&yv)[(YV + kLrThreads - 1) / kLrThreads]) {
+        const int64_t n = r0 + ur;
+        u = unit_load<NBITS>(p, n * p.K + k0 + uk, col_ok && n < re);
+#pragma unroll
+        for (int v = 0; v < (YV + kLrThreads - 1) / kLrThreads; ++v) {
+            const int idx = t + v * kLrThreads;
+            const int r = idx / CG, c4 = idx % CG;
+            yv[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (idx < YV && r0 + r < re)
+                yv[v] = __ldg(reinterpret_cast<const float4*>(Y + (r0 + r) * L) + c4);
+        }
+    };
+    UnitLoad u;
+    float4 yv[(YV + kLrThreads - 1) / kLrThreads];
+    if (rb < re) load(rb, u, yv);
     for (int64_t r0 = rb; r0 < re; r0 += 32) {
-        if (t < 128) {
-            const int r = t >> 2, u = t & 3;
-            const int64_t n = r0 + r, k = k0 + 8 * u;
-            float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (n < re && k < p.K) unit_delta<NBITS>(p, n * p.K + k, d);
+        float d[8];
+        unit_delta<NBITS>(u, d);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) As[r][8 * u + i] = d[i];
-        } else {
-            for (int idx = t - 128; idx < 32 * L / 4; idx += 128) {
-                const int r = idx / (L / 4), c4 = idx % (L / 4);
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (r0 + r < re) v = __ldg(reinterpret_cast<const float4*>(Y + (r0 + r) * L) + c4);
-                *reinterpret_cast<float4*>(&Bs[r][4 * c4]) = v;
+        for (int i = 0; i < 8; ++i) As[ur][uk + i] = d[i];
+#pragma unroll
+        for (int v = 0; v < (YV + kLrThreads - 1) / kLrThreads; ++v) {
+            const int idx = t + v * kLrThreads;
+            if (idx < YV) *reinterpret_cast<float4*>(&Bs[idx / CG][4 * (idx % CG)]) = yv[v];
+        }
+        __syncthreads();
+        if (r0 + 32 < re) load(r0 + 32, u, yv);
+#pragma unroll 8
+        for (int r = 0; r < 32; ++r) {
+            const float4 b = *reinterpret_cast<const float4*>(&Bs[r][tc]);
+            float a[RPT];
+            if constexpr (RPT == 4) {
+                const float4 a4 = *reinterpret_cast<const float4*>(&As[r][tk]);
+                a[0] = a4.x; a[1] = a4.y; a[2] = a4.z; a[3] = a4.w;
+            } else if constexpr (RPT == 2) {
+                const float2 a2 = *reinterpret_cast<const float2*>(&As[r][tk]);
+                a[0] = a2.x; a[1] = a2.y;
+            } else {
+                a[0] = As[r][tk];
+            }
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                acc[i][0] = __fmaf_rn(a[i], b.x, acc[i][0]);
+                acc[i][1] = __fmaf_rn(a[i], b.y, acc[i][1]);
+                acc[i][2] = __fmaf_rn(a[i], b.z, acc[i][2]);
+                acc[i][3] = __fmaf_rn(a[i], b.w, acc[i][3]);
             }
         }
         __syncthreads();
-#pragma unroll 8
-        for (int r = 0; r < 32; ++r) {
-            const float a = As[r][kk];
-#pragma unroll
-            for (int c = 0; c < CPT; ++c) acc[c] = __fmaf_rn(a, Bs[r][c0 + c], acc[c]);
-        }
-        __syncthreads();
     }
-    if (k0 + kk < p.K) {
-        float* z = Zp + ((int64_t)blockIdx.y * p.K + k0 + kk) * L + c0;
+    float* o = out + (int64_t)blockIdx.y * p.K * L;
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) z[c] = acc[c];
-    }
+    for (int i = 0; i < RPT; ++i)
+        if (k0 + tk + i < p.K)
+            *reinterpret_cast<float4*>(o + (k0 + tk + i) * L + tc) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
 }
 
 // Z[i] = sum_s Zp[s * n + i].
@@ -397,20 +483,30 @@ lr_jacobi_kernel(const double* __restrict__ GP, int nparts, int rank, float* __r
     if (t < rank) sigma[t] = (float)sg[t];
 }
 
-constexpr int64_t kGramRows = 1024;                // rows per Gram block
+constexpr int64_t kGramRows = 128;                 // rows per Gram block
 
 int64_t align256(int64_t b) { return (b + 255) & ~(int64_t)255; }
 
-int64_t left_splits(int64_t K) {
-    const int64_t tiles = (K + 31) / 32;
-    int64_t s = (512 + tiles - 1) / tiles;
+// Splits of a product's reduction dimension: enough CTAs for about two per SM
+// of a 148-SM part (a fixed rule, so that the workspace size does not depend
+// on the device).
+int64_t splits_for(int64_t tiles) {
+    int64_t s = (296 + tiles - 1) / tiles;
     return s < 1 ? 1 : s > 16 ? 16 : s;
 }
+int64_t right_splits(int64_t N) { return splits_for((N + 63) / 64); }
+int64_t left_splits(int64_t K) { return splits_for((K + 63) / 64); }
 
 struct LrWorkspace {
-    float *Y, *Z, *Zp, *R, *Mr, *Mi;
+    float *Y, *Z, *P, *R, *Mr, *Mi;            // P: split partials of either product
     double* GP;
 };
+
+int64_t partial_floats(int64_t N, int64_t K, int L) {
+    const int64_t sr = right_splits(N), sl = left_splits(K);
+    const int64_t a = sr > 1 ? sr * N * L : 0, b = sl > 1 ? sl * K * L : 0;
+    return a > b ? a : b;
+}
 
 LrWorkspace carve(void* ws, int64_t N, int64_t K, int L) {
     uint8_t* b = static_cast<uint8_t*>(ws);
@@ -419,8 +515,8 @@ LrWorkspace carve(void* ws, int64_t N, int64_t K, int L) {
     b += align256(N * L * 4);
     w.Z = reinterpret_cast<float*>(b);
     b += align256(K * L * 4);
-    w.Zp = reinterpret_cast<float*>(b);
-    b += align256(left_splits(K) * K * L * 4);
+    w.P = reinterpret_cast<float*>(b);
+    b += align256(partial_floats(N, K, L) * 4);
     w.GP = reinterpret_cast<double*>(b);
     const int64_t parts = ((N > K ? N : K) + kGramRows - 1) / kGramRows;
     b += align256(parts * (int64_t)L * L * 8);
@@ -443,15 +539,19 @@ cudaError_t run(const LrParams& p, int rank, int power_iters, const float* omega
         e = cudaFuncSetAttribute(lr_jacobi_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kJacobiSmem);
     if (e != cudaSuccess) return e;
-    const int64_t S = left_splits(p.K);
-    const int64_t rps = ((p.N + S - 1) / S + 31) / 32 * 32;
+    const int64_t SR = right_splits(p.N), SL = left_splits(p.K);
+    const int64_t ktiles = (p.K + 31) / 32;
+    const int64_t tps = (ktiles + SR - 1) / SR;                 // k-tiles per right split
+    const int64_t rps = ((p.N + SL - 1) / SL + 31) / 32 * 32;   // rows per left split
     auto right = [&](const float* M) {
-        lr_right_kernel<NBITS, L><<<(unsigned)((p.N + 31) / 32), kLrThreads, 0, st>>>(p, M, w.Y);
+        lr_right_kernel<NBITS, L><<<dim3((unsigned)((p.N + 63) / 64), (unsigned)SR), kLrThreads, 0,
+                                    st>>>(p, M, SR > 1 ? w.P : w.Y, tps);
+        if (SR > 1) lr_reduce_kernel<<<592, kLrThreads, 0, st>>>(w.P, (int)SR, p.N * L, w.Y);
     };
     auto left = [&]() {
-        lr_left_kernel<NBITS, L><<<dim3((unsigned)((p.K + 31) / 32), (unsigned)S), kLrThreads, 0, st>>>(
-            p, w.Y, w.Zp, rps);
-        lr_reduce_kernel<<<592, kLrThreads, 0, st>>>(w.Zp, (int)S, p.K * L, w.Z);
+        lr_left_kernel<NBITS, L><<<dim3((unsigned)((p.K + 63) / 64), (unsigned)SL), kLrThreads, 0,
+                                   st>>>(p, w.Y, SL > 1 ? w.P : w.Z, rps);
+        if (SL > 1) lr_reduce_kernel<<<592, kLrThreads, 0, st>>>(w.P, (int)SL, p.K * L, w.Z);
     };
     auto gram = [&](const float* X, int64_t n) {
         const int64_t parts = (n + kGramRows - 1) / kGramRows;
@@ -502,7 +602,7 @@ cudaError_t run_l(const LrParams& p, int rank, int sketch, int power_iters, cons
 int64_t lowrank_workspace_bytes(int64_t N, int64_t K, int sketch) {
     const int64_t L = sketch;
     const int64_t parts = ((N > K ? N : K) + kGramRows - 1) / kGramRows;
-    return align256(N * L * 4) + align256(K * L * 4) + align256(left_splits(K) * K * L * 4) +
+    return align256(N * L * 4) + align256(K * L * 4) + align256(partial_floats(N, K, sketch) * 4) +
            align256(parts * L * L * 8) + 3 * align256(L * L * 4) + 256;   // + sigma slot
 }
 
