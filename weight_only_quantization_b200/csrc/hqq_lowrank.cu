@@ -80,7 +80,9 @@ __device__ __forceinline__ void unit_delta(const UnitLoad& u, float (&d)[8]) {
 
 // Y[N, L] = dW[N, K] M[K, L] over the k-tiles of split blockIdx.y (out: Y, or
 // the split's partial block when gridDim.y > 1).  CTA: 64 rows x L, k-tiles
-// of 32; thread t forms one unit of the dW tile (row t/4, k 8(t%4)) and owns
+// of 32; the dW tile is stored k-major with its rows rotated by 8 (k / 8)
+// (conflict-free stores of the four units of a row); thread t forms one unit
+// of the dW tile (row t/4, k 8(t%4)) and owns
 // RPT = L/16 consecutive rows x 4 columns of the result (two vector shared
 // loads per k for 4 RPT FMAs).  The next tile's loads are issued before the
 // current tile's FMAs.
@@ -121,7 +123,7 @@ lr_right_kernel(const __grid_constant__ LrParams p, const float* __restrict__ M,
         float d[8];
         unit_delta<NBITS>(u, d);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) As[uk + i][ur] = d[i];
+        for (int i = 0; i < 8; ++i) As[uk + i][(ur + uk) & 63] = d[i];   // rows rotated by 8 (k / 8)
 #pragma unroll
         for (int v = 0; v < (MV + kLrThreads - 1) / kLrThreads; ++v) {
             const int idx = t + v * kLrThreads;
@@ -132,15 +134,16 @@ lr_right_kernel(const __grid_constant__ LrParams p, const float* __restrict__ M,
 #pragma unroll 8
         for (int kk = 0; kk < 32; ++kk) {
             const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tc]);
+            const int ar = (tr + (kk & ~7)) & 63;    // same rotation; RPT-groups stay whole
             float a[RPT];
             if constexpr (RPT == 4) {
-                const float4 a4 = *reinterpret_cast<const float4*>(&As[kk][tr]);
+                const float4 a4 = *reinterpret_cast<const float4*>(&As[kk][ar]);
                 a[0] = a4.x; a[1] = a4.y; a[2] = a4.z; a[3] = a4.w;
             } else if constexpr (RPT == 2) {
-                const float2 a2 = *reinterpret_cast<const float2*>(&As[kk][tr]);
+                const float2 a2 = *reinterpret_cast<const float2*>(&As[kk][ar]);
                 a[0] = a2.x; a[1] = a2.y;
             } else {
-                a[0] = As[kk][tr];
+                a[0] = As[kk][ar];
             }
 #pragma unroll
             for (int i = 0; i < RPT; ++i) {
@@ -198,8 +201,14 @@ lr_left_kernel(const __grid_constant__ LrParams p, const float* __restrict__ Y,
     for (int64_t r0 = rb; r0 < re; r0 += 32) {
         float d[8];
         unit_delta<NBITS>(u, d);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) As[ur][uk + i] = d[i];
+        {   // lanes 4..7 of each group of 8 write their upper half first: the 8
+            // lanes of a quarter-warp then cover all 32 banks in each store
+            const int h = (t & 4) ? 4 : 0;
+            *reinterpret_cast<float4*>(&As[ur][uk + h]) =
+                h ? make_float4(d[4], d[5], d[6], d[7]) : make_float4(d[0], d[1], d[2], d[3]);
+            *reinterpret_cast<float4*>(&As[ur][uk + 4 - h]) =
+                h ? make_float4(d[0], d[1], d[2], d[3]) : make_float4(d[4], d[5], d[6], d[7]);
+        }
 #pragma unroll
         for (int v = 0; v < (YV + kLrThreads - 1) / kLrThreads; ++v) {
             const int idx = t + v * kLrThreads;
