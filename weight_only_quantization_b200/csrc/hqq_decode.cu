@@ -52,7 +52,8 @@ __device__ __forceinline__ float2 field_pair(uint32_t x, int b) {
 
 // A run of S codes of one feature: load(packed, f, ok) with f the flat index of
 // its first code; pair(pp) = codes 2pp and 2pp + 1 as exact floats (pp a
-// compile-time constant after unrolling).  ok == false leaves every code 0.
+// compile-time constant after unrolling); dq(pp, z, s) = their fp16 weights
+// packed in one word.  ok == false leaves every code 0.
 template <int NBITS, int S, bool VEC>
 struct Run;
 
@@ -86,6 +87,7 @@ struct Run<3, S, VEC> {
         const int m = 2 * pp, sl = m % 10;
         return sl < 6 ? field_pair<3>(r[m / 10], 3 * sl) : field_pair<3>(r[m / 10] >> 12, 3 * sl - 12);
     }
+    __device__ __forceinline__ uint32_t dq(int pp, float z, float s) const { return dq2(pair(pp), z, s); }
 };
 
 template <int S, bool VEC>
@@ -118,6 +120,32 @@ struct Run<4, S, VEC> {
         const int m = 2 * pp, sl = m % 8;
         return sl < 4 ? field_pair<4>(w[m / 8], 4 * sl) : field_pair<4>(w[m / 8] >> 16, 4 * sl - 16);
     }
+    // Two codes per mask: nibbles i and i + 4 of a word sit 16 bits apart, so
+    // (x & 0x000F000F) | 0x64006400 is the half2 (1024 + c_i, 1024 + c_i+4);
+    // an exact fp16 subtraction (or, for the odd nibbles shifted by 4, an
+    // exact fp16 fma by 1/16 and -64) leaves the codes, and one mixed-precision
+    // add per code gives fl32(c - z) from the fp16 code and the fp32 -z, the
+    // same value as the f32 path; the product by s and the fp16 pack follow.
+    __device__ __forceinline__ uint32_t dq(int pp, float z, float s) const { return dq2(pair(pp), z, s); }
+    // (measured faster for one token only; chosen at launch)
+    __device__ __forceinline__ uint32_t dq_mx(int pp, float z, float s) const {
+        const int m = 2 * pp, sl = m % 8;
+        const uint32_t x = (sl & 2) ? (w[m / 8] >> 8) : w[m / 8];   // nibbles 2,3,6,7 shifted down
+        const uint32_t lo = (x & 0x000F000Fu) | 0x64006400u;          // codes i, i + 4 (i even)
+        const uint32_t hi = (x & 0x00F000F0u) | 0x64006400u;          // codes i + 1, i + 5, times 16
+        const __half2 e0 = __hsub2(*reinterpret_cast<const __half2*>(&lo), __float2half2_rn(1024.0f));
+        const __half2 e1 = __hfma2(*reinterpret_cast<const __half2*>(&hi), __float2half2_rn(0.0625f),
+                                   __float2half2_rn(-64.0f));
+        const bool up = sl >= 4;                                     // codes 4..7: high halves
+        const __half c0 = up ? __high2half(e0) : __low2half(e0);
+        const __half c1 = up ? __high2half(e1) : __low2half(e1);
+        float d0, d1;
+        asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d0) : "h"(__half_as_ushort(c0)), "f"(-z));
+        asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d1) : "h"(__half_as_ushort(c1)), "f"(-z));
+        const float2 v = __fmul2_rn(make_float2(d0, d1), make_float2(s, s));
+        const __half2 h = __floats2half2_rn(v.x, v.y);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
 };
 
 template <int S, bool VEC>
@@ -138,6 +166,7 @@ struct Run<2, S, VEC> {
         return sl < 10 ? field_pair<2>(w[m / 16], 2 * sl)
                        : field_pair<2>(w[m / 16] >> 12, 2 * sl - 12);
     }
+    __device__ __forceinline__ uint32_t dq(int pp, float z, float s) const { return dq2(pair(pp), z, s); }
 };
 
 // 1 bit: a row starts on a 16-code boundary, so the run loads as 16-bit halves.
@@ -158,6 +187,7 @@ struct Run<1, S, VEC> {
         const int m = 2 * pp;
         return field_pair<1>(h[m / 16], m % 16);
     }
+    __device__ __forceinline__ uint32_t dq(int pp, float z, float s) const { return dq2(pair(pp), z, s); }
 };
 
 // 8 bits: byte i becomes the mantissa of 2^23 by one byte permute.
@@ -191,6 +221,7 @@ struct Run<8, S, VEC> {
                                      __uint_as_float(__byte_perm(x, 0x4B000000u, (uint32_t)(b + 1) | 0x7440u)));
         return __fadd2_rn(f, make_float2(-8388608.0f, -8388608.0f));
     }
+    __device__ __forceinline__ uint32_t dq(int pp, float z, float s) const { return dq2(pair(pp), z, s); }
 };
 
 // Staging geometry of one chunk (4 runs = 4S codes) of one feature: its bytes
@@ -262,19 +293,23 @@ __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0
 // S/4 MMAs per 8-token block of one chunk: codes 4i..4i+3 of the lane's runs of
 // features r and r + 8 against X[m, k + 4i .. k + 4i + 3]; xo[c] = row offset
 // of token 8c + r in X (the last token for rows past M).
-template <int NBITS, int S, bool VEC, int NT>
+template <int NBITS, int S, bool VEC, int NT, bool MX>
 __device__ __forceinline__ void chunk_mma(float (&acc)[NT][4], const Run<NBITS, S, VEC>& a,
                                           const Run<NBITS, S, VEC>& b, __half2 sz0, __half2 sz1,
                                           const __half* __restrict__ X, const int64_t (&xo)[NT],
                                           int64_t k) {
     const float s0 = __low2float(sz0), z0 = __high2float(sz0);
     const float s1 = __low2float(sz1), z1 = __high2float(sz1);
+    auto dq = [&](const Run<NBITS, S, VEC>& run, int pp, float z, float s) {
+        if constexpr (MX) return run.dq_mx(pp, z, s);
+        else return run.dq(pp, z, s);
+    };
 #pragma unroll
     for (int i = 0; i < S / 4; i += 2) {
-        const uint32_t a0 = dq2(a.pair(2 * i), z0, s0), a1 = dq2(b.pair(2 * i), z1, s1);
-        const uint32_t a2 = dq2(a.pair(2 * i + 1), z0, s0), a3 = dq2(b.pair(2 * i + 1), z1, s1);
-        const uint32_t a4 = dq2(a.pair(2 * i + 2), z0, s0), a5 = dq2(b.pair(2 * i + 2), z1, s1);
-        const uint32_t a6 = dq2(a.pair(2 * i + 3), z0, s0), a7 = dq2(b.pair(2 * i + 3), z1, s1);
+        const uint32_t a0 = dq(a, 2 * i, z0, s0), a1 = dq(b, 2 * i, z1, s1);
+        const uint32_t a2 = dq(a, 2 * i + 1, z0, s0), a3 = dq(b, 2 * i + 1, z1, s1);
+        const uint32_t a4 = dq(a, 2 * i + 2, z0, s0), a5 = dq(b, 2 * i + 2, z1, s1);
+        const uint32_t a6 = dq(a, 2 * i + 3, z0, s0), a7 = dq(b, 2 * i + 3, z1, s1);
 #pragma unroll
         for (int c = 0; c < NT; ++c) {
             const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + xo[c] + k) + i / 2);
@@ -293,7 +328,7 @@ __device__ __forceinline__ void chunk_mma(float (&acc)[NT][4], const Run<NBITS, 
 // copies granules j, j+4, .. of features r and r + 8; past the buffer's end
 // the copy is zero-filled), so two chunks are in flight while one is decoded;
 // otherwise the lanes load their runs from global memory directly.
-template <int NBITS, int S, bool VEC, bool STAGED, int NT>
+template <int NBITS, int S, bool VEC, bool STAGED, int NT, bool MX>
 __global__ void __launch_bounds__(kDcThreads, NT == 1 ? 3 : 2)
 decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams p, int split,
               int64_t packed_bytes) {
@@ -403,7 +438,7 @@ decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams
                 b.read(s1 + l1.off, l1.o);
             }
             const int64_t q = 4 * ch + j;
-            chunk_mma(acc, a, b, sz0, sz1, X, xo, q < runs ? q * S : 0);
+            chunk_mma<NBITS, S, VEC, NT, MX>(acc, a, b, sz0, sz1, X, xo, q < runs ? q * S : 0);
             sz0 = nz0;
             sz1 = nz1;
         }
@@ -418,7 +453,8 @@ decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams
             Run<NBITS, S, VEC> a, b;
             a.load(p.packed, f0, v0);
             b.load(p.packed, f1, v1);
-            chunk_mma(acc, a, b, group_of(ch, g0, ok0), group_of(ch, g1, ok1), X, xo, k);
+            chunk_mma<NBITS, S, VEC, NT, MX>(acc, a, b, group_of(ch, g0, ok0), group_of(ch, g1, ok1),
+                                             X, xo, k);
         }
     }
 
@@ -475,10 +511,10 @@ decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams
     }
 }
 
-template <int NBITS, int S, bool VEC, bool STAGED, int NT>
+template <int NBITS, int S, bool VEC, bool STAGED, int NT, bool MX>
 cudaError_t launch_s(const LinearParams& p, const void* X, int64_t packed_bytes,
                      cudaStream_t stream) {
-    auto kern = decode_kernel<NBITS, S, VEC, STAGED, NT>;
+    auto kern = decode_kernel<NBITS, S, VEC, STAGED, NT, MX>;
     constexpr size_t smem = decode_smem<NBITS, S, STAGED, NT>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -525,25 +561,30 @@ cudaError_t launch_s(const LinearParams& p, const void* X, int64_t packed_bytes,
 }
 
 // S = min(group, 64) codes per run (32 at 8 bits), so a run never leaves its group.
-template <int NBITS, bool VEC, bool STAGED, int NT>
+template <int NBITS, bool VEC, bool STAGED, int NT, bool MX>
 cudaError_t launch_g(const LinearParams& p, const void* X, int64_t pb, cudaStream_t stream) {
     constexpr int SMAX = NBITS == 8 ? 32 : 64;
-    if (p.log2_group == 4) return launch_s<NBITS, 16, VEC, STAGED, NT>(p, X, pb, stream);
-    if (p.log2_group == 5 || SMAX == 32) return launch_s<NBITS, 32, VEC, STAGED, NT>(p, X, pb, stream);
-    return launch_s<NBITS, SMAX, VEC, STAGED, NT>(p, X, pb, stream);
+    if (p.log2_group == 4) return launch_s<NBITS, 16, VEC, STAGED, NT, MX>(p, X, pb, stream);
+    if (p.log2_group == 5 || SMAX == 32)
+        return launch_s<NBITS, 32, VEC, STAGED, NT, MX>(p, X, pb, stream);
+    return launch_s<NBITS, SMAX, VEC, STAGED, NT, MX>(p, X, pb, stream);
 }
 
-template <int NBITS, bool VEC, int NT>
+template <int NBITS, bool VEC, int NT, bool MX>
 cudaError_t launch_st(const LinearParams& p, const void* X, int64_t pb, cudaStream_t stream) {
     const bool staged = (reinterpret_cast<uintptr_t>(p.packed) & 15u) == 0 && p.K < ((int64_t)1 << 30);
-    return staged ? launch_g<NBITS, VEC, true, NT>(p, X, pb, stream)
-                  : launch_g<NBITS, VEC, false, NT>(p, X, pb, stream);
+    return staged ? launch_g<NBITS, VEC, true, NT, MX>(p, X, pb, stream)
+                  : launch_g<NBITS, VEC, false, NT, MX>(p, X, pb, stream);
 }
 
 template <int NBITS, bool VEC>
 cudaError_t launch_nt(const LinearParams& p, const void* X, int64_t pb, cudaStream_t stream) {
-    if (p.M <= 8) return launch_st<NBITS, VEC, 1>(p, X, pb, stream);
-    return launch_st<NBITS, VEC, 2>(p, X, pb, stream);
+    // 4 bits, one token: codes in pairs through half-precision magic numbers
+    // (measured on 8192 x 8192: 25.0 -> 22.4 us; slower from 2 tokens)
+    if constexpr (NBITS == 4)
+        if (p.M == 1) return launch_st<NBITS, VEC, 1, true>(p, X, pb, stream);
+    if (p.M <= 8) return launch_st<NBITS, VEC, 1, false>(p, X, pb, stream);
+    return launch_st<NBITS, VEC, 2, false>(p, X, pb, stream);
 }
 
 }  // namespace
