@@ -187,7 +187,10 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-constexpr int kPrefetch = 2;                          // k-tiles of codes in flight per thread (2 keeps two CTAs per SM; 3 and 4 measured slower for few tokens)
+// k-tiles of codes in flight per producer thread: 2 keeps two CTAs per SM for
+// small token tiles (3 and 4 measured slower there); from 256 tokens a CTA has
+// an SM to itself and takes a deeper ring.
+__host__ __device__ constexpr int prefetch_of(int bn) { return bn >= 256 ? 4 : 2; }
 
 // gridDim.z > 1: the CTAs of a (1, 1, gridDim.z) cluster split the k-tiles of
 // one output tile; each keeps its partial sums in its own tensor memory, the
@@ -292,6 +295,7 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
         }
     } else {
         // ---- producers of W_hat: quads of 4 units, a ring of kPrefetch k-tiles
+        constexpr int kPrefetch = prefetch_of(BN);
         // of codes in registers (indices fixed by unrolling)
         const int pw = warp - 2, j4 = lane & 1;
         const int r = pw * 16 + (lane >> 1);
