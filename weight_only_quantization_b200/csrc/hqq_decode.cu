@@ -1,5 +1,6 @@
-// hqq_decode.cu -- the weight-only linear layer for up to eight tokens (the
-// decode shape): Y[m, n] = sum_k X[m, k] * W_hat[n, k] with W_hat =
+// hqq_decode.cu -- the weight-only linear layer for few tokens (the decode
+// shape: up to 16 at 3 bits, 8 otherwise; decode_max_tokens in hqq_params.cuh):
+// Y[m, n] = sum_k X[m, k] * W_hat[n, k] with W_hat =
 // fp16((code - z) * s) (section 2's Q^-1 of "Half-Quadratic Quantization of
 // Large Machine Learning Models"), the same product as hqq_linear.cu.
 //
@@ -9,14 +10,15 @@
 // straight from registers: lane (r, j) = (lane / 4, lane % 4) decodes a run of
 // S consecutive codes (inside one quantization group) of features r and r + 8
 // and supplies four codes of each per MMA, in the k slots 2j, 2j+1, 2j+8, 2j+9.
-// The B operand holds X in the same k order (column m = token m; columns past
-// M repeat the last token and are not stored), so the fp32 accumulation runs
-// in the tensor core and each weight costs its decode (a mask, then four fp32
-// pair operations for exact fp16 W_hat) and nothing else.  The 4 lanes of a
-// feature cover 4 consecutive runs (a chunk); a CTA's 8 warps take interleaved
-// chunks of the same 16 features, a cluster of up to 8 CTAs splits the chunks
-// further when the matrix has few features, and the partial tiles meet in
-// shared memory and distributed shared memory.
+// The B operand holds X in the same k order (column m = token m of an 8-token
+// block; columns past M repeat the last token and are not stored), so the fp32
+// accumulation runs in the tensor core and each weight costs its decode (a
+// mask, then four fp32 pair operations for exact fp16 W_hat) and nothing else.
+// The 4 lanes of a feature cover 4 consecutive runs (a chunk); a CTA's 8 warps
+// take interleaved chunks of the same 16 features, staged through per-warp
+// cp.async rings; a cluster of up to 8 CTAs splits the chunks further when the
+// matrix has few features or long rows, and the partial tiles meet in shared
+// memory and distributed shared memory.
 #include <cooperative_groups.h>
 
 #include "hqq_unpack.cuh"
