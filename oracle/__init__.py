@@ -3,7 +3,10 @@
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  It wraps ``hqq_oracle.c`` (plain scalar
 fp32, see the header comment of that file for the method, its source sections
-and the readings taken) through ctypes.  It shares no code with the CUDA path.
+and the readings taken) through ctypes.  Three functions are plain numpy in
+fp64 instead: ``linear`` (the product with the dequantized weights),
+``quant_error`` (W - W_hat) and ``lowrank`` (the truncated SVD of the
+quantization error).  It shares no code with the CUDA path.
 """
 from __future__ import annotations
 
