@@ -2,11 +2,23 @@
 Y = X W_hat^T with W_hat the dequantized fp16 weights, against the oracle's
 fp64 product on the oracle's own quantization of the same weights.
 
-Tolerance (from the arithmetic): the kernel forms the products of fp16 values
-exactly and sums them in fp32 in an unspecified order, then rounds to fp16.
-With S = sum_k |x_k w_k| and g = K * 2^-23 (a generous bound on the relative
-accumulation error of K fp32 additions, tensor-core internal rounding
-included):  |Y_gpu - Y_exact| <= 2^-11 |Y_exact| + 2 g S + 2^-24.
+Tolerance (from the arithmetic of both kernels): every product of two fp16
+values is exact in fp32, and the kernels add them in fp32 along chains of
+bounded length -- the tensor-core kernel accumulates ceil(K/16) MMAs of 16
+products each in tensor memory, then adds at most 8 split-k partials; the
+few-token kernel accumulates each warp's 16-wide k steps, then the 8 warps'
+sums and at most 8 cluster ranks' sums.  No product passes through more than
+D = ceil(K/16) + 40 additions (16 products inside one MMA: at most 5 levels),
+so with u = 2^-23 (one unit of an fp32 add, truncating or rounding) and
+S = sum_k |x_k w_k| the fp32 result is within 1.001 D u S of the exact sum
+(first-order bound of any summation tree of depth D); one fp16 rounding adds
+2^-11 of the value and at most 2^-25 near zero:
+    |Y_gpu - Y_exact| <= 2^-11 |Y_exact| + 1.001 D 2^-23 S + 2^-24.
+At K = 8192 this is 6.6e-5 S, where one group of 64 weights with a wrong
+scale or code offset moves an output by about 8 |x| |w| -- some 20x the
+bound on the synthetic weights, so such a defect cannot hide in it.  On small
+integer data every partial sum is an integer below 2^24 and the result must
+equal the exact one rounded to fp16 (tested up to K = 28672).
 """
 import numpy as np
 import pytest
@@ -43,11 +55,17 @@ def _tokens(M, K, seed):
     return rng.standard_normal((M, K)).astype(np.float16)
 
 
+def _depth(K):
+    """Longest chain of fp32 additions any product passes through."""
+    return -(-K // 16) + 40
+
+
 def _check(Y_gpu, X, Wh, label):
     ref = oracle.linear(X, Wh)
     K = X.shape[1]
     y = Y_gpu.astype(np.float64)
-    tol = 2.0 ** -11 * np.abs(ref["y64"]) + 2 * K * 2.0 ** -23 * ref["absum"] + 2.0 ** -24
+    tol = 2.0 ** -11 * np.abs(ref["y64"]) + 1.001 * _depth(K) * 2.0 ** -23 * ref["absum"] \
+        + 2.0 ** -24
     err = np.abs(y - ref["y64"])
     bad = err > tol
     assert not bad.any(), (label, int(bad.sum()), float((err / tol).max()))
@@ -119,6 +137,49 @@ def test_linear_exact_on_integer_data(hqq, M):
     assert np.array_equal(Y.cpu().numpy(), ref["y"])
 
 
+def _integer_matrix(hqq, rows, cols, nbits, group, seed):
+    """A quantized matrix whose W_hat is exact on small numbers: random codes,
+    per-group scales in {1/2, 1, 2} and integer zero points in [0, L], packed
+    by the oracle.  W_hat = (c - z) s is a multiple of 1/2 with |W_hat| <= 2L,
+    so any wrong scale or zero of a group changes the exact product."""
+    L = (1 << nbits) - 1
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, L + 1, rows * cols).astype(np.uint8)
+    ng = rows * cols // group
+    scale = rng.choice(np.array([0.5, 1.0, 2.0], np.float16), ng)
+    zero = rng.integers(0, L + 1, ng).astype(np.float16)
+    q = hqq.QuantizedMatrix(torch.from_numpy(oracle.pack(codes, nbits)).cuda(),
+                            torch.from_numpy(scale.reshape(rows, cols // group)).cuda(),
+                            torch.from_numpy(zero.reshape(rows, cols // group)).cuda(),
+                            rows, cols, nbits, group)
+    Wh = oracle.dequantize(codes, scale, zero, group).reshape(rows, cols)
+    return q, Wh
+
+
+@pytest.mark.parametrize("rows,cols", [(200, 8192), (130, 28672)])
+@pytest.mark.parametrize("nbits", [3, 4])
+@pytest.mark.parametrize("M", [1, 8, 16, 17, 32, 256, 1030, 2048])
+def test_linear_exact_full_size_k(hqq, rows, cols, nbits, M):
+    """Bit-exact at the 70B shapes' input sizes (K = 8192 and 28672): with
+    |x| <= 4 and |W_hat| <= 30 in steps of 1/2, every partial sum of any order
+    is a multiple of 1/2 below 2^23 in magnitude, hence exact in fp32, so Y
+    must equal the exact product rounded once to fp16.  Rows off the 128-row
+    tile; token counts covering the few-token kernel (1-16 tokens, clusters
+    splitting k), the tensor-memory kernel's small tiles with split-k
+    clusters (17, 32), its 256-token tiles and its 512-token tiles (1030,
+    2048)."""
+    q, Wh = _integer_matrix(hqq, rows, cols, nbits, 64, seed=rows + nbits)
+    rng = np.random.default_rng(M + cols)
+    X = rng.integers(-4, 5, (M, cols)).astype(np.float16)
+    Y = hqq.hqq_linear(torch.from_numpy(X).cuda(), q)
+    torch.cuda.synchronize()
+    ref = oracle.linear(X, Wh)
+    assert np.abs(ref["absum"]).max() < 2.0 ** 23
+    got = Y.cpu().numpy()
+    bad = got.view(np.uint16) != ref["y"].view(np.uint16)
+    assert not bad.any(), (int(bad.sum()), np.argwhere(bad)[:5].tolist())
+
+
 @pytest.mark.parametrize("nbits,group", [(3, 64), (4, 64), (2, 16), (8, 32), (1, 128)])
 @pytest.mark.parametrize("M", [4, 8, 9, 15, 24, 32, 33])
 def test_linear_decode_token_blocks(hqq, nbits, group, M):
@@ -157,13 +218,15 @@ def test_linear_decode_packed_alignment(hqq, nbits, group, rows, cols, M):
     _check(Yu.cpu().numpy(), X.cpu().numpy(), Wh, f"unaligned {nbits}b M={M}")
 
 
+@pytest.mark.parametrize("shape,stream", [((28672, 8192), 4), ((8192, 28672), 6)])
 @pytest.mark.parametrize("M", [1, 16, 256, 2048])
-def test_linear_full_size_70b_gate_sampled(hqq, M):
-    """The 28672 x 8192 3-bit g64 gate matrix quantized on the GPU; sampled
-    output features checked against the oracle's own quantization of those
-    rows (whose codes, scales and zeros must equal the GPU's)."""
-    rows, cols, nbits, group = 28672, 8192, 3, 64
-    W = synth.student_t_device((rows, cols), seed=5, stream=4)
+def test_linear_full_size_70b_gate_sampled(hqq, M, shape, stream):
+    """The 28672 x 8192 gate and 8192 x 28672 down matrices (3-bit g64)
+    quantized on the GPU; sampled output features checked against the
+    oracle's own quantization of those rows (whose codes, scales and zeros
+    must equal the GPU's)."""
+    (rows, cols), nbits, group = shape, 3, 64
+    W = synth.student_t_device((rows, cols), seed=5, stream=stream)
     q = hqq.hqq_quantize(W, nbits=nbits, group=group)
     X = _tokens(M, cols, seed=77)
     Y = hqq.hqq_linear(torch.from_numpy(X).cuda(), q)
@@ -180,7 +243,7 @@ def test_linear_full_size_70b_gate_sampled(hqq, M):
     codes_all = oracle.unpack(q.packed.cpu().numpy(), rows * cols, nbits).reshape(rows, cols)
     assert np.array_equal(codes_all[sample].reshape(-1), r["codes"])
     Wh = oracle.dequantize(r["codes"], r["scale"], r["zero"], group).reshape(len(sample), cols)
-    _check(Y.cpu().numpy()[:, sample], X, Wh, f"70b gate M={M}")
+    _check(Y.cpu().numpy()[:, sample], X, Wh, f"70b {rows}x{cols} M={M}")
 
 
 def test_linear_bad_arguments(hqq):
