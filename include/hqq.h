@@ -322,9 +322,11 @@ int hqq_lowrank(const void* W, const void* packed, const void* scale, const void
  * hqq_lowrank_workspace_bytes() exceeds it returns HQQ_ERR_SCRATCH (at a
  * 32-column sketch every Llama-2-70B matrix fits).  No call allocates device
  * or host memory.
- * The first call on each device looks up the array's device address with that
- * device current and keeps it; make that first call before any stream
- * capture.  All calls share the one array: calls whose work overlaps on the
+ * The first call in each CUDA context looks up the array's device address
+ * (with that context current) and keeps it for that context; a call made
+ * under another context -- a second context on the device, or the new one
+ * after cudaDeviceReset -- looks it up again.  Make the first call in a
+ * context before any stream capture.  All calls share the one array: calls whose work overlaps on the
  * GPU (other streams, other host threads) race and give wrong results, so the
  * caller orders them.  Nothing in the array needs to start at zero.
  */

@@ -19,7 +19,9 @@
 // The l x l eigenproblem is solved by cyclic Jacobi in fp64 (Golub and Van
 // Loan, "Matrix Computations", the symmetric Schur rotation), L/2 disjoint
 // rotations at a time in round-robin order.
+#include <cuda.h>
 #include <mutex>
+#include <utility>
 
 #include "hqq_unpack.cuh"
 
@@ -646,25 +648,62 @@ static __device__ __align__(256) uint8_t g_lowrank_scratch[kLowrankScratchBytes]
 
 int64_t lowrank_scratch_bytes() { return kLowrankScratchBytes; }
 
-// The device address of this GPU's scratch array, looked up once per device
-// (with that device current) and cached; host code can only name the array's
-// host-side stand-in, which is not a device address.
+// Id of the calling thread's current CUDA context (the driver's cuCtxGetId:
+// unique for the life of the process, so a context created after a
+// cudaDeviceReset, or a second context on the same device, has a new one).
+// The two driver calls are looked up once through the runtime.
+static bool current_context_id(unsigned long long* id) {
+    using GetCurrentFn = CUresult (*)(CUcontext*);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+    static const auto fns = [] {
+        void* a = nullptr;
+        void* b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+            qa != cudaDriverEntryPointSuccess)
+            a = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+            qb != cudaDriverEntryPointSuccess)
+            b = nullptr;
+        cudaGetLastError();                    // a failed lookup leaves no error behind
+        return std::make_pair(reinterpret_cast<GetCurrentFn>(a), reinterpret_cast<GetIdFn>(b));
+    }();
+    if (!fns.first || !fns.second) return false;
+    CUcontext ctx = nullptr;
+    if (fns.first(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return fns.second(ctx, id) == CUDA_SUCCESS;
+}
+
+// The device address of the scratch array in the current context, looked up
+// (with that context current) on the first call and whenever the current
+// context differs from the one the cached address belongs to; host code can
+// only name the array's host-side stand-in, which is not a device address.
+// Without the driver's context id the address is looked up on every call.
 cudaError_t lowrank_scratch(void** ptr) {
     constexpr int kMaxDevices = 64;
+    struct Entry {
+        unsigned long long ctx;
+        void* addr;
+    };
     static std::mutex mu;
-    static void* cached[kMaxDevices] = {};
+    static Entry cached[kMaxDevices] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    unsigned long long ctx = 0;
+    const bool have_id = current_context_id(&ctx);
     std::lock_guard<std::mutex> lock(mu);
-    if (!cached[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_lowrank_scratch);
-        if (e != cudaSuccess) return e;
-        cached[dev] = p;
+    if (have_id && cached[dev].addr && cached[dev].ctx == ctx) {
+        *ptr = cached[dev].addr;
+        return cudaSuccess;
     }
-    *ptr = cached[dev];
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_lowrank_scratch);   // makes the runtime's context current
+    if (e != cudaSuccess) return e;
+    unsigned long long now = 0;
+    cached[dev] = current_context_id(&now) ? Entry{now, p} : Entry{0ull, nullptr};
+    *ptr = p;
     return cudaSuccess;
 }
 
