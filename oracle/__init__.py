@@ -48,6 +48,12 @@ def _load():
             lib.hqq_oracle_quantize.restype = I
             lib.hqq_oracle_trace_group.argtypes = [P, I, I, F, F, F, I, P, P, P, P, P, P, P, P, P]
             lib.hqq_oracle_trace_group.restype = I
+            lib.hqq_oracle_quantize_half.argtypes = [P, I64, I, I, F, F, F, I, I, P, P, P, P, P,
+                                                     P, P, P]
+            lib.hqq_oracle_quantize_half.restype = I
+            lib.hqq_oracle_trace_group_half.argtypes = [P, I, I, F, F, F, I, P, P, P, P, P, P,
+                                                        P, P, P]
+            lib.hqq_oracle_trace_group_half.restype = I
             lib.hqq_oracle_shrink.argtypes = [P, I64, F, F, P]
             lib.hqq_oracle_shrink.restype = None
             lib.hqq_oracle_z_update.argtypes = [P, P, P, I, F]
@@ -87,14 +93,22 @@ DEFAULTS = dict(p=0.7, beta=1.0, kappa=1.01, iters=20)
 
 
 def quantize(W: np.ndarray, nbits: int, group: int, p: float = 0.7, beta: float = 1.0,
-             kappa: float = 1.01, iters: int = 20, threads: int | None = None) -> dict:
+             kappa: float = 1.01, iters: int = 20, threads: int | None = None,
+             precision: str = "fp32") -> dict:
     """HQQ-quantize an fp16 array (any shape, flat size a multiple of ``group``;
     groups are contiguous runs of ``group`` elements of the flat row-major order).
 
+    ``precision`` "fp32": the single-precision solver; "fp16": the half-precision
+    solver (groups outside its fp16 bounds solved in single precision; ``half``
+    in the result marks the groups solved in fp16).
+
     Returns codes (uint8 per weight, flat), packed bytes, fp16 scale/zero per
-    group, the fp32 zero and scale, the accepted minimum of the error sum
-    (+inf when iters = 0) and the accepted-iteration count per group.
+    group, the fp32 zero and scale, the accepted minimum of the error (the
+    binary32 sum; the fp16 mean for groups solved in half precision; +inf when
+    iters = 0) and the accepted-iteration count per group.
     """
+    if precision not in ("fp32", "fp16"):
+        raise ValueError("precision must be 'fp32' or 'fp16'")
     lib = _load()
     W = np.ascontiguousarray(W, dtype=np.float16).reshape(-1)
     n = W.size
@@ -110,39 +124,52 @@ def quantize(W: np.ndarray, nbits: int, group: int, p: float = 0.7, beta: float 
     err = np.empty(ng, np.float32)
     if threads is None:
         threads = os.cpu_count() or 1
-    st = lib.hqq_oracle_quantize(_ptr(W.view(np.uint16)), ng, group, nbits, p, beta, kappa,
-                                 iters, threads, _ptr(codes), _ptr(scale), _ptr(zero),
-                                 _ptr(zf), _ptr(sf), _ptr(err), _ptr(it))
+    half = np.zeros(ng, np.uint8)
+    if precision == "fp32":
+        st = lib.hqq_oracle_quantize(_ptr(W.view(np.uint16)), ng, group, nbits, p, beta, kappa,
+                                     iters, threads, _ptr(codes), _ptr(scale), _ptr(zero),
+                                     _ptr(zf), _ptr(sf), _ptr(err), _ptr(it))
+    else:
+        st = lib.hqq_oracle_quantize_half(_ptr(W.view(np.uint16)), ng, group, nbits, p, beta,
+                                          kappa, iters, threads, _ptr(codes), _ptr(scale),
+                                          _ptr(zero), _ptr(zf), _ptr(sf), _ptr(err), _ptr(it),
+                                          _ptr(half))
     if st:
         raise ValueError(f"oracle rejected the arguments (status {st})")
     return dict(codes=codes, packed=pack(codes, nbits), scale=scale.view(np.float16),
-                zero=zero.view(np.float16), zero_f32=zf, scale_f32=sf, err=err, iters=it)
+                zero=zero.view(np.float16), zero_f32=zf, scale_f32=sf, err=err, iters=it,
+                half=half.astype(bool))
 
 
 def trace_group(w, nbits: int, p: float = 0.7, beta: float = 1.0, kappa: float = 1.01,
-                iters: int = 20) -> dict:
-    """Solve one fp32 group and return its whole per-iteration record."""
+                iters: int = 20, precision: str = "fp32") -> dict:
+    """Solve one group (fp32 values; for "fp16" they must be fp16 values) and
+    return its whole per-iteration record; ``half`` tells whether the
+    half-precision solver took the group."""
+    if precision not in ("fp32", "fp16"):
+        raise ValueError("precision must be 'fp32' or 'fp16'")
     lib = _load()
     w = np.ascontiguousarray(w, dtype=np.float32)
     G = w.size
     T = max(iters, 1)
     codes = np.empty(G, np.uint8)
     out6 = np.empty(6, np.float32)
-    counts = np.empty(2, np.int32)
+    counts = np.zeros(3, np.int32)
     z = np.full(T, np.nan, np.float32)
     e = np.full(T, np.nan, np.float32)
     bh = np.full(T, np.nan, np.float32)
     q = np.full((T, G), np.nan, np.float32)
     d = np.full((T, G), np.nan, np.float32)
     we = np.full((T, G), np.nan, np.float32)
-    st = lib.hqq_oracle_trace_group(_ptr(w), G, nbits, p, beta, kappa, iters, _ptr(codes),
-                                    _ptr(out6), _ptr(counts), _ptr(z), _ptr(e), _ptr(bh),
-                                    _ptr(q), _ptr(d), _ptr(we))
+    fn = lib.hqq_oracle_trace_group if precision == "fp32" else lib.hqq_oracle_trace_group_half
+    st = fn(_ptr(w), G, nbits, p, beta, kappa, iters, _ptr(codes), _ptr(out6), _ptr(counts),
+            _ptr(z), _ptr(e), _ptr(bh), _ptr(q), _ptr(d), _ptr(we))
     if st:
         raise ValueError(f"oracle rejected the arguments (status {st})")
     ne = int(counts[1])
     return dict(codes=codes, s=out6[0], inv=out6[1], z0=out6[2], z_best=out6[3],
                 e_best=out6[4], accepted=int(counts[0]), evaluations=ne,
+                half=bool(counts[2]),
                 z=z[:ne], e=e[:ne], beta=bh[:ne], q=q[:ne], d=d[:ne], we=we[:ne])
 
 

@@ -222,6 +222,122 @@ static void solve_group(const float *w, const solver_cfg *cfg, uint8_t *codes,
 }
 
 /* ------------------------------------------------------------------------- */
+/* The same solver in half precision                                         */
+/* ------------------------------------------------------------------------- */
+/* Section 2.2 of the page holds 1/s because it "is more stable in half
+   precision", and section 3 runs the whole solve on the GPU in half precision.
+   The page fixes no rounding step; the readings taken:
+     - every element-wise step takes fp16 operands and rounds its result once
+       to fp16 (round to nearest even), with no fused multiply-add; computing
+       a +, -, * or / of fp16 values in binary32 and rounding to fp16 gives the
+       correctly rounded fp16 result (24 >= 2*11 + 2 bits), so h(a op b) below
+       is exact fp16 arithmetic;
+     - the group reductions (the error and the sp2 mean) accumulate in
+       binary32, in the PSUM order, and round the result once to fp16;
+     - the error is the group MEAN of |W - s(Wq - z)|^p (never overflows
+       fp16), compared in fp16;
+     - |x|^p and |x|^(p-1) are powp of the fp16 value, rounded to fp16;
+     - the hyper-parameters p, beta, kappa stay binary32 scalars: beta_t is
+       the binary32 schedule of the single-precision solver, and the shrink
+       divides its fp16 power by it and rounds to fp16;
+     - initialisation: r = h(max - min), s = h(r / L), 1/s = h(1 / s),
+       z = -h(min * (1/s)); a constant group has s = 1/s = 1, z = -min;
+     - fp16 cannot hold every intermediate of every group: a group whose
+       largest |W| exceeds 8192, whose s rounds to zero, or whose
+       max|W| * (1/s) exceeds 2^14 (binary32 product) is solved by the
+       single-precision solver above instead.  Inside those bounds the
+       starting point and every update with W_e = 0 stay in the fp16 range
+       (|W/s| <= 2^14, |z| <= 2^14 + L, |s (Wq - z)| <= 2 (max - min) +
+       max|W|); an update that an active shrink drives out of range gives an
+       infinite error at its evaluation and is never accepted. */
+static float h16(float x) { return half_bits_to_float(float_to_half_bits(x)); }
+
+/* 1 when the group is solved in half precision (see above), with its fp16
+   s, 1/s and starting z. */
+static int half_init(const float *w, int G, float L, float *s, float *inv, float *z) {
+    float mn = w[0], mx = w[0];
+    for (int i = 1; i < G; ++i) {
+        if (w[i] < mn) mn = w[i];
+        if (w[i] > mx) mx = w[i];
+    }
+    const float rng = h16(mx - mn);
+    if (rng == 0.0f) {
+        *s = 1.0f;
+        *inv = 1.0f;
+        *z = -mn;
+        return 1;
+    }
+    const float m = fmaxf(fabsf(mn), fabsf(mx));
+    *s = h16(rng / L);
+    *inv = h16(1.0f / *s);
+    if (!(m <= 8192.0f) || !(*s > 0.0f) || !(m * *inv <= 16384.0f)) return 0;
+    *z = -h16(mn * *inv);
+    return 1;
+}
+
+static void solve_group_half(const float *w, const solver_cfg *cfg, uint8_t *codes,
+                             group_result *res, group_trace *tr, int *half) {
+    const int G = cfg->G;
+    const float L = (float)((1 << cfg->nbits) - 1);
+    float s, inv, z;
+    if (!half_init(w, G, L, &s, &inv, &z)) {
+        *half = 0;
+        solve_group(w, cfg, codes, res, tr);
+        return;
+    }
+    *half = 1;
+    float u[HQQ_ORACLE_MAX_GROUP], q[HQQ_ORACLE_MAX_GROUP], d[HQQ_ORACLE_MAX_GROUP];
+    float pw[HQQ_ORACLE_MAX_GROUP], term[HQQ_ORACLE_MAX_GROUP];
+    for (int i = 0; i < G; ++i) u[i] = h16(w[i] * inv);          /* W / s, held as W * (1/s) */
+    const float z0 = z;
+    float z_best = z, e_best = INFINITY, beta_t = cfg->beta;
+    int accepted = 0, evaluations = 0;
+
+    for (int t = 0; t < cfg->iters; ++t) {
+        /* Wq = round(W/s + z);  residual W - s(Wq - z);  mean of |.|^p */
+        for (int i = 0; i < G; ++i) {
+            q[i] = clamp_code(h16(u[i] + z), L);
+            d[i] = h16(w[i] - h16(s * h16(q[i] - z)));
+            pw[i] = h16(powp(&cfg->tp, fabsf(d[i])));
+        }
+        const float e = h16(psum(pw, G) * (1.0f / (float)G));
+        ++evaluations;
+        if (tr) {
+            tr->z[t] = z;
+            tr->e[t] = e;
+            tr->beta[t] = beta_t;
+            memcpy(tr->q + (size_t)t * G, q, sizeof(float) * G);
+            memcpy(tr->d + (size_t)t * G, d, sizeof(float) * G);
+        }
+        if (!(e < e_best)) break;           /* error stopped falling */
+        e_best = e;
+        z_best = z;
+        ++accepted;
+
+        /* sp1: W_e = shrink_lp(residual, beta);  sp2: z = <Wq - (W - W_e)/s> */
+        for (int i = 0; i < G; ++i) {
+            const float a = fabsf(d[i]);
+            const float y = h16(a - h16(h16(powp(&cfg->tq, a)) / beta_t));
+            const float we = copysignf(fmaxf(y, 0.0f), d[i]);
+            if (tr) tr->we[(size_t)t * G + i] = we;
+            term[i] = h16(q[i] - h16(h16(w[i] - we) * inv));
+        }
+        z = h16(psum(term, G) * (1.0f / (float)G));
+        beta_t = beta_t * cfg->kappa;
+    }
+
+    for (int i = 0; i < G; ++i) codes[i] = (uint8_t)clamp_code(h16(u[i] + z_best), L);
+
+    res->s = s;
+    res->inv = inv;
+    res->z0 = z0;
+    res->z_best = z_best;
+    res->e_best = e_best;
+    res->accepted = accepted;
+    res->evaluations = evaluations;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Exported entry points (test infrastructure)                               */
 /* ------------------------------------------------------------------------- */
 static int check_cfg(int nbits, int G, float p, float beta, float kappa, int iters) {
@@ -252,6 +368,8 @@ typedef struct {
     uint16_t *scale, *zero;
     float *zero_f32, *scale_f32, *err;
     uint8_t *iters_out;
+    int half;            /* 1: the half-precision solver                 */
+    uint8_t *half_out;   /* per group: 1 when it was solved in fp16      */
 } work_range;
 
 static void *run_range(void *arg) {
@@ -262,7 +380,12 @@ static void *run_range(void *arg) {
         const uint16_t *src = wr->W + g * G;
         for (int i = 0; i < G; ++i) w[i] = half_bits_to_float(src[i]);
         group_result r;
-        solve_group(w, wr->cfg, wr->codes + g * G, &r, NULL);
+        int h = 0;
+        if (wr->half)
+            solve_group_half(w, wr->cfg, wr->codes + g * G, &r, NULL, &h);
+        else
+            solve_group(w, wr->cfg, wr->codes + g * G, &r, NULL);
+        if (wr->half_out) wr->half_out[g] = (uint8_t)h;
         wr->scale[g] = float_to_half_bits(r.s);
         wr->zero[g] = float_to_half_bits(r.z_best);
         if (wr->zero_f32) wr->zero_f32[g] = r.z_best;
@@ -277,10 +400,11 @@ static void *run_range(void *arg) {
    with in % G == 0 is exactly this flat layout).  codes: one byte per weight.
    scale/zero: fp16 bits per group.  zero_f32/scale_f32/err/iters_out nullable;
    err is the accepted minimum of the error sum (+inf when iters = 0). */
-int hqq_oracle_quantize(const uint16_t *W, int64_t n_groups, int G, int nbits,
-                        float p, float beta, float kappa, int iters, int nthreads,
-                        uint8_t *codes, uint16_t *scale, uint16_t *zero,
-                        float *zero_f32, float *scale_f32, float *err, uint8_t *iters_out) {
+static int quantize_groups(const uint16_t *W, int64_t n_groups, int G, int nbits,
+                           float p, float beta, float kappa, int iters, int nthreads,
+                           uint8_t *codes, uint16_t *scale, uint16_t *zero,
+                           float *zero_f32, float *scale_f32, float *err, uint8_t *iters_out,
+                           int half, uint8_t *half_out) {
     const int st = check_cfg(nbits, G, p, beta, kappa, iters);
     if (st) return st;
     if (n_groups <= 0) return 0;
@@ -303,6 +427,8 @@ int hqq_oracle_quantize(const uint16_t *W, int64_t n_groups, int G, int nbits,
         wr[k].scale_f32 = scale_f32;
         wr[k].err = err;
         wr[k].iters_out = iters_out;
+        wr[k].half = half;
+        wr[k].half_out = half_out;
     }
     if (nthreads == 1) {
         run_range(&wr[0]);
@@ -311,6 +437,26 @@ int hqq_oracle_quantize(const uint16_t *W, int64_t n_groups, int G, int nbits,
     for (int k = 0; k < nthreads; ++k) pthread_create(&th[k], NULL, run_range, &wr[k]);
     for (int k = 0; k < nthreads; ++k) pthread_join(th[k], NULL);
     return 0;
+}
+
+int hqq_oracle_quantize(const uint16_t *W, int64_t n_groups, int G, int nbits,
+                        float p, float beta, float kappa, int iters, int nthreads,
+                        uint8_t *codes, uint16_t *scale, uint16_t *zero,
+                        float *zero_f32, float *scale_f32, float *err, uint8_t *iters_out) {
+    return quantize_groups(W, n_groups, G, nbits, p, beta, kappa, iters, nthreads, codes,
+                           scale, zero, zero_f32, scale_f32, err, iters_out, 0, NULL);
+}
+
+/* The half-precision solver over the same layout; err is the accepted minimum
+   of the group's mean error in fp16 (of its binary32 error sum for a group
+   outside the fp16 bounds, which half_out marks 0). */
+int hqq_oracle_quantize_half(const uint16_t *W, int64_t n_groups, int G, int nbits,
+                             float p, float beta, float kappa, int iters, int nthreads,
+                             uint8_t *codes, uint16_t *scale, uint16_t *zero,
+                             float *zero_f32, float *scale_f32, float *err,
+                             uint8_t *iters_out, uint8_t *half_out) {
+    return quantize_groups(W, n_groups, G, nbits, p, beta, kappa, iters, nthreads, codes,
+                           scale, zero, zero_f32, scale_f32, err, iters_out, 1, half_out);
 }
 
 /* One group in fp32 with its full per-iteration record (for the pins). */
@@ -333,6 +479,32 @@ int hqq_oracle_trace_group(const float *w, int G, int nbits, float p, float beta
     out6[5] = 0.0f;
     counts2[0] = r.accepted;
     counts2[1] = r.evaluations;
+    return 0;
+}
+
+/* One group of the half-precision solver with its record; counts2[2] receives
+   1 when the group was solved in fp16. */
+int hqq_oracle_trace_group_half(const float *w, int G, int nbits, float p, float beta,
+                                float kappa, int iters, uint8_t *codes, float *out6,
+                                int *counts3, float *z, float *e, float *beta_hist,
+                                float *q, float *d, float *we) {
+    const int st = check_cfg(nbits, G, p, beta, kappa, iters);
+    if (st) return st;
+    solver_cfg cfg;
+    cfg_init(&cfg, nbits, G, p, beta, kappa, iters);
+    group_trace tr = {z, e, beta_hist, q, d, we};
+    group_result r;
+    int h = 0;
+    solve_group_half(w, &cfg, codes, &r, &tr, &h);
+    out6[0] = r.s;
+    out6[1] = r.inv;
+    out6[2] = r.z0;
+    out6[3] = r.z_best;
+    out6[4] = r.e_best;
+    out6[5] = 0.0f;
+    counts3[0] = r.accepted;
+    counts3[1] = r.evaluations;
+    counts3[2] = h;
     return 0;
 }
 
