@@ -123,6 +123,41 @@ int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nbits, int gr
                     float* zero_f32, float* err_out, uint8_t* iters_out, void* stream);
 
 /*
+ * hqq_quantize_half -- hqq_quantize_ex with the solver in half precision, the
+ * way the method runs it: section 2.2 holds 1/s because it "is more stable in
+ * half precision", and section 3 runs the whole solve on the GPU in half
+ * precision.  The page fixes no rounding step; this library takes:
+ *   - every element-wise step (W*(1/s), + z, Wq - z, s*(.), W - ., the shrink's
+ *     power, quotient and difference, the sp2 terms) rounded once to fp16,
+ *     round to nearest even, never fused;
+ *   - |x|^p and |x|^(p-1) as the binary32 table power rounded to fp16;
+ *   - the group reductions accumulated in binary32 (pairwise over contiguous
+ *     halves) and rounded once to fp16: the error is the group MEAN of |r|^p
+ *     (compared in fp16), z the group mean of the sp2 terms;
+ *   - p, beta, kappa and beta_t as in hqq_quantize (binary32 scalars);
+ *   - s = fp16(fp16(max - min)/L), 1/s = fp16(1/s), z = -fp16(min*(1/s))
+ *     (s = 1/s = 1, z = -min for a constant group).
+ * fp16 cannot hold every group's intermediates: a group whose largest |W|
+ * exceeds 8192, whose s rounds to zero, or whose max|W|*(1/s) (binary32
+ * product) exceeds 2^14 is solved in single precision exactly as
+ * hqq_quantize_ex solves it.  iters = 0 gives min-max round-to-nearest with
+ * these fp16 steps.
+ *   Arguments as for hqq_quantize_ex, except:
+ *   err_out   [out] float [rows, cols/group] or NULL: the accepted minimum of
+ *                   the group's error -- its fp16 mean for a group solved in
+ *                   half precision, the binary32 sum otherwise; +inf when
+ *                   iters = 0.
+ *   half_out  [out] uint8 [rows, cols/group] or NULL: 1 where the group was
+ *                   solved in half precision, 0 where in single precision.
+ * Errors as for hqq_quantize.
+ */
+int hqq_quantize_half(const void* W, int64_t rows, int64_t cols, int nbits, int group,
+                      float p, float beta, float kappa, int iters,
+                      void* packed, void* scale, void* zero,
+                      float* zero_f32, float* err_out, uint8_t* iters_out, uint8_t* half_out,
+                      void* stream);
+
+/*
  * hqq_dequantize -- Q^-1 of the method's section 2: W_hat = s (Wq - z), computed
  * as fp16( (code - z) * s ) in binary32 from the stored fp16 s and z.
  *

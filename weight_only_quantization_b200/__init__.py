@@ -12,7 +12,7 @@ import ctypes
 import os
 from dataclasses import dataclass
 
-__all__ = ["HQQError", "hqq_quantize", "hqq_quantize_ex", "hqq_dequantize",
+__all__ = ["HQQError", "hqq_quantize", "hqq_quantize_ex", "hqq_quantize_half", "hqq_dequantize",
            "hqq_packed_bytes", "hqq_status_string", "QuantizedMatrix", "LIB_PATH",
            "Meta8", "hqq_meta_groups", "hqq_meta_quantize", "hqq_meta_dequantize",
            "hqq_dequantize_meta", "hqq_linear", "hqq_linear_meta",
@@ -38,6 +38,9 @@ _lib.hqq_quantize.restype = _I
 _lib.hqq_quantize_ex.argtypes = [_P, _I64, _I64, _I, _I, _F, _F, _F, _I, _P, _P, _P, _P, _P, _P,
                                  _P]
 _lib.hqq_quantize_ex.restype = _I
+_lib.hqq_quantize_half.argtypes = [_P, _I64, _I64, _I, _I, _F, _F, _F, _I, _P, _P, _P, _P, _P, _P,
+                                   _P, _P]
+_lib.hqq_quantize_half.restype = _I
 _lib.hqq_dequantize.argtypes = [_P, _P, _P, _I64, _I64, _I, _I, _P, _P]
 _lib.hqq_dequantize.restype = _I
 _lib.hqq_meta_groups.argtypes = [_I64, _I64]
@@ -114,6 +117,7 @@ class QuantizedMatrix:
     zero_f32: "torch.Tensor | None" = None
     iters: "torch.Tensor | None" = None
     err: "torch.Tensor | None" = None
+    half: "torch.Tensor | None" = None      # uint8: group solved in half precision
 
 
 def _outputs(W, nbits, group, packed, scale, zero):
@@ -135,32 +139,49 @@ def _check_tensor(t, name):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
 
 
+def _precision(precision: str) -> bool:
+    if precision not in ("fp32", "fp16"):
+        raise ValueError("precision must be 'fp32' (single-precision solver) or 'fp16' "
+                         "(the half-precision solver)")
+    return precision == "fp16"
+
+
 def hqq_quantize(W, nbits: int = 4, group: int = 64, p: float = DEFAULT_P,
                  beta: float = DEFAULT_BETA, kappa: float = DEFAULT_KAPPA,
                  iters: int = DEFAULT_ITERS, packed=None, scale=None, zero=None,
-                 stream=None) -> QuantizedMatrix:
-    """Quantize a contiguous fp16 CUDA matrix [rows, cols] (see include/hqq.h)."""
+                 stream=None, precision: str = "fp32") -> QuantizedMatrix:
+    """Quantize a contiguous fp16 CUDA matrix [rows, cols] (see include/hqq.h);
+    ``precision="fp16"`` runs the half-precision solver (hqq_quantize_half)."""
     import torch
     if W.dtype != torch.float16 or W.dim() != 2:
         raise ValueError("W must be a 2-D float16 tensor")
+    half = _precision(precision)
     for t, n in ((W, "W"), (packed, "packed"), (scale, "scale"), (zero, "zero")):
         _check_tensor(t, n)
     packed, scale, zero = _outputs(W, nbits, group, packed, scale, zero)
     rows, cols = W.shape
-    _check(_lib.hqq_quantize(_ptr(W), rows, cols, nbits, group, p, beta, kappa, iters,
-                             _ptr(packed), _ptr(scale), _ptr(zero), _stream(stream)))
+    if half:
+        _check(_lib.hqq_quantize_half(_ptr(W), rows, cols, nbits, group, p, beta, kappa, iters,
+                                      _ptr(packed), _ptr(scale), _ptr(zero), None, None, None,
+                                      None, _stream(stream)))
+    else:
+        _check(_lib.hqq_quantize(_ptr(W), rows, cols, nbits, group, p, beta, kappa, iters,
+                                 _ptr(packed), _ptr(scale), _ptr(zero), _stream(stream)))
     return QuantizedMatrix(packed, scale, zero, rows, cols, nbits, group)
 
 
 def hqq_quantize_ex(W, nbits: int = 4, group: int = 64, p: float = DEFAULT_P,
                     beta: float = DEFAULT_BETA, kappa: float = DEFAULT_KAPPA,
                     iters: int = DEFAULT_ITERS, packed=None, scale=None, zero=None,
-                    zero_f32=None, iters_out=None, err_out=None, stream=None) -> QuantizedMatrix:
-    """hqq_quantize plus the fp32 zero, the solver's l_p error sum and the
-    accepted-iteration count of every group."""
+                    zero_f32=None, iters_out=None, err_out=None, stream=None,
+                    precision: str = "fp32", half_out=None) -> QuantizedMatrix:
+    """hqq_quantize plus the fp32 zero, the solver's l_p error and the
+    accepted-iteration count of every group (and, with ``precision="fp16"``,
+    which groups were solved in half precision)."""
     import torch
     if W.dtype != torch.float16 or W.dim() != 2:
         raise ValueError("W must be a 2-D float16 tensor")
+    half = _precision(precision)
     for t, n in ((W, "W"), (packed, "packed"), (scale, "scale"), (zero, "zero"),
                  (zero_f32, "zero_f32"), (iters_out, "iters_out"), (err_out, "err_out")):
         _check_tensor(t, n)
@@ -173,11 +194,21 @@ def hqq_quantize_ex(W, nbits: int = 4, group: int = 64, p: float = DEFAULT_P,
         iters_out = torch.empty(meta, dtype=torch.uint8, device=W.device)
     if err_out is None:
         err_out = torch.empty(meta, dtype=torch.float32, device=W.device)
-    _check(_lib.hqq_quantize_ex(_ptr(W), rows, cols, nbits, group, p, beta, kappa, iters,
-                                _ptr(packed), _ptr(scale), _ptr(zero), _ptr(zero_f32),
-                                _ptr(err_out), _ptr(iters_out), _stream(stream)))
+    if half:
+        _check_tensor(half_out, "half_out")
+        if half_out is None:
+            half_out = torch.empty(meta, dtype=torch.uint8, device=W.device)
+        _check(_lib.hqq_quantize_half(_ptr(W), rows, cols, nbits, group, p, beta, kappa, iters,
+                                      _ptr(packed), _ptr(scale), _ptr(zero), _ptr(zero_f32),
+                                      _ptr(err_out), _ptr(iters_out), _ptr(half_out),
+                                      _stream(stream)))
+    else:
+        half_out = None
+        _check(_lib.hqq_quantize_ex(_ptr(W), rows, cols, nbits, group, p, beta, kappa, iters,
+                                    _ptr(packed), _ptr(scale), _ptr(zero), _ptr(zero_f32),
+                                    _ptr(err_out), _ptr(iters_out), _stream(stream)))
     return QuantizedMatrix(packed, scale, zero, rows, cols, nbits, group, zero_f32, iters_out,
-                           err_out)
+                           err_out, half_out)
 
 
 def hqq_dequantize(q: QuantizedMatrix, out=None, stream=None):

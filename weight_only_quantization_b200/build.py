@@ -16,8 +16,8 @@ from concurrent.futures import ThreadPoolExecutor
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["hqq_api.cu", "hqq_quantize.cu", "hqq_dequantize.cu", "hqq_meta.cu", "hqq_linear.cu", "hqq_decode.cu", "hqq_rtn.cu", "hqq_lowrank.cu"]
-HEADERS = ["hqq_common.cuh", "hqq_params.cuh", "hqq_unpack.cuh"]
+SOURCES = ["hqq_api.cu", "hqq_quantize.cu", "hqq_quantize_half.cu", "hqq_dequantize.cu", "hqq_meta.cu", "hqq_linear.cu", "hqq_decode.cu", "hqq_rtn.cu", "hqq_lowrank.cu"]
+HEADERS = ["hqq_common.cuh", "hqq_params.cuh", "hqq_unpack.cuh", "hqq_quantize.cuh"]
 LIB = os.path.join(PKG, "libhqq.so")
 
 COMPILE_FLAGS = [

@@ -9,6 +9,8 @@
 
 namespace hqq {
 cudaError_t launch_quantize(const QuantParams& prm, int nbits, int group, cudaStream_t stream);
+cudaError_t launch_quantize_half(const QuantParams& prm, int nbits, int group,
+                                 cudaStream_t stream);
 struct RtnParams {
     const __half* W;
     uint8_t* packed;
@@ -139,10 +141,13 @@ extern "C" const char* hqq_status_string(int status) {
     }
 }
 
-extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nbits, int group,
-                               float p, float beta, float kappa, int iters, void* packed,
-                               void* scale, void* zero, float* zero_f32, float* err_out,
-                               uint8_t* iters_out, void* stream) {
+namespace {
+
+// Shared body of hqq_quantize_ex (binary32 solver) and hqq_quantize_half.
+int quantize_common(const void* W, int64_t rows, int64_t cols, int nbits, int group, float p,
+                    float beta, float kappa, int iters, void* packed, void* scale, void* zero,
+                    float* zero_f32, float* err_out, uint8_t* iters_out, bool half,
+                    uint8_t* half_out, void* stream) {
     int st = validate_common(rows, cols, nbits, group);
     if (st != HQQ_OK) return st;
     if (!(p > 0.0f && p <= 1.0f)) return HQQ_ERR_PARAM;
@@ -157,7 +162,7 @@ extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nb
         (err_out && !aligned(err_out, 4)))
         return HQQ_ERR_ALIGN;
 
-    if (iters == 0) {                  // min-max round-to-nearest: the streaming kernel
+    if (iters == 0 && !half) {         // min-max round-to-nearest: the streaming kernel
         RtnParams rp;
         rp.W = static_cast<const __half*>(W);
         rp.packed = static_cast<uint8_t*>(packed);
@@ -180,6 +185,7 @@ extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nb
     prm.zero_f32 = zero_f32;
     prm.err_out = err_out;
     prm.iters_out = iters_out;
+    prm.half_out = half_out;
     prm.n_groups = n / group;
     prm.n_elems = n;
     prm.iters = iters;
@@ -197,18 +203,44 @@ extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nb
     prm.tp = g_cache.tp;
     prm.tq = g_cache.tq;
 
-    // Shrink shortcut: |r| - |r|^(p-1)/beta > 0  <=>  |r| > beta^(-1/(2-p)).  Below
-    // the threshold lowered by a 1e-4 relative margin (far above the rounding
-    // error of the table power), W_e is exactly zero, so the kernel may skip it.
+    // Shrink shortcut: |r| - |r|^(p-1)/beta > 0  <=>  |r| > T = beta^(-1/(2-p)).
+    // Below T lowered by a 1e-4 relative margin (far above the rounding error
+    // of the binary32 table power), W_e is exactly zero, so the kernel may skip
+    // it.  The half-precision shrink rounds the power and its quotient by beta
+    // to fp16 (2^-11 each); below T (1 - 1e-2) the computed |r|^(p-1)/beta still
+    // exceeds |r| by at least (1 + (2-p) 1e-2)(1 - 2^-10) > 1, so its W_e is
+    // exactly zero too.
     float bt = beta;
     for (int t = 0; t < iters; ++t) {
         const double T = std::pow((double)bt, -1.0 / (2.0 - (double)p));
         prm.shrink_thr[t] = (float)(T * (1.0 - 1e-4));
+        prm.shrink_thr16[t] = (float)(T * (1.0 - 1e-2));
         bt = bt * kappa;
     }
 
-    const cudaError_t err = launch_quantize(prm, nbits, group, static_cast<cudaStream_t>(stream));
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const cudaError_t err = half ? launch_quantize_half(prm, nbits, group, cs)
+                                 : launch_quantize(prm, nbits, group, cs);
     return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, int nbits, int group,
+                               float p, float beta, float kappa, int iters, void* packed,
+                               void* scale, void* zero, float* zero_f32, float* err_out,
+                               uint8_t* iters_out, void* stream) {
+    return quantize_common(W, rows, cols, nbits, group, p, beta, kappa, iters, packed, scale,
+                           zero, zero_f32, err_out, iters_out, false, nullptr, stream);
+}
+
+extern "C" int hqq_quantize_half(const void* W, int64_t rows, int64_t cols, int nbits,
+                                 int group, float p, float beta, float kappa, int iters,
+                                 void* packed, void* scale, void* zero, float* zero_f32,
+                                 float* err_out, uint8_t* iters_out, uint8_t* half_out,
+                                 void* stream) {
+    return quantize_common(W, rows, cols, nbits, group, p, beta, kappa, iters, packed, scale,
+                           zero, zero_f32, err_out, iters_out, true, half_out, stream);
 }
 
 extern "C" int hqq_quantize(const void* W, int64_t rows, int64_t cols, int nbits, int group,

@@ -40,6 +40,7 @@ struct QuantParams {
     float* zero_f32;       // nullable
     float* err_out;        // nullable
     uint8_t* iters_out;    // nullable
+    uint8_t* half_out;     // nullable: 1 where a group was solved in half precision
     int64_t n_groups;
     int64_t n_elems;
     int iters;
@@ -48,6 +49,7 @@ struct QuantParams {
     PowTable tp;           // exponent p     (l_p error)
     PowTable tq;           // exponent p - 1 (generalised shrink)
     float shrink_thr[kMaxIters];  // |r| <= thr[t] guarantees W_e == 0 at step t
+    float shrink_thr16[kMaxIters];  // the same for the half-precision shrink
 };
 
 // Shared-memory image of one PowTable (separate arrays, so that the two values

@@ -1,728 +1,12 @@
-// hqq_quantize.cu -- fused HQQ solver + code packing kernel (sm_100a).
-//
-// "Half-Quadratic Quantization of Large Machine Learning Models", section 2
-// (Q, Q^-1, l_p error, sp1 shrink, sp2 mean, beta <- kappa beta, 1/s held) and
-// section 4.1 (solver parameters, early exit when the error stops improving).
-//
-// Work decomposition (persistent warps):
-//  * A group of G weights is held by a sub-warp of K = G/(8 NB) lanes, each lane
-//    owning NB blocks of 8 consecutive weights.  Within a block the weights sit
-//    in f32x2 register pairs (x_k, x_k+4), k = 0..3, for the packed element-wise
-//    arithmetic; the pairwise sum over contiguous halves then reads the halves
-//    with scalar adds, and lane sums are combined by xor-shuffles 1, 2, .., K/2
-//    (same pairwise order).
-//  * Each warp owns chunks of 2560 consecutive weights (five groups of any size
-//    fill whole 3-bit words), staged once into the warp's shared memory.
-//  * Phase A: every group of the chunk is initialised and runs its first two
-//    error evaluations in lock-step -- every group needs at least two, so no
-//    lane idles.  Groups that stop are finalised; the others are queued with
-//    their state in shared memory.
-//  * Phase B: each sub-warp pulls queued groups, iterates until its group stops,
-//    finalises it and pulls the next, so the early-stop divergence costs almost
-//    nothing.  No block-wide barrier is ever taken after start-up.
-//  * Two exact shortcuts, both tested per group and per step: when
-//    fma(min, 1/s, z) >= -1/2 and fma(max, 1/s, z) < L + 1/2 no code can leave
-//    [0, L] (fma is monotone in the weight), so the clamp is skipped; when a
-//    bound on |W - Q^-1(Q(W))| lies below the shrink threshold, W_e is exactly
-//    zero, so sp1 reduces to W - W_e = W.
-#include <type_traits>
-
-#include "hqq_common.cuh"
+// hqq_quantize.cu -- the single-precision instantiations of the fused HQQ
+// solver + packing kernel (hqq_quantize.cuh): every step of section 2 of "Half-
+// Quadratic Quantization of Large Machine Learning Models" in binary32.
+#include "hqq_quantize.cuh"
 
 namespace hqq {
 
-constexpr int kQWarps = 8;                 // warps per CTA (share the 32 KiB table)
-constexpr int kChunk = 2560;               // weights per warp chunk
-constexpr unsigned kFull = 0xFFFFFFFFu;
-
-template <int NBITS, int G, int NB>
-struct QCfg {
-    static constexpr int EPL = 8 * NB;           // weights per lane
-    static constexpr int K = G / EPL;            // lanes per group
-    static constexpr int GPW = 32 / K;           // groups per warp round
-    static constexpr int ROUND = 32 * EPL;       // weights per warp round
-    static constexpr int ROUNDS = kChunk / ROUND;
-    static constexpr int CG = kChunk / G;        // groups per chunk
-    static constexpr int L = (1 << NBITS) - 1;
-    static constexpr int W_BYTES = kChunk * 2;
-    static constexpr int ST_BYTES = CG * 16;     // (z, zb, eb, s) per group
-    static constexpr int ST2_BYTES = CG * 16;    // (1/s, min, max, t << 16 | accepted)
-    static constexpr int Q_BYTES = (CG + 15) / 16 * 16;
-    static constexpr int SLOTS = GPW;            // phase-B slots per warp (this layout)
-    static constexpr int POOL_W_BYTES = SLOTS * G * 2;
-    static constexpr int POOL_ST_BYTES = SLOTS * 32;
-    static constexpr int POOL_GI_BYTES = (SLOTS * 8 + 15) / 16 * 16;
-    static constexpr int CHUNK_BYTES = W_BYTES + ST_BYTES + ST2_BYTES + Q_BYTES;
-    static constexpr int POOL_BYTES = POOL_W_BYTES + POOL_ST_BYTES + POOL_GI_BYTES;
-    // every region starts on a 16-byte boundary (128-bit shared-memory accesses)
-    static_assert(W_BYTES % 16 == 0 && ST_BYTES % 16 == 0 && ST2_BYTES % 16 == 0 &&
-                  Q_BYTES % 16 == 0 && POOL_W_BYTES % 16 == 0 && POOL_ST_BYTES % 16 == 0 &&
-                  POOL_GI_BYTES % 16 == 0, "shared-memory regions must be 16-byte multiples");
-    static_assert(K >= 1 && K <= 32 && kChunk % ROUND == 0, "bad layout");
-};
-
-// TAB2: the hot |x|^p uses the combined 32 KiB exponent x cell table (one
-// lookup fewer); otherwise the separate small tables (less shared memory).
-template <bool TAB2>
-struct QuantSmem {
-    std::conditional_t<TAB2, PowSmem2, PowSmem> tp;   // |x|^p
-    PowSmem tq;                 // |x|^(p-1)
-    float beta[kMaxIters + 1];  // beta_t = beta * kappa^t by repeated binary32 products
-    float thr[kMaxIters + 1];   // shrink thresholds
-};
-
-template <int K>
-__device__ __forceinline__ float2 group_sum2(float2 v) {
-#pragma unroll
-    for (int o = 1; o < K; o <<= 1) {
-        const float ux = __shfl_xor_sync(kFull, v.x, o), uy = __shfl_xor_sync(kFull, v.y, o);
-        v = make_float2(__fadd_rn(v.x, ux), __fadd_rn(v.y, uy));
-    }
-    return v;
-}
-
-template <int K>
-__device__ __forceinline__ void group_minmax(float& mn, float& mx) {
-#pragma unroll
-    for (int o = 1; o < K; o <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-    }
-}
-
-// NB blocks of 8 fp16 weights -> pairs (x_k, x_k+4) of each block.
-template <int NB>
-__device__ __forceinline__ void load_lane(const __half* src, float2 (&w)[NB][4]) {
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-        const uint4 raw = reinterpret_cast<const uint4*>(src)[b];
-        const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
-        const __half2 h23 = *reinterpret_cast<const __half2*>(&raw.y);
-        const __half2 h45 = *reinterpret_cast<const __half2*>(&raw.z);
-        const __half2 h67 = *reinterpret_cast<const __half2*>(&raw.w);
-        w[b][0] = make_float2(__low2float(h01), __low2float(h45));
-        w[b][1] = make_float2(__high2float(h01), __high2float(h45));
-        w[b][2] = make_float2(__low2float(h23), __low2float(h67));
-        w[b][3] = make_float2(__high2float(h23), __high2float(h67));
-    }
-}
-
-// load_lane plus the lane's min and max, taken on the packed fp16 values
-// (exact: the conversion to binary32 is exact and monotone).
-template <int NB>
-__device__ __forceinline__ void load_lane_minmax(const __half* src, float2 (&w)[NB][4],
-                                                 float& mn, float& mx) {
-    __half2 hmn, hmx;
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-        const uint4 raw = reinterpret_cast<const uint4*>(src)[b];
-        const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
-        const __half2 h23 = *reinterpret_cast<const __half2*>(&raw.y);
-        const __half2 h45 = *reinterpret_cast<const __half2*>(&raw.z);
-        const __half2 h67 = *reinterpret_cast<const __half2*>(&raw.w);
-        const __half2 bmn = __hmin2(__hmin2(h01, h23), __hmin2(h45, h67));
-        const __half2 bmx = __hmax2(__hmax2(h01, h23), __hmax2(h45, h67));
-        hmn = b == 0 ? bmn : __hmin2(hmn, bmn);
-        hmx = b == 0 ? bmx : __hmax2(hmx, bmx);
-        w[b][0] = make_float2(__low2float(h01), __low2float(h45));
-        w[b][1] = make_float2(__high2float(h01), __high2float(h45));
-        w[b][2] = make_float2(__low2float(h23), __low2float(h67));
-        w[b][3] = make_float2(__high2float(h23), __high2float(h67));
-    }
-    mn = fminf(__low2float(hmn), __high2float(hmn));
-    mx = fmaxf(__low2float(hmx), __high2float(hmx));
-}
-
-// Per-group constants of one evaluation, as f32x2 pairs.
-struct EvalConst {
-    float2 z, nz, ns, inv, ninv;
-    float s, invs;
-};
-
-// One error evaluation of the lane's weights at zero-point z.  Returns the
-// lane's pairwise sums of (|r|^p, sp2 term) where r = W - s(Wq - z) and the sp2
-// term is Wq - (W - W_e)/s.  CLAMP: codes may leave [0, L].  SHRINK: W_e is
-// evaluated exactly; otherwise W_e is known to be zero.
-template <int L, int NB, bool CLAMP, bool SHRINK, class SM>
-__device__ __forceinline__ float2 eval_lane(const SM& S, const float2 (&w)[NB][4],
-                                            const EvalConst& c, float2 pa1, float2 pa2,
-                                            float2 pa3, float qa1, float qa2, float qa3,
-                                            float beta) {
-    const float2 sh = make_float2(kRoundShift, kRoundShift);
-    const float2 nsh = make_float2(-kRoundShift, -kRoundShift);
-    float pe = 0.0f, pt = 0.0f;
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-        float2 P[4], T[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float2 v = __ffma2_rn(w[b][k], c.inv, c.z);                // W/s + z
-            if (CLAMP) {
-                v.x = fminf(fmaxf(v.x, 0.0f), (float)L);
-                v.y = fminf(fmaxf(v.y, 0.0f), (float)L);
-            }
-            const float2 q = __fadd2_rn(__fadd2_rn(v, sh), nsh);      // round half even
-            const float2 qz = __fadd2_rn(q, c.nz);                     // Wq - z
-            const float2 d = __ffma2_rn(qz, c.ns, w[b][k]);            // W - s(Wq - z)
-            P[k] = powp_hot(S.tp, pa1, pa2, pa3, d);
-            if (SHRINK) {
-                float we[2];
-                const float dd[2] = {d.x, d.y};
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float a = fabsf(dd[e]);
-                    const float y = __fsub_rn(a, __fdiv_rn(powp1(S.tq, qa1, qa2, qa3, a), beta));
-                    we[e] = copysignf(fmaxf(y, 0.0f), dd[e]);
-                }
-                T[k].x = __fmaf_rn(-__fsub_rn(w[b][k].x, we[0]), c.invs, q.x);
-                T[k].y = __fmaf_rn(-__fsub_rn(w[b][k].y, we[1]), c.invs, q.y);
-            } else {
-                T[k] = __ffma2_rn(w[b][k], c.ninv, q);                 // Wq - W/s
-            }
-        }
-        // ((x0+x1)+(x2+x3)) + ((x4+x5)+(x6+x7)) with pairs (x_k, x_k+4).  The
-        // reduction reads the pair halves one by one with scalar adds: a packed
-        // f32x2 add fed by the packed power results was found to combine the
-        // halves in the wrong order on this toolchain (the sums came out as if
-        // the pairs held adjacent weights), so no packed add is used here.
-        const float bp = __fadd_rn(__fadd_rn(__fadd_rn(P[0].x, P[1].x), __fadd_rn(P[2].x, P[3].x)),
-                                   __fadd_rn(__fadd_rn(P[0].y, P[1].y), __fadd_rn(P[2].y, P[3].y)));
-        const float bt = __fadd_rn(__fadd_rn(__fadd_rn(T[0].x, T[1].x), __fadd_rn(T[2].x, T[3].x)),
-                                   __fadd_rn(__fadd_rn(T[0].y, T[1].y), __fadd_rn(T[2].y, T[3].y)));
-        if (b == 0) {
-            pe = bp;
-            pt = bt;
-        } else {
-            pe = __fadd_rn(pe, bp);
-            pt = __fadd_rn(pt, bt);
-        }
-    }
-    return make_float2(pe, pt);
-}
-
-struct GroupState {
-    float z, zb, eb, s, inv, mn, mx;
-    int t;    // evaluations done
-    int na;   // evaluations accepted
-};
-
-// One solver iteration (error evaluation, early-stop test, sp1 + sp2) for the
-// sub-warp's group; `live` lanes only change state.  Returns true when the
-// group has finished (stopped, or used its iterations).
-template <int NBITS, int G, int NB, class SM>
-__device__ __forceinline__ bool solver_step(const SM& S, const QuantParams& prm,
-                                            const float2 (&w)[NB][4], GroupState& g, bool live,
-                                            float2 pa1, float2 pa2, float2 pa3,
-                                            float qa1, float qa2, float qa3) {
-    using C = QCfg<NBITS, G, NB>;
-    constexpr float L = (float)C::L;
-    const int t = live ? g.t : 0;
-    const float beta = S.beta[t];
-    const float vmin = __fmaf_rn(g.mn, g.inv, g.z);
-    const float vmax = __fmaf_rn(g.mx, g.inv, g.z);
-    const bool inside = vmin >= -0.5f && vmax < L + 0.5f;
-    const float reach = fmaxf(0.5f, fmaxf(-vmin, vmax - L)) + 1e-3f * (1.0f + fabsf(g.z));
-    const bool shrink = 2.0f * g.s * reach > S.thr[t];
-    EvalConst c;
-    c.z = make_float2(g.z, g.z);
-    c.nz = make_float2(-g.z, -g.z);
-    c.ns = make_float2(-g.s, -g.s);
-    c.inv = make_float2(g.inv, g.inv);
-    c.ninv = make_float2(-g.inv, -g.inv);
-    c.s = g.s;
-    c.invs = g.inv;
-    float2 r;
-    if (__any_sync(kFull, live && shrink))
-        r = eval_lane<C::L, NB, true, true>(S, w, c, pa1, pa2, pa3, qa1, qa2, qa3, beta);
-    else if (__all_sync(kFull, !live || inside))
-        r = eval_lane<C::L, NB, false, false>(S, w, c, pa1, pa2, pa3, qa1, qa2, qa3, beta);
-    else
-        r = eval_lane<C::L, NB, true, false>(S, w, c, pa1, pa2, pa3, qa1, qa2, qa3, beta);
-    r = group_sum2<C::K>(r);                       // (error, sp2 sum) of the whole group
-    const bool acc = live && r.x < g.eb;
-    bool repeat = false;
-    if (acc) {
-        const float zn = __fmul_rn(r.y, 1.0f / (float)G);
-        // the update reproduced the z just evaluated: the next evaluation would
-        // repeat this one exactly, its error would not fall, and the group would
-        // stop with the same best z -- so it stops now (identical outputs)
-        repeat = zn == g.z;
-        g.eb = r.x;
-        g.zb = g.z;
-        g.z = zn;
-        ++g.na;
-    }
-    if (live) ++g.t;
-    return live && (!acc || repeat || g.t == prm.iters);
-}
-
-// Group state kept in the chunk's shared memory between phases.
-__device__ __forceinline__ void save_state(float4* st, float4* st2, int gl, const GroupState& g) {
-    st[gl] = make_float4(g.z, g.zb, g.eb, g.s);
-    st2[gl] = make_float4(g.inv, g.mn, g.mx, __int_as_float((g.t << 16) | g.na));
-}
-
-__device__ __forceinline__ void load_state(const float4* st, const float4* st2, int gl,
-                                           GroupState& g) {
-    const float4 a = st[gl];
-    const float4 b = st2[gl];
-    g.z = a.x;
-    g.zb = a.y;
-    g.eb = a.z;
-    g.s = a.w;
-    g.inv = b.x;
-    g.mn = b.y;
-    g.mx = b.z;
-    const int tn = __float_as_int(b.w);
-    g.t = (tn >> 16) & 0xFF;
-    g.na = tn & 0xFFFF;
-}
-
-constexpr int kCarried = 1 << 30;   // flag in the packed (t, accepted) word
-constexpr int kPoolTag = 256;       // queue handles >= kPoolTag name pool entries
-
-// Pack the lane's weights back to fp16 in memory order (exact: they came from fp16).
-template <int NB>
-__device__ __forceinline__ void store_lane(__half* dst, const float2 (&w)[NB][4]) {
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-        const __half2 h01 = __floats2half2_rn(w[b][0].x, w[b][1].x);
-        const __half2 h23 = __floats2half2_rn(w[b][2].x, w[b][3].x);
-        const __half2 h45 = __floats2half2_rn(w[b][0].y, w[b][1].y);
-        const __half2 h67 = __floats2half2_rn(w[b][2].y, w[b][3].y);
-        uint4 raw;
-        raw.x = *reinterpret_cast<const uint32_t*>(&h01);
-        raw.y = *reinterpret_cast<const uint32_t*>(&h23);
-        raw.z = *reinterpret_cast<const uint32_t*>(&h45);
-        raw.w = *reinterpret_cast<const uint32_t*>(&h67);
-        reinterpret_cast<uint4*>(dst)[b] = raw;
-    }
-}
-
-// Final codes of one group finished after its chunk was written (a group
-// carried over to a later chunk): codes go straight to HBM; 3 bit codes are
-// OR-ed into the words, whose bits for this group were written as zero.
-template <int NBITS, int G, int NB>
-__device__ __forceinline__ void finalize_direct(const QuantParams& prm, const float2 (&w)[NB][4],
-                                                const GroupState& g, int64_t gi, int kl) {
-    constexpr float L = (float)((1 << NBITS) - 1);
-    const float2 inv2 = make_float2(g.inv, g.inv), zb2 = make_float2(g.zb, g.zb);
-    uint32_t c[NB][8];
-#pragma unroll
-    for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float2 v = __ffma2_rn(w[b][k], inv2, zb2);
-            v.x = fminf(fmaxf(v.x, 0.0f), L);
-            v.y = fminf(fmaxf(v.y, 0.0f), L);
-            const float2 t = __fadd2_rn(v, make_float2(kRoundShift, kRoundShift));
-            c[b][k] = __float_as_uint(t.x) & 0xFFu;
-            c[b][k + 4] = __float_as_uint(t.y) & 0xFFu;
-        }
-    if constexpr (NBITS == 3) {
-        const int64_t e0 = gi * G + (int64_t)kl * 8 * NB;    // first element of the lane
-        const int64_t w0 = e0 / 10;
-        uint32_t acc[3] = {0u, 0u, 0u};                       // 8 NB <= 16 codes span <= 3 words
-        int off = (int)(e0 - w0 * 10);
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int pos = off + 8 * b + i;
-                const int wi = pos / 10;
-                const uint32_t bits = c[b][i] << (3 * (pos - 10 * wi));
-                if (wi == 0) acc[0] |= bits;
-                else if (wi == 1) acc[1] |= bits;
-                else acc[2] |= bits;
-            }
-        uint32_t* p32 = reinterpret_cast<uint32_t*>(prm.packed);
-#pragma unroll
-        for (int k = 0; k < 3; ++k)
-            if (acc[k]) atomicOr(p32 + w0 + k, acc[k]);
-    } else {
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            const int64_t unit = gi * (G / 8) + kl * NB + b;
-            uint32_t word = 0;
-            if constexpr (NBITS == 8) {
-                uint2 bb;
-                bb.x = c[b][0] | (c[b][1] << 8) | (c[b][2] << 16) | (c[b][3] << 24);
-                bb.y = c[b][4] | (c[b][5] << 8) | (c[b][6] << 16) | (c[b][7] << 24);
-                reinterpret_cast<uint2*>(prm.packed)[unit] = bb;
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) word |= c[b][i] << (NBITS * i);
-                if constexpr (NBITS == 4)
-                    reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
-                else if constexpr (NBITS == 2)
-                    reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)word;
-                else
-                    prm.packed[unit] = (uint8_t)word;
-            }
-        }
-    }
-    if (kl == 0) {
-        prm.scale[gi] = __float2half_rn(g.s);
-        prm.zero[gi] = __float2half_rn(g.zb);
-        if (prm.zero_f32) prm.zero_f32[gi] = g.zb;
-        if (prm.err_out) prm.err_out[gi] = g.eb;
-        if (prm.iters_out) prm.iters_out[gi] = (uint8_t)g.na;
-    }
-}
-
-// Final codes of every group of a chunk (one uniform pass, phase-A layout),
-// from the staged weights and each group's (z_best, 1/s); 8, 4, 2 and 1 bit
-// codes are stored straight to HBM, 3 bit code bytes overwrite the front of the
-// chunk's weight buffer (round r writes bytes [512r, 512r+512), never ahead of
-// the weights still to be read) for word packing.  Scale, zero and the
-// diagnostics are written by each group's first lane.
-template <int NBITS, int G, int NB>
-__device__ __forceinline__ void final_pass(const QuantParams& prm, __half* s_w, const float4* st,
-                                           const float4* st2, int64_t chunk, int cg, int lane) {
-    using C = QCfg<NBITS, G, NB>;
-    constexpr float L = (float)C::L;
-    const int sub = lane / C::K, kl = lane % C::K;
-    uint8_t* codes = reinterpret_cast<uint8_t*>(s_w);
-    for (int r = 0; r < C::ROUNDS; ++r) {
-        if (r * C::GPW >= cg) break;
-        const int gl = r * C::GPW + sub;
-        const bool valid = gl < cg;
-        float2 w[NB][4];
-        GroupState g;
-        bool mine = valid;                          // false: carried over, finalised later
-        if (valid) {
-            load_lane<NB>(s_w + gl * G + kl * C::EPL, w);
-            load_state(st, st2, gl, g);
-            mine = (__float_as_int(st2[gl].w) & kCarried) == 0;
-        } else {
-#pragma unroll
-            for (int b = 0; b < NB; ++b)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) w[b][k] = make_float2(0.0f, 0.0f);
-            g.zb = 0.0f;
-            g.inv = 1.0f;
-        }
-        if constexpr (NBITS == 3) __syncwarp();     // all reads of the round before any write
-        const float2 inv2 = make_float2(g.inv, g.inv), zb2 = make_float2(g.zb, g.zb);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            uint32_t c[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float2 v = __ffma2_rn(w[b][k], inv2, zb2);
-                v.x = fminf(fmaxf(v.x, 0.0f), L);
-                v.y = fminf(fmaxf(v.y, 0.0f), L);
-                const float2 t = __fadd2_rn(v, make_float2(kRoundShift, kRoundShift));
-                c[k] = mine ? __float_as_uint(t.x) & 0xFFu : 0u;
-                c[k + 4] = mine ? __float_as_uint(t.y) & 0xFFu : 0u;
-            }
-            if (!valid || (!mine && NBITS != 3)) continue;
-            const int64_t unit = chunk * (kChunk / 8) + gl * (G / 8) + kl * NB + b;
-            if constexpr (NBITS == 4) {
-                uint32_t word = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) word |= c[i] << (4 * i);
-                reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
-            } else if constexpr (NBITS == 2) {
-                uint32_t h = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) h |= c[i] << (2 * i);
-                reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)h;
-            } else if constexpr (NBITS == 1) {
-                uint32_t h = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) h |= c[i] << i;
-                prm.packed[unit] = (uint8_t)h;
-            } else if constexpr (NBITS == 8) {
-                uint2 bb;
-                bb.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-                bb.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-                reinterpret_cast<uint2*>(prm.packed)[unit] = bb;
-            } else {
-                uint2 bb;
-                bb.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-                bb.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-                *reinterpret_cast<uint2*>(codes + gl * G + (kl * NB + b) * 8) = bb;
-            }
-        }
-        if (mine && kl == 0) {
-            const int64_t gi = chunk * C::CG + gl;
-            prm.scale[gi] = __float2half_rn(g.s);
-            prm.zero[gi] = __float2half_rn(g.zb);
-            if (prm.zero_f32) prm.zero_f32[gi] = g.zb;
-            if (prm.err_out) prm.err_out[gi] = g.eb;
-            if (prm.iters_out) prm.iters_out[gi] = (uint8_t)g.na;
-        }
-    }
-}
-
-// NB / NBB: 8-weight blocks per lane in phase A / phase B.  CARRY: park the
-// last busy groups of a chunk and resume them with the next chunk, parking
-// once at most PARK/4 of the phase-B slots are busy.  TAB2: combined power
-// table (off for G = 16, whose per-group state already fills the shared memory
-// that two resident CTAs per SM can have).
-template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK, bool TAB2>
-__global__ void __launch_bounds__(kQWarps * 32, 2)
-quantize_kernel(const __grid_constant__ QuantParams prm) {
-    using C = QCfg<NBITS, G, NB>;      // phase A layout (and the chunk's shared memory)
-    using CB = QCfg<NBITS, G, NBB>;    // phase B layout
-    __shared__ QuantSmem<TAB2> S;
-    extern __shared__ __align__(16) uint8_t dyn[];
-
-    load_pow_hot(S.tp, prm.tp);
-    load_pow_smem(S.tq, prm.tq);
-    for (int i = threadIdx.x; i < prm.iters; i += blockDim.x) S.thr[i] = prm.shrink_thr[i];
-    if (threadIdx.x == 0) {
-        float b = prm.beta;
-        for (int t = 0; t < prm.iters; ++t) {
-            S.beta[t] = b;
-            b = __fmul_rn(b, prm.kappa);
-        }
-        S.beta[prm.iters] = b;
-        S.thr[prm.iters] = 0.0f;
-    }
-    __syncthreads();
-
-    const float2 pa1 = make_float2(prm.tp.a1, prm.tp.a1);
-    const float2 pa2 = make_float2(prm.tp.a2, prm.tp.a2);
-    const float2 pa3 = make_float2(prm.tp.a3, prm.tp.a3);
-    const float qa1 = prm.tq.a1, qa2 = prm.tq.a2, qa3 = prm.tq.a3;
-
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int sub = lane / C::K;
-    const int kl = lane % C::K;
-    const bool leader = kl == 0;
-    constexpr int WARP_BYTES = C::CHUNK_BYTES + (CARRY ? CB::POOL_BYTES : 0);
-    uint8_t* wb = dyn + warp * WARP_BYTES;
-    __half* s_w = reinterpret_cast<__half*>(wb);
-    float4* s_st = reinterpret_cast<float4*>(wb + C::W_BYTES);
-    float4* s_st2 = reinterpret_cast<float4*>(wb + C::W_BYTES + C::ST_BYTES);
-    uint8_t* s_q = wb + C::W_BYTES + C::ST_BYTES + C::ST2_BYTES;
-    __half* pool_w = reinterpret_cast<__half*>(s_q + C::Q_BYTES);
-    float4* pool_st = reinterpret_cast<float4*>(s_q + C::Q_BYTES + CB::POOL_W_BYTES);
-    int64_t* pool_gi = reinterpret_cast<int64_t*>(s_q + C::Q_BYTES + CB::POOL_W_BYTES +
-                                                  CB::POOL_ST_BYTES);
-    int np = 0;                        // groups parked in the pool by the last yield
-
-    const int64_t n_chunks = (prm.n_elems + kChunk - 1) / kChunk;
-    for (int64_t chunk = (int64_t)blockIdx.x * kQWarps + warp; chunk < n_chunks;
-         chunk += (int64_t)gridDim.x * kQWarps) {
-        const int64_t e0 = chunk * kChunk;
-        const int64_t left = prm.n_elems - e0;
-        const int n_here = left < kChunk ? (int)left : kChunk;
-        const int cg = n_here / G;
-
-        // ---- stage the chunk's weights (one pass over HBM) ---------------------
-        {
-            const uint4* src = reinterpret_cast<const uint4*>(prm.W + e0);
-            uint4* dst = reinterpret_cast<uint4*>(s_w);
-            for (int u = lane; u < n_here / 8; u += 32) dst[u] = __ldg(src + u);
-        }
-        __syncwarp();
-
-        // ---- phase A: initialise + first two iterations, all groups in step ---
-        int qn = 0;
-        for (int r = 0; r < C::ROUNDS; ++r) {
-            if (r * C::GPW >= cg) break;
-            const int gl = r * C::GPW + sub;
-            const bool valid = gl < cg;
-            float2 w[NB][4];
-            float mn, mx;
-            if (valid) {
-                load_lane_minmax<NB>(s_w + gl * G + kl * C::EPL, w, mn, mx);
-            } else {
-#pragma unroll
-                for (int b = 0; b < NB; ++b)
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) w[b][k] = make_float2(0.0f, 0.0f);
-                mn = mx = 0.0f;
-            }
-            GroupState g;
-            group_minmax<C::K>(mn, mx);
-            g.mn = mn;
-            g.mx = mx;
-            const float rng = __fsub_rn(mx, mn);
-            g.s = 1.0f;
-            g.inv = 1.0f;
-            if (rng != 0.0f) {
-                g.s = __fdiv_rn(rng, (float)C::L);
-                g.inv = __frcp_rn(g.s);             // correctly rounded 1/s
-            }
-            g.z = -__fmul_rn(mn, g.inv);
-            g.zb = g.z;
-            g.eb = __int_as_float(0x7F800000);
-            g.t = 0;
-            g.na = 0;
-            bool live = valid && prm.iters > 0;
-            bool done = valid && prm.iters == 0;
-            const int ta = prm.iters < 2 ? prm.iters : 2;
-            for (int tt = 0; tt < ta; ++tt) {
-                const bool fin = solver_step<NBITS, G, NB>(S, prm, w, g, live, pa1, pa2, pa3,
-                                                           qa1, qa2, qa3);
-                done = done || fin;
-                live = live && !fin;
-            }
-            if ((done || live) && leader) save_state(s_st, s_st2, gl, g);
-            const unsigned pmask = __ballot_sync(kFull, live && leader);
-            if (live && leader) s_q[qn + __popc(pmask & ((1u << lane) - 1u))] = (uint8_t)gl;
-            qn += __popc(pmask);
-        }
-        __syncwarp();
-
-        // ---- phase B: queued groups, refilled as each sub-warp finishes -------
-        // The queue holds the groups parked by the previous chunk (pool entries
-        // 0..np-1) and then this chunk's continuing groups.  Once the queue is
-        // empty and at most half the slots are busy, the warp parks the busy
-        // groups in the pool and moves on (unless this is its last chunk), so the
-        // longest groups never leave the other slots idle.
-        {
-            const int subb = lane / CB::K;
-            const int klb = lane % CB::K;
-            const bool leadb = klb == 0;
-            const bool more = CARRY && chunk + (int64_t)gridDim.x * kQWarps < n_chunks;
-            const int nq = np + qn;
-            int head = 0;
-            bool live = false;
-            int hnd = 0;                   // < kPoolTag: chunk group gl; else pool entry
-            int64_t gi = 0;
-            GroupState g;
-            g.z = g.zb = g.eb = g.s = g.inv = g.mn = g.mx = 0.0f;
-            g.t = 0;
-            g.na = 0;
-            float2 w[NBB][4];
-#pragma unroll
-            for (int b = 0; b < NBB; ++b)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) w[b][k] = make_float2(0.0f, 0.0f);
-            int parked = 0;
-            while (true) {
-                const unsigned want = __ballot_sync(kFull, !live && leadb);
-                if (head < nq && want) {
-                    const int slot = head + __popc(want & ((1u << (subb * CB::K)) - 1u));
-                    if (!live && slot < nq) {
-                        if (CARRY && slot < np) {
-                            hnd = kPoolTag + slot;
-                            load_lane<NBB>(pool_w + slot * G + klb * CB::EPL, w);
-                            load_state(pool_st, pool_st + CB::SLOTS, slot, g);
-                            gi = pool_gi[slot];
-                        } else {
-                            hnd = s_q[slot - np];
-                            load_lane<NBB>(s_w + hnd * G + klb * CB::EPL, w);
-                            load_state(s_st, s_st2, hnd, g);
-                            gi = chunk * C::CG + hnd;
-                        }
-                        live = true;
-                    }
-                    head = min(nq, head + __popc(want));
-                }
-                const unsigned lmask = __ballot_sync(kFull, live && leadb);
-                if (lmask == 0) break;
-                if (more && head >= nq && 4 * __popc(lmask) <= PARK * CB::SLOTS) {
-                    // park the busy groups (the pool's old entries are all taken)
-                    __syncwarp();
-                    if (live) {
-                        const int j = __popc(lmask & ((1u << (subb * CB::K)) - 1u));
-                        store_lane<NBB>(pool_w + j * G + klb * CB::EPL, w);
-                        if (leadb) {
-                            save_state(pool_st, pool_st + CB::SLOTS, j, g);
-                            pool_gi[j] = gi;
-                            if (hnd < kPoolTag)          // exclude it from the chunk pass
-                                s_st2[hnd].w = __int_as_float(__float_as_int(s_st2[hnd].w) |
-                                                              kCarried);
-                        }
-                    }
-                    parked = __popc(lmask);
-                    break;
-                }
-                const bool fin = solver_step<NBITS, G, NBB>(S, prm, w, g, live, pa1, pa2, pa3,
-                                                            qa1, qa2, qa3);
-                if (fin) {
-                    if (!CARRY || hnd < kPoolTag) {
-                        if (leadb) save_state(s_st, s_st2, hnd, g);
-                    } else {
-                        finalize_direct<NBITS, G, NBB>(prm, w, g, gi, klb);
-                    }
-                }
-                live = live && !fin;
-            }
-            np = parked;
-        }
-
-        // ---- final codes of the whole chunk, then 3-bit words -------------------
-        __syncwarp();
-        final_pass<NBITS, G, NB>(prm, s_w, s_st, s_st2, chunk, cg, lane);
-        if constexpr (NBITS == 3) {
-            uint8_t* s_codes = reinterpret_cast<uint8_t*>(s_w);
-            __syncwarp();
-            const int n_words = (n_here + 9) / 10;
-            if (lane < n_words * 10 - n_here) s_codes[n_here + lane] = 0;   // zero padding
-            __syncwarp();
-            const int64_t total_words = (prm.n_elems + 9) / 10;
-            for (int k = lane; k < n_words; k += 32) {
-                const uint16_t* src = reinterpret_cast<const uint16_t*>(s_codes) + k * 5;
-                uint32_t word = 0;
-#pragma unroll
-                for (int i = 0; i < 5; ++i) {
-                    const uint32_t two = src[i];
-                    word |= ((two & 0xFFu) | ((two >> 8) << 3)) << (6 * i);
-                }
-                const int64_t wi = chunk * (kChunk / 10) + k;
-                if (wi < total_words) reinterpret_cast<uint32_t*>(prm.packed)[wi] = word;
-            }
-        }
-        __syncwarp();
-    }
-}
-
-template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK, bool TAB2 = (G > 16)>
-static cudaError_t launch_quantize_g(const QuantParams& prm, cudaStream_t stream) {
-    using C = QCfg<NBITS, G, NB>;
-    using CB = QCfg<NBITS, G, NBB>;
-    constexpr int SMEM = kQWarps * (C::CHUNK_BYTES + (CARRY ? CB::POOL_BYTES : 0));
-    auto kern = quantize_kernel<NBITS, G, NB, NBB, CARRY, PARK, TAB2>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    if (err != cudaSuccess) return err;
-    int dev = 0, sms = 148, per_sm = 1;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQWarps * 32, SMEM);
-    if (err != cudaSuccess) return err;
-    if (per_sm < 1) per_sm = 1;
-    const int64_t n_chunks = (prm.n_elems + kChunk - 1) / kChunk;
-    const int64_t want = (n_chunks + kQWarps - 1) / kQWarps;
-    const int64_t cap = (int64_t)sms * per_sm;
-    const unsigned grid = (unsigned)(want < cap ? want : cap);
-    kern<<<grid, kQWarps * 32, SMEM, stream>>>(prm);
-    return cudaGetLastError();
-}
-
-// 16 weights per lane in both phases.  4 bit: park the last busy groups of a
-// chunk once at most half the slots are busy (measured faster); 3 and 2 bit:
-// drain each chunk (measured faster: their carried groups cost more to
-// finalise one by one than the idle slots they save).
-template <int NBITS>
-static cudaError_t launch_quantize_b(const QuantParams& prm, int group, cudaStream_t stream) {
-    constexpr bool carry = NBITS == 4;
-    switch (group) {
-        case 16: return launch_quantize_g<NBITS, 16, 2, 2, carry, 2>(prm, stream);
-        case 32: return launch_quantize_g<NBITS, 32, 2, 2, carry, 2>(prm, stream);
-        case 64: return launch_quantize_g<NBITS, 64, 2, 2, carry, 2>(prm, stream);
-        case 128: return launch_quantize_g<NBITS, 128, 2, 2, carry, 2>(prm, stream);
-        case 256: return launch_quantize_g<NBITS, 256, 2, 2, carry, 2>(prm, stream);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
 cudaError_t launch_quantize(const QuantParams& prm, int nbits, int group, cudaStream_t stream) {
-    switch (nbits) {
-        case 1: return launch_quantize_b<1>(prm, group, stream);
-        case 2: return launch_quantize_b<2>(prm, group, stream);
-        case 3: return launch_quantize_b<3>(prm, group, stream);
-        case 4: return launch_quantize_b<4>(prm, group, stream);
-        case 8: return launch_quantize_b<8>(prm, group, stream);
-        default: return cudaErrorInvalidValue;
-    }
+    return launch_quantize_nb<false>(prm, nbits, group, stream);
 }
 
 }  // namespace hqq
