@@ -32,14 +32,18 @@ if ROOT not in sys.path:
 
 METRIC = "Gparams/s quantized & achieved HBM GB/s vs B200 peak; Llama-2-70B-shaped wall time"
 
-# Algorithmic binary32 operations per weight of the canonical solver (see the
-# design notes): initialisation (convert, min, max), one error evaluation
-# (code: fma, 2 clamps, round; residual: sub, fma; |.|; table power: 4 bit-field
-# ops, sub, mul, 3 fma, 2 mul; accumulate), one accepted update with W_e == 0
-# (threshold test, fma, accumulate), final code and packing (fma, 2 clamps,
-# round, shift, or).
+# Algorithmic binary32 operations per weight of the canonical solver, counted
+# by hand from its steps (reported beside the measured instruction count, not
+# used for the roofline): initialisation (convert, min, max), one error
+# evaluation (code: fma, 2 clamps, round; residual: sub, fma; |.|; table power:
+# 4 bit-field ops, sub, mul, 3 fma, 2 mul; accumulate), one accepted update
+# with W_e == 0 (threshold test, fma, accumulate), final code and packing
+# (fma, 2 clamps, round, shift, or).
 OPS_INIT, OPS_EVAL, OPS_UPDATE, OPS_FINAL = 3, 19, 3, 6
 ALU_LANES_PER_SM = 128
+# Each SM has four warp schedulers, each issuing at most one warp instruction
+# per cycle: the issue peak the quantize kernel's instruction count is held to.
+ISSUE_PER_SM_CLK = 4
 
 
 # ------------------------------------------------------------------ workloads
@@ -175,12 +179,14 @@ def tensor_peak():
         return 1590.0
 
 
-def profiled_traffic(kernel: str, fmt: str):
-    """DRAM bytes per weight of `kernel` from the committed ncu summary, or None
-    when the kernel's sources changed since the counters were taken."""
+def profiled_counters(kernel: str, fmt: str):
+    """Per-weight counters of `kernel` from the committed ncu summary whose
+    source hash matches the current sources: DRAM bytes per weight and warp
+    instructions per weight (each None when absent), and the summary's path;
+    all None when the kernel's sources changed since the counters were taken."""
     import glob
     import hashlib
-    srcs = {"quantize_kernel": ["hqq_quantize.cu", "hqq_common.cuh"],
+    srcs = {"quantize_kernel": ["hqq_quantize.cuh", "hqq_common.cuh"],
             "dequantize_kernel": ["hqq_dequantize.cu", "hqq_common.cuh"]}[kernel]
     m = hashlib.sha256()
     for f in srcs:
@@ -194,9 +200,12 @@ def profiled_traffic(kernel: str, fmt: str):
                 if ":" in line and not line.startswith("#"):
                     k, _, v = line.partition(":")
                     kv[k.strip()] = v.strip()
-        if kv.get("source_sha256_16") == cur and "traffic_bytes_per_param" in kv:
-            return float(kv["traffic_bytes_per_param"]), os.path.relpath(path, ROOT)
-    return None, None
+        if kv.get("source_sha256_16") == cur:
+            get = lambda k: float(kv[k]) if k in kv else None
+            return {"traffic_bytes_per_param": get("traffic_bytes_per_param"),
+                    "warp_inst_per_param": get("warp_inst_per_param"),
+                    "source": os.path.relpath(path, ROOT)}
+    return {"traffic_bytes_per_param": None, "warp_inst_per_param": None, "source": None}
 
 
 def cpu_model():
@@ -241,17 +250,21 @@ def oracle_sample(mats, W_source, target_s: float):
     rows = max(8, min(min(s[0] for _, s, *_ in picks), int(budget / total_cols)))
     sample = [(lab, W_source(lab, shape, rows, seed, stream), nb, g)
               for lab, shape, nb, g, seed, stream in picks]
-    desc = ", ".join(f"first {rows} rows of {lab.split('.')[-1]} {shape[0]}x{shape[1]}"
-                     for lab, shape, *_ in picks)
+    desc = "quantize + dequantize of the first %d rows of each distinct matrix: " % rows + \
+        ", ".join(f"{lab.split('.')[-1]} {shape[0]}x{shape[1]}" for lab, shape, *_ in picks)
     return sample, desc, cores
 
 
 def run_oracle_sample(sample, cores):
+    """The step on the sample: quantize every sampled matrix, then dequantize
+    its codes (the oracle's quantize is threaded over groups, its dequantize
+    runs on one core)."""
     import oracle
     n = 0
     t0 = time.perf_counter()
     for _, W, nb, g in sample:
-        oracle.quantize(W, nb, g, threads=cores)
+        r = oracle.quantize(W, nb, g, threads=cores)
+        oracle.dequantize(r["codes"], r["scale"], r["zero"], g)
         n += W.size
     return n, time.perf_counter() - t0
 
@@ -333,6 +346,16 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
         pg = dist
+
+    # ---- the other workloads first (their memory is released before the main
+    # set is allocated): quantize and dequantize GB/s per matrix (single
+    # matrices and the 70B pair) or per set (the 7B-shaped set), each pass
+    # replayed as a CUDA graph with L2 flushed before every repetition
+    configs = None
+    if not args.no_configs:
+        configs = run_configs(hqq, dev, measured_peaks()[0], pg, rank)
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
 
     mats = workload(args.workload, rank, args.layers)
     params = sum(r * c for _, (r, c), *_ in mats)
@@ -468,14 +491,37 @@ def run_gpu(args):
     mean_acc = float((acc_hist * acc).sum() / n_groups_hist)
     mean_eval = float((acc_hist * evals).sum() / n_groups_hist)
     ops_per_weight = OPS_INIT + OPS_FINAL + mean_eval * OPS_EVAL + mean_acc * OPS_UPDATE
-    ops_per_launch = ops_per_weight * params / len(views)
     props = torch.cuda.get_device_properties(dev)
     sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
-    alu_peak = props.multi_processor_count * ALU_LANES_PER_SM * sm_mhz * 1e6 / 1e12  # Tops/s
-    achieved = ops_per_launch / (q_launch_ms / 1e3) / 1e12
+
+    # ---- roofline of the dominant kernel (quantize_kernel): the issue rate of
+    # its warp instructions (counted by ncu on the committed profile of the
+    # same sources, per weight) against 4 warp instructions per SM per cycle at
+    # the SM clock sampled during the timed region; HBM fraction beside it
     fmts = sorted({f"{m[2]}b_g{m[3]}" for m in mats})
-    tpp, tsrc = profiled_traffic("quantize_kernel", fmts[0]) if len(fmts) == 1 else (None, None)
-    traffic = tpp * params / len(views) if tpp is not None else None
+    ctr = profiled_counters("quantize_kernel", fmts[0]) if len(fmts) == 1 else \
+        {"traffic_bytes_per_param": None, "warp_inst_per_param": None, "source": None}
+    w_per_launch = params / len(views)
+    traffic = (ctr["traffic_bytes_per_param"] * w_per_launch
+               if ctr["traffic_bytes_per_param"] is not None else None)
+    issue_peak = props.multi_processor_count * ISSUE_PER_SM_CLK * sm_mhz * 1e6 / 1e12  # T inst/s
+    ipw = ctr["warp_inst_per_param"]
+    issue_achieved = ipw * params / q_step_s / 1e12 if ipw is not None else None
+    alu_peak = props.multi_processor_count * ALU_LANES_PER_SM * sm_mhz * 1e6 / 1e12  # Tops/s
+    roof = {"kernel": "quantize_kernel", "bound": "alu",
+            "achieved": issue_achieved, "peak": issue_peak, "unit": "T warp-inst/s",
+            "frac": issue_achieved / issue_peak if issue_achieved is not None else None,
+            "traffic": traffic, "traffic_unit": "bytes per launch",
+            "counter_source": ctr["source"],
+            "peak_source": f"{props.multi_processor_count} SMs x {ISSUE_PER_SM_CLK} warp "
+                           f"instructions per cycle x {sm_mhz:.0f} MHz (sampled)",
+            "warp_inst_per_weight_measured": ipw,
+            "ops_per_weight_algorithmic": ops_per_weight,
+            "algorithmic_ops_frac_of_fp32_lanes":
+                ops_per_weight * params / q_step_s / 1e12 / alu_peak,
+            "hbm": {"achieved_gbs": quant_gbs, "peak_gbs": hbm_peak,
+                    "frac": quant_gbs / hbm_peak, "peak_kind": peak_kind,
+                    "algorithmic_bytes_per_weight": qbytes / params}}
 
     line = {"metric": METRIC, "value": value, "unit": "Gparam/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -488,15 +534,7 @@ def run_gpu(args):
                          "mean_accepted_iters": mean_acc, "mean_evaluations": mean_eval},
             "dequantize": {"gbs": dq_gbs, "hbm_frac": dq_gbs / hbm_peak,
                            "ms_per_pass": dq_ms_step},
-            "roofline": {"kernel": "quantize_kernel", "bound": "alu", "achieved": achieved,
-                         "peak": alu_peak, "unit": "Tops/s", "frac": achieved / alu_peak,
-                         "traffic": traffic, "traffic_unit": "bytes per launch",
-                         "traffic_source": tsrc,
-                         "peak_source": f"{props.multi_processor_count} SMs x "
-                                        f"{ALU_LANES_PER_SM} fp32 lanes x {sm_mhz:.0f} MHz",
-                         "ops_per_weight": ops_per_weight,
-                         "hbm": {"achieved_gbs": quant_gbs, "peak_gbs": hbm_peak,
-                                 "frac": quant_gbs / hbm_peak, "peak_kind": peak_kind}},
+            "roofline": roof,
             "gpu_launches": 2 * len(views) * args.steps,
             "clocks": clk}
 
@@ -512,6 +550,10 @@ def run_gpu(args):
     # which overwrites the HQQ codes)
     if not args.no_lowrank:
         line["lowrank"] = run_lowrank(views, hqq, dev, alu_peak, pg)
+
+    # ---- the half-precision solver over the same set (overwrites the codes;
+    # runs after the sections above, which use the single-precision ones)
+    line["quantize_fp16"] = run_quantize_half(views, hqq, dev, hbm_peak, qbytes, pg)
 
     # ---- memory-side calibration: round-to-nearest quantize pass (HBM-bound;
     # runs after the sections above, which use the HQQ codes)
@@ -542,6 +584,8 @@ def run_gpu(args):
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, mats, views, hqq, dev, pg, ws)
 
+    if configs is not None:
+        line["configs"] = configs
     del views, Wbuf, Pbuf, Sbuf, Zbuf, Obuf
     if rank == 0:
         print(json.dumps(line))
@@ -549,6 +593,89 @@ def run_gpu(args):
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def run_configs(hqq, dev, hbm_peak, pg, rank):
+    """Quantize and dequantize GB/s of every other workload, on device-resident
+    inputs: the 1024x1024 matrix (4-bit g64), the 4096x4096 matrix at 4-bit g64
+    and 2-bit g32, the 8192x8192 and 28672x8192 pair at 2-bit g32 and g128 (per
+    matrix), and the 7B-shaped set at 4-bit g64 (the whole set per pass).  Each
+    pass is a CUDA graph of the library calls, repeated with a 256 MiB buffer
+    written before every repetition (outside its events), so no repetition
+    starts with its inputs in the 126 MB L2."""
+    import torch
+    import synth
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps):
+        g = torch.cuda.CUDAGraph()
+        fn()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(3):
+            flush.fill_(1)
+            g.replay()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        torch.cuda.synchronize()
+        for r in range(reps):
+            flush.fill_(r & 0xFF)
+            evs[r][0].record(stream)
+            g.replay()
+            evs[r][1].record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+        del g
+        return max_over_ranks([ms], pg, dev)[0]
+
+    def record(mats, ms_q, ms_d):
+        params = sum(r * c for _, (r, c), *_ in mats)
+        nbytes = algorithmic_bytes(mats)
+        out = {}
+        for name, ms in (("quantize", ms_q), ("dequantize", ms_d)):
+            gbs = nbytes / (ms / 1e3) / 1e9
+            out[name] = {"ms": ms, "gparam_s": params / (ms / 1e3) / 1e9, "gbs": gbs,
+                         "hbm_frac": gbs / hbm_peak}
+        return out
+
+    def prepare(mats):
+        res = []
+        for lab, (r, c), nb, g, seed, st in mats:
+            W = torch.empty((r, c), dtype=torch.float16, device=dev)
+            synth.fill_student_t_(W, seed=seed, stream=st)
+            q = hqq.hqq_quantize(W, nb, g)
+            res.append((lab, W, q, torch.empty((r, c), dtype=torch.float16, device=dev)))
+        return res
+
+    out = {"method": "median of the repetitions; CUDA graph per pass; 256 MiB written "
+                     "between repetitions (L2 flush); algorithmic bytes 2 + packed + 4/group "
+                     "per weight in both directions"}
+    for name in ("matrix-1024", "matrix-4096", "70b-pair"):
+        mats = workload(name, rank)
+        rows = []
+        for (lab, W, q, O), m in zip(prepare(mats), mats):
+            ms_q = timed(lambda: hqq.hqq_quantize(W, q.nbits, q.group, packed=q.packed,
+                                                  scale=q.scale, zero=q.zero), 20)
+            ms_d = timed(lambda: hqq.hqq_dequantize(q, out=O), 20)
+            rows.append({"matrix": lab, **record([m], ms_q, ms_d)})
+        out[name] = rows
+        torch.cuda.empty_cache()
+    mats = workload("llama2-7b", rank)
+    set7 = prepare(mats)
+
+    def q_all():
+        for lab, W, q, O in set7:
+            hqq.hqq_quantize(W, q.nbits, q.group, packed=q.packed, scale=q.scale, zero=q.zero)
+
+    def d_all():
+        for lab, W, q, O in set7:
+            hqq.hqq_dequantize(q, out=O)
+    out["llama2-7b"] = {"matrices": len(mats), **record(mats, timed(q_all, 5), timed(d_all, 5))}
+    del set7
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_meta8(args, views, hqq, dev, hbm_peak, pg):
@@ -630,6 +757,52 @@ def run_meta8(args, views, hqq, dev, hbm_peak, pg):
                                 "hbm_frac": dq_gbs / hbm_peak,
                                 "gparam_s": params / (dq_ms / 1e3) / 1e9,
                                 "bytes_per_param": dq_bytes / params}}
+
+
+def run_quantize_half(views, hqq, dev, hbm_peak, qbytes, pg):
+    """The quantize pass with the half-precision solver (hqq_quantize_half: the
+    page's fp16 solve) over every matrix, replayed as a CUDA graph; with the
+    mean accepted iterations and the share of groups solved in fp16."""
+    import torch
+    stream = torch.cuda.current_stream()
+
+    def half_all():
+        for W, q, _ in views:
+            hqq.hqq_quantize(W, q.nbits, q.group, packed=q.packed, scale=q.scale, zero=q.zero,
+                             precision="fp16")
+
+    half_all()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        half_all()
+    for _ in range(2):
+        g.replay()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    reps = 3
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(reps):
+        g.replay()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps], pg, dev)[0]
+    del g
+    acc = n_half = n_groups = 0
+    for W, q, _ in views[:7]:
+        qq = hqq.hqq_quantize_ex(W, q.nbits, q.group, precision="fp16")
+        acc += int(qq.iters.long().sum())
+        n_half += int(qq.half.long().sum())
+        n_groups += qq.iters.numel()
+        del qq
+    params = sum(q.rows * q.cols for _, q, _ in views)
+    gbs = qbytes / (ms / 1e3) / 1e9
+    return {"what": "quantize pass with the half-precision solver (each element-wise step "
+                    "rounded to fp16, error and z as fp16 group means)",
+            "ms_per_pass": ms, "gparam_s": params / (ms / 1e3) / 1e9, "gbs": gbs,
+            "hbm_frac": gbs / hbm_peak,
+            "mean_accepted_iters_first7": acc / max(n_groups, 1),
+            "half_precision_group_frac_first7": n_half / max(n_groups, 1)}
 
 
 def run_rtn(views, hqq, dev, hbm_peak, qbytes, pg):
@@ -907,6 +1080,8 @@ def main():
     ap.add_argument("--no-meta", action="store_true", help="skip the 8-bit meta-data timing")
     ap.add_argument("--no-linear", action="store_true", help="skip the linear-layer timing")
     ap.add_argument("--no-lowrank", action="store_true", help="skip the low-rank residual timing")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-matrix timings of the other workloads")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every library call from Python each pass instead of replaying "
                          "CUDA graphs of the passes")
