@@ -137,6 +137,16 @@ __device__ __forceinline__ void load_lane_minmax(const __half* src, float2 (&w)[
     mx = fmaxf(__low2float(hmx), __high2float(hmx));
 }
 
+// Pairwise sum ((x0+x1)+(x2+x3)) + ((x4+x5)+(x6+x7)) of one block of 8 values
+// held as pairs (x_k, x_k+4).  The pair halves are read one by one with scalar
+// adds: packed f32x2 adds of these pairs were found, twice, to give error sums
+// one unit off the canonical order in some groups on this toolchain, so no
+// packed add is used for a reduction.
+__device__ __forceinline__ float block_sum8(const float2 (&v)[4]) {
+    return __fadd_rn(__fadd_rn(__fadd_rn(v[0].x, v[1].x), __fadd_rn(v[2].x, v[3].x)),
+                     __fadd_rn(__fadd_rn(v[0].y, v[1].y), __fadd_rn(v[2].y, v[3].y)));
+}
+
 // Per-group constants of one evaluation, as f32x2 pairs.
 struct EvalConst {
     float2 z, nz, ns, inv, ninv;
@@ -184,15 +194,7 @@ __device__ __forceinline__ float2 eval_lane(const SM& S, const float2 (&w)[NB][4
                 T[k] = __ffma2_rn(w[b][k], c.ninv, q);                 // Wq - W/s
             }
         }
-        // ((x0+x1)+(x2+x3)) + ((x4+x5)+(x6+x7)) with pairs (x_k, x_k+4).  The
-        // reduction reads the pair halves one by one with scalar adds: a packed
-        // f32x2 add fed by the packed power results was found to combine the
-        // halves in the wrong order on this toolchain (the sums came out as if
-        // the pairs held adjacent weights), so no packed add is used here.
-        const float bp = __fadd_rn(__fadd_rn(__fadd_rn(P[0].x, P[1].x), __fadd_rn(P[2].x, P[3].x)),
-                                   __fadd_rn(__fadd_rn(P[0].y, P[1].y), __fadd_rn(P[2].y, P[3].y)));
-        const float bt = __fadd_rn(__fadd_rn(__fadd_rn(T[0].x, T[1].x), __fadd_rn(T[2].x, T[3].x)),
-                                   __fadd_rn(__fadd_rn(T[0].y, T[1].y), __fadd_rn(T[2].y, T[3].y)));
+        const float bp = block_sum8(P), bt = block_sum8(T);
         if (b == 0) {
             pe = bp;
             pt = bt;
@@ -314,10 +316,7 @@ __device__ __forceinline__ float2 eval_lane16(const SM& S, const float2 (&w)[NB]
                 ab = ab || fabsf(d32.x) > thr16 || fabsf(d32.y) > thr16;
             }
         }
-        const float bp = __fadd_rn(__fadd_rn(__fadd_rn(P[0].x, P[1].x), __fadd_rn(P[2].x, P[3].x)),
-                                   __fadd_rn(__fadd_rn(P[0].y, P[1].y), __fadd_rn(P[2].y, P[3].y)));
-        const float bt = __fadd_rn(__fadd_rn(__fadd_rn(T[0].x, T[1].x), __fadd_rn(T[2].x, T[3].x)),
-                                   __fadd_rn(__fadd_rn(T[0].y, T[1].y), __fadd_rn(T[2].y, T[3].y)));
+        const float bp = block_sum8(P), bt = block_sum8(T);
         if (b == 0) {
             pe = bp;
             pt = bt;
@@ -550,6 +549,58 @@ __device__ __forceinline__ void finalize_direct(const QuantParams& prm, const fl
     }
 }
 
+// Codes of one round of the final pass (the lane's NB blocks): 8, 4, 2 and 1
+// bit codes to HBM, 3 bit code bytes to the chunk's code buffer (zero for a
+// carried group, whose codes are OR-ed in later).  CLAMP: codes may leave
+// [0, L].  A code is the low byte of W/s + z_best + 1.5 * 2^23.
+template <int NBITS, int G, int NB, bool HALF, bool CLAMP>
+__device__ __forceinline__ void final_codes(const QuantParams& prm, uint8_t* codes,
+                                            const float2 (&w)[NB][4], const GroupState& g,
+                                            int64_t chunk, int gl, int kl, bool valid, bool mine) {
+    constexpr float L = (float)((1 << NBITS) - 1);
+    const float2 inv2 = make_float2(g.inv, g.inv), zb2 = make_float2(g.zb, g.zb);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        uint32_t t[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float2 v = final_v<HALF>(w[b][k], inv2, zb2, g.h);
+            if (CLAMP) {
+                v.x = fminf(fmaxf(v.x, 0.0f), L);
+                v.y = fminf(fmaxf(v.y, 0.0f), L);
+            }
+            const float2 r = __fadd2_rn(v, make_float2(kRoundShift, kRoundShift));
+            t[k] = __float_as_uint(r.x);
+            t[k + 4] = __float_as_uint(r.y);
+        }
+        if (!valid || (!mine && NBITS != 3)) continue;
+        const int64_t unit = chunk * (kChunk / 8) + (int64_t)gl * (G / 8) + kl * NB + b;
+        if constexpr (NBITS == 8 || NBITS == 3) {
+            // the eight low bytes in order, two byte permutes per word
+            uint2 bb;
+            bb.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040),
+                               0x5410);
+            bb.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040),
+                               0x5410);
+            if (NBITS == 3 && !mine) bb = make_uint2(0u, 0u);
+            if constexpr (NBITS == 8)
+                reinterpret_cast<uint2*>(prm.packed)[unit] = bb;
+            else
+                *reinterpret_cast<uint2*>(codes + gl * G + (kl * NB + b) * 8) = bb;
+        } else {
+            uint32_t word = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) word |= (t[i] & 0xFFu) << (NBITS * i);
+            if constexpr (NBITS == 4)
+                reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
+            else if constexpr (NBITS == 2)
+                reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)word;
+            else
+                prm.packed[unit] = (uint8_t)word;
+        }
+    }
+}
+
 // Final codes of every group of a chunk (one uniform pass, phase-A layout),
 // from the staged weights and each group's (z_best, 1/s); 8, 4, 2 and 1 bit
 // codes are stored straight to HBM, 3 bit code bytes overwrite the front of the
@@ -584,48 +635,24 @@ __device__ __forceinline__ void final_pass(const QuantParams& prm, __half* s_w, 
             g.h = false;
         }
         if constexpr (NBITS == 3) __syncwarp();     // all reads of the round before any write
-        const float2 inv2 = make_float2(g.inv, g.inv), zb2 = make_float2(g.zb, g.zb);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            uint32_t c[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float2 v = final_v<HALF>(w[b][k], inv2, zb2, g.h);
-                v.x = fminf(fmaxf(v.x, 0.0f), L);
-                v.y = fminf(fmaxf(v.y, 0.0f), L);
-                const float2 t = __fadd2_rn(v, make_float2(kRoundShift, kRoundShift));
-                c[k] = mine ? __float_as_uint(t.x) & 0xFFu : 0u;
-                c[k + 4] = mine ? __float_as_uint(t.y) & 0xFFu : 0u;
-            }
-            if (!valid || (!mine && NBITS != 3)) continue;
-            const int64_t unit = chunk * (kChunk / 8) + gl * (G / 8) + kl * NB + b;
-            if constexpr (NBITS == 4) {
-                uint32_t word = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) word |= c[i] << (4 * i);
-                reinterpret_cast<uint32_t*>(prm.packed)[unit] = word;
-            } else if constexpr (NBITS == 2) {
-                uint32_t h = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) h |= c[i] << (2 * i);
-                reinterpret_cast<uint16_t*>(prm.packed)[unit] = (uint16_t)h;
-            } else if constexpr (NBITS == 1) {
-                uint32_t h = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) h |= c[i] << i;
-                prm.packed[unit] = (uint8_t)h;
-            } else if constexpr (NBITS == 8) {
-                uint2 bb;
-                bb.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-                bb.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-                reinterpret_cast<uint2*>(prm.packed)[unit] = bb;
+        // codes need no clamp when every group of the warp has its extreme
+        // weights (hence, by monotonicity, all weights) inside [-1/2, L + 1/2)
+        bool inside = true;
+        if (valid && mine) {
+            float vmin, vmax;
+            if (HALF && g.h) {
+                vmin = r16(__fadd_rn(r16(__fmul_rn(g.mn, g.inv)), g.zb));
+                vmax = r16(__fadd_rn(r16(__fmul_rn(g.mx, g.inv)), g.zb));
             } else {
-                uint2 bb;
-                bb.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-                bb.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-                *reinterpret_cast<uint2*>(codes + gl * G + (kl * NB + b) * 8) = bb;
+                vmin = __fmaf_rn(g.mn, g.inv, g.zb);
+                vmax = __fmaf_rn(g.mx, g.inv, g.zb);
             }
+            inside = vmin >= -0.5f && vmax < L + 0.5f;
         }
+        if (__all_sync(kFull, inside))
+            final_codes<NBITS, G, NB, HALF, false>(prm, codes, w, g, chunk, gl, kl, valid, mine);
+        else
+            final_codes<NBITS, G, NB, HALF, true>(prm, codes, w, g, chunk, gl, kl, valid, mine);
         if (mine && kl == 0) {
             const int64_t gi = chunk * C::CG + gl;
             prm.scale[gi] = __float2half_rn(g.s);
