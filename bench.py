@@ -697,13 +697,14 @@ def run_meta8(args, views, hqq, dev, hbm_peak, pg):
                        torch.empty(ng, dtype=torch.float16, device=dev), 128)
         metas.append((zq, sq))
 
+    # every matrix's zero points (one group) and scales (groups of 128): one
+    # batched call per pass
+    tensors = [(q.zero.view(-1), 0) for _, q, _ in views] + \
+        [(q.scale.view(-1), 128) for _, q, _ in views]
+    outs = [zq for zq, _ in metas] + [sq for _, sq in metas]
+
     def meta_all():
-        for k, (W, q, O) in enumerate(views):
-            zq, sq = metas[k]
-            hqq.hqq_meta_quantize(q.zero.view(-1), 0, codes=zq.codes, scale=zq.scale,
-                                  zero=zq.zero)
-            hqq.hqq_meta_quantize(q.scale.view(-1), 128, codes=sq.codes, scale=sq.scale,
-                                  zero=sq.zero)
+        hqq.hqq_meta_quantize_batch(tensors, outputs=outs)
 
     def dq_all():
         for k, (W, q, O) in enumerate(views):
@@ -752,7 +753,9 @@ def run_meta8(args, views, hqq, dev, hbm_peak, pg):
     return {"what": "zero points 8-bit (one group per matrix), scales 8-bit (groups of 128); "
                     "weights dequantized in one pass from that form",
             "meta_quantize": {"ms_per_pass": mq_ms, "gbs": mq_gbs, "hbm_frac": mq_gbs / hbm_peak,
-                              "launches_per_pass": 2 * len(views)},
+                              "tensors_per_pass": 2 * len(views),
+                              "launches_per_pass": 2 * -(-len(views) // 128),
+                              "api": "hqq_meta_quantize_batch (all tensors in one call)"},
             "dequantize_meta": {"ms_per_pass": dq_ms, "gbs": dq_gbs,
                                 "hbm_frac": dq_gbs / hbm_peak,
                                 "gparam_s": params / (dq_ms / 1e3) / 1e9,

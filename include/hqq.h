@@ -207,6 +207,32 @@ int64_t hqq_meta_groups(int64_t n, int64_t mgroup);
 int hqq_meta_quantize(const void* x, int64_t n, int64_t mgroup, uint8_t* codes,
                       void* scale, void* zero, void* stream);
 
+/* One meta tensor of a batch: the arguments of hqq_meta_quantize. */
+typedef struct hqq_meta_job {
+    const void* x;          /* fp16 [n], 16-byte aligned                    */
+    int64_t n;              /* values (>= 0; 0 is skipped)                  */
+    int64_t mgroup;         /* 0 or a power of two up to 2^30               */
+    uint8_t* codes;         /* uint8 [n], 8-byte aligned                    */
+    void* scale;            /* fp16 [hqq_meta_groups(n, mgroup)]            */
+    void* zero;             /* fp16 [hqq_meta_groups(n, mgroup)]            */
+} hqq_meta_job;
+
+/*
+ * hqq_meta_quantize_batch -- hqq_meta_quantize of `count` meta tensors at once
+ * (say every zero-point and scale tensor of a layer or of a whole model),
+ * with the same results, bit for bit, as one call per tensor.  The tensors
+ * share launches: each one-group tensor is reduced by a cluster of thread
+ * blocks of its own and the grouped tensors split one grid, up to 128 tensors
+ * per launch, so that a batch of small tensors occupies the whole GPU.
+ *   jobs   [in] HOST array of `count` descriptors (device pointers inside);
+ *              it may be freed when the call returns.
+ *   count  [in] >= 0 (0: no-op).
+ * Every descriptor is validated first (errors as for hqq_meta_quantize); on
+ * any error nothing is launched.  Tensors of one batch must not overlap each
+ * other's outputs.
+ */
+int hqq_meta_quantize_batch(const hqq_meta_job* jobs, int64_t count, void* stream);
+
 /*
  * hqq_meta_dequantize -- the inverse: out = fp16((c - z) * s) per value.
  *   codes [in] uint8 [n], 8-byte aligned.   scale, zero [in] fp16, 2-byte aligned.

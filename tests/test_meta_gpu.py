@@ -165,3 +165,42 @@ def test_meta_bad_arguments(hqq):
         hqq.hqq_dequantize_meta(torch.zeros(32, dtype=torch.uint8, device="cuda"), m, 1, 64, 4,
                                 64, scale=torch.zeros(1, dtype=torch.float16, device="cuda"),
                                 scale_q=m)
+
+
+def test_meta_quantize_batch_matches_oracle_and_single_calls(hqq):
+    """One batch of whole-tensor and grouped meta tensors (ragged, tiny, empty,
+    more than one launch's worth) equals the oracle and the per-tensor calls
+    bit for bit."""
+    rng = np.random.default_rng(31)
+    specs = []
+    for i in range(150):                      # > 128 tensors: several launches
+        n = int(rng.choice([0, 1, 7, 100, 1000, 4099, 70001, 262144]))
+        mg = int(rng.choice([0, 0, 1, 8, 128, 256, 1 << 20]))
+        specs.append((n, mg))
+    xs = []
+    for i, (n, mg) in enumerate(specs):
+        x = (rng.standard_normal(n) * (1 + i % 5) + i % 3).astype(np.float16)
+        xs.append(x)
+    dev = [torch.from_numpy(x).cuda() for x in xs]
+    got = hqq.hqq_meta_quantize_batch([(d, mg) for d, (n, mg) in zip(dev, specs)])
+    single = [hqq.hqq_meta_quantize(d, mg) if d.numel() else None
+              for d, (n, mg) in zip(dev, specs)]
+    torch.cuda.synchronize()
+    for x, (n, mg), m, one in zip(xs, specs, got, single):
+        ref = oracle.meta_quantize(x, mg)
+        assert np.array_equal(m.codes.cpu().numpy(), ref["codes"]), (n, mg)
+        assert np.array_equal(m.scale.cpu().numpy().view(np.uint16), ref["scale"].view(np.uint16))
+        assert np.array_equal(m.zero.cpu().numpy().view(np.uint16), ref["zero"].view(np.uint16))
+        if one is not None:
+            assert torch.equal(one.codes, m.codes) and torch.equal(one.zero, m.zero)
+
+
+def test_meta_quantize_batch_bad_job_launches_nothing(hqq):
+    x = torch.zeros(64, dtype=torch.float16, device="cuda")
+    good = hqq.Meta8(torch.full((64,), 7, dtype=torch.uint8, device="cuda"),
+                     torch.zeros(1, dtype=torch.float16, device="cuda"),
+                     torch.zeros(1, dtype=torch.float16, device="cuda"), 0)
+    with pytest.raises(hqq.HQQError):
+        hqq.hqq_meta_quantize_batch([(x, 0), (x, 3)], outputs=[good, good])   # 3: not 2^k
+    torch.cuda.synchronize()
+    assert torch.all(good.codes == 7)

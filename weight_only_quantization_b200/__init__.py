@@ -14,7 +14,8 @@ from dataclasses import dataclass
 
 __all__ = ["HQQError", "hqq_quantize", "hqq_quantize_ex", "hqq_quantize_half", "hqq_dequantize",
            "hqq_packed_bytes", "hqq_status_string", "QuantizedMatrix", "LIB_PATH",
-           "Meta8", "hqq_meta_groups", "hqq_meta_quantize", "hqq_meta_dequantize",
+           "Meta8", "hqq_meta_groups", "hqq_meta_quantize", "hqq_meta_quantize_batch",
+           "hqq_meta_dequantize",
            "hqq_dequantize_meta", "hqq_linear", "hqq_linear_meta",
            "DEFAULT_P", "DEFAULT_BETA", "DEFAULT_KAPPA", "DEFAULT_ITERS"]
 
@@ -56,6 +57,14 @@ class _CMeta8(ctypes.Structure):
     _fields_ = [("codes", _P), ("scale", _P), ("zero", _P), ("group", _I64)]
 
 
+class _CMetaJob(ctypes.Structure):
+    """struct hqq_meta_job of include/hqq.h."""
+    _fields_ = [("x", _P), ("n", _I64), ("mgroup", _I64), ("codes", _P), ("scale", _P),
+                ("zero", _P)]
+
+
+_lib.hqq_meta_quantize_batch.argtypes = [ctypes.POINTER(_CMetaJob), _I64, _P]
+_lib.hqq_meta_quantize_batch.restype = _I
 _lib.hqq_dequantize_meta.argtypes = [_P, ctypes.POINTER(_CMeta8), _P, ctypes.POINTER(_CMeta8),
                                      _I64, _I64, _I, _I, _P, _P]
 _lib.hqq_dequantize_meta.restype = _I
@@ -264,6 +273,34 @@ def hqq_meta_quantize(x, mgroup: int = 0, codes=None, scale=None, zero=None,
     _check(_lib.hqq_meta_quantize(_ptr(x), n, mgroup, _ptr(codes), _ptr(scale), _ptr(zero),
                                   _stream(stream)))
     return Meta8(codes, scale, zero, mgroup)
+
+
+def hqq_meta_quantize_batch(tensors, stream=None, outputs=None) -> list:
+    """hqq_meta_quantize of many fp16 meta tensors in shared launches.
+    ``tensors`` is a list of (x, mgroup); ``outputs`` optionally a list of
+    Meta8 to write into (same order).  Returns the list of Meta8."""
+    import torch
+    out = []
+    jobs = (_CMetaJob * max(len(tensors), 1))()
+    for i, (x, mgroup) in enumerate(tensors):
+        if x.dtype != torch.float16:
+            raise ValueError("x must be float16")
+        _check_tensor(x, "x")
+        n = x.numel()
+        if outputs is not None:
+            m = outputs[i]
+        else:
+            ng = hqq_meta_groups(n, mgroup)
+            m = Meta8(torch.empty(n, dtype=torch.uint8, device=x.device),
+                      torch.empty(ng, dtype=torch.float16, device=x.device),
+                      torch.empty(ng, dtype=torch.float16, device=x.device), mgroup)
+        for t, nm in ((m.codes, "codes"), (m.scale, "scale"), (m.zero, "zero")):
+            _check_tensor(t, nm)
+        jobs[i] = _CMetaJob(x.data_ptr(), n, mgroup, m.codes.data_ptr(), m.scale.data_ptr(),
+                            m.zero.data_ptr())
+        out.append(m)
+    _check(_lib.hqq_meta_quantize_batch(jobs, len(tensors), _stream(stream)))
+    return out
 
 
 def hqq_meta_dequantize(m: Meta8, out=None, stream=None):

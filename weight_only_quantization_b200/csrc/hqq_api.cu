@@ -3,6 +3,7 @@
 // kernel dispatch.  Nothing is launched unless every check passes.
 #include <cmath>
 #include <cstring>
+#include <vector>
 
 #include "../../include/hqq.h"
 #include "hqq_params.cuh"
@@ -38,6 +39,7 @@ cudaError_t launch_meta_quantize(const __half* x, int64_t n, int log2g, uint8_t*
                                  __half* scale, __half* zero, cudaStream_t stream);
 cudaError_t launch_meta_dequantize(const uint8_t* codes, const __half* scale, const __half* zero,
                                    int64_t n, int log2g, __half* out, cudaStream_t stream);
+cudaError_t launch_meta_quantize_batch(const MetaJobIn* jobs, int64_t count, cudaStream_t stream);
 
 namespace {
 
@@ -294,6 +296,34 @@ extern "C" int hqq_meta_quantize(const void* x, int64_t n, int64_t mgroup, uint8
     const cudaError_t err = launch_meta_quantize(
         static_cast<const __half*>(x), n, lg, codes, static_cast<__half*>(scale),
         static_cast<__half*>(zero), static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
+extern "C" int hqq_meta_quantize_batch(const hqq_meta_job* jobs, int64_t count, void* stream) {
+    if (count < 0) return HQQ_ERR_SHAPE;
+    if (count == 0) return HQQ_OK;
+    if (!jobs) return HQQ_ERR_NULL;
+    for (int64_t i = 0; i < count; ++i) {          // every job checked before any launch
+        const hqq_meta_job& j = jobs[i];
+        if (j.n < 0 || j.mgroup < 0 || j.n > ((int64_t)1 << 40)) return HQQ_ERR_SHAPE;
+        if (meta_log2(j.mgroup) == -2) return HQQ_ERR_UNSUPPORTED;
+        if (j.n == 0) continue;
+        if (!j.x || !j.codes || !j.scale || !j.zero) return HQQ_ERR_NULL;
+        if (!aligned(j.x, 16) || !aligned(j.codes, 8) || !aligned(j.scale, 2) ||
+            !aligned(j.zero, 2))
+            return HQQ_ERR_ALIGN;
+    }
+    std::vector<MetaJobIn> in((size_t)count);
+    for (int64_t i = 0; i < count; ++i) {
+        in[i].x = static_cast<const __half*>(jobs[i].x);
+        in[i].n = jobs[i].n;
+        in[i].log2g = meta_log2(jobs[i].mgroup);
+        in[i].codes = jobs[i].codes;
+        in[i].scale = static_cast<__half*>(jobs[i].scale);
+        in[i].zero = static_cast<__half*>(jobs[i].zero);
+    }
+    const cudaError_t err =
+        launch_meta_quantize_batch(in.data(), count, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }
 

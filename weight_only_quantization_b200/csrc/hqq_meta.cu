@@ -80,18 +80,23 @@ __device__ __forceinline__ void minmax8(uint4 v, __half2& mn, __half2& mx) {
 }
 
 constexpr int kGroupThreads = 256;
+constexpr int kMetaBatchMax = 128;                    // jobs per batched launch
 
-__global__ void __launch_bounds__(kGroupThreads)
-meta_group_kernel(const __half* __restrict__ x, int64_t n, int log2g, int64_t ngroups,
-                  uint8_t* __restrict__ codes, __half* __restrict__ scale,
-                  __half* __restrict__ zero) {
+// Groups of 2^k values, one value per lane and step; `block` of `nblocks`
+// blocks working on this tensor.
+__device__ __forceinline__ void meta_group_body(const __half* __restrict__ x, int64_t n,
+                                                int log2g, int64_t ngroups,
+                                                uint8_t* __restrict__ codes,
+                                                __half* __restrict__ scale,
+                                                __half* __restrict__ zero, int64_t block,
+                                                int64_t nblocks) {
     const int lane = threadIdx.x & 31;
     const int lseg = log2g < 5 ? log2g : 5;          // log2(lanes per group)
     const int seg = 1 << lseg;
     const int per_warp = 32 >> lseg;                  // groups per warp step
     const int64_t gs = (int64_t)1 << log2g;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t warp = (block * kGroupThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (nblocks * kGroupThreads) >> 5;
     const int k0 = lane & (seg - 1);
     for (int64_t gb = warp * per_warp; gb < ngroups; gb += nwarps * per_warp) {
         const int64_t gi = gb + (lane >> lseg);
@@ -123,17 +128,19 @@ meta_group_kernel(const __half* __restrict__ x, int64_t n, int log2g, int64_t ng
 // Groups of 2^k >= 8 values: each lane takes 16-byte vectors (8 values), a
 // segment of min(2^k/8, 32) lanes per group.  The vector that holds the end of
 // a ragged last group is read value by value.
-__global__ void __launch_bounds__(kGroupThreads)
-meta_group_vec_kernel(const __half* __restrict__ x, int64_t n, int log2g, int64_t ngroups,
-                      uint8_t* __restrict__ codes, __half* __restrict__ scale,
-                      __half* __restrict__ zero) {
+__device__ __forceinline__ void meta_group_vec_body(const __half* __restrict__ x, int64_t n,
+                                                    int log2g, int64_t ngroups,
+                                                    uint8_t* __restrict__ codes,
+                                                    __half* __restrict__ scale,
+                                                    __half* __restrict__ zero, int64_t block,
+                                                    int64_t nblocks) {
     const int lane = threadIdx.x & 31;
     const int lv = log2g - 3;                         // log2(vectors per group)
     const int lseg = lv < 5 ? lv : 5;
     const int seg = 1 << lseg;
     const int per_warp = 32 >> lseg;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t warp = (block * kGroupThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (nblocks * kGroupThreads) >> 5;
     const int k0 = lane & (seg - 1);
     const uint4* xv = reinterpret_cast<const uint4*>(x);
     const int64_t nfull = n >> 3;                     // vectors entirely inside x
@@ -179,12 +186,28 @@ meta_group_vec_kernel(const __half* __restrict__ x, int64_t n, int log2g, int64_
     }
 }
 
+__global__ void __launch_bounds__(kGroupThreads)
+meta_group_kernel(const __half* __restrict__ x, int64_t n, int log2g, int64_t ngroups,
+                  uint8_t* __restrict__ codes, __half* __restrict__ scale,
+                  __half* __restrict__ zero) {
+    meta_group_body(x, n, log2g, ngroups, codes, scale, zero, blockIdx.x, gridDim.x);
+}
+
+__global__ void __launch_bounds__(kGroupThreads)
+meta_group_vec_kernel(const __half* __restrict__ x, int64_t n, int log2g, int64_t ngroups,
+                      uint8_t* __restrict__ codes, __half* __restrict__ scale,
+                      __half* __restrict__ zero) {
+    meta_group_vec_body(x, n, log2g, ngroups, codes, scale, zero, blockIdx.x, gridDim.x);
+}
+
 constexpr int kWholeThreads = 1024;
 constexpr int kWholeBatch = 8;                        // 16-byte loads in flight per thread
 
-__global__ void __launch_bounds__(kWholeThreads)
-meta_whole_kernel(const __half* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
-                  __half* __restrict__ scale, __half* __restrict__ zero) {
+// One tensor reduced and quantized by the calling thread-block cluster.
+__device__ __forceinline__ void meta_whole_body(const __half* __restrict__ x, int64_t n,
+                                                uint8_t* __restrict__ codes,
+                                                __half* __restrict__ scale,
+                                                __half* __restrict__ zero) {
     cg::cluster_group cluster = cg::this_cluster();
     const int64_t rank = cluster.block_rank();
     const int64_t ncta = cluster.num_blocks();
@@ -274,6 +297,54 @@ meta_whole_kernel(const __half* __restrict__ x, int64_t n, uint8_t* __restrict__
     }
 }
 
+__global__ void __launch_bounds__(kWholeThreads)
+meta_whole_kernel(const __half* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
+                  __half* __restrict__ scale, __half* __restrict__ zero) {
+    meta_whole_body(x, n, codes, scale, zero);
+}
+
+// ---- batches: many meta tensors per launch ----------------------------------
+// Whole-tensor jobs: cluster c of the grid takes job c.  Grouped jobs: job j owns
+// blocks [first[j], first[j+1]) of the grid.
+struct MetaJob {
+    const __half* x;
+    int64_t n;
+    uint8_t* codes;
+    __half* scale;
+    __half* zero;
+    int64_t ngroups;
+    int log2g;
+};
+
+struct MetaBatch {
+    int count;
+    int first[kMetaBatchMax + 1];
+    MetaJob job[kMetaBatchMax];
+};
+
+__global__ void __launch_bounds__(kWholeThreads)
+meta_whole_batch_kernel(const __grid_constant__ MetaBatch b) {
+    const MetaJob& j = b.job[blockIdx.x / cg::this_cluster().num_blocks()];
+    meta_whole_body(j.x, j.n, j.codes, j.scale, j.zero);
+}
+
+__global__ void __launch_bounds__(kGroupThreads)
+meta_group_batch_kernel(const __grid_constant__ MetaBatch b) {
+    int lo = 0, hi = b.count - 1;                     // the job whose block range holds us
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (b.first[mid] <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+    }
+    const MetaJob& j = b.job[lo];
+    const int64_t block = (int64_t)blockIdx.x - b.first[lo];
+    const int64_t nblocks = b.first[lo + 1] - b.first[lo];
+    if (j.log2g >= 3)
+        meta_group_vec_body(j.x, j.n, j.log2g, j.ngroups, j.codes, j.scale, j.zero, block,
+                            nblocks);
+    else
+        meta_group_body(j.x, j.n, j.log2g, j.ngroups, j.codes, j.scale, j.zero, block, nblocks);
+}
+
 constexpr int kMdqThreads = 256;
 
 __device__ __forceinline__ uint32_t restore2(uint32_t c01, float z0, float s0, float z1, float s1) {
@@ -323,11 +394,12 @@ int sm_count() {
 
 // Cluster size of the whole-tensor kernel: 16 CTAs where the device can place
 // such a cluster (non-portable size), else the portable 8.
-int whole_cluster_size() {
+template <class Kern>
+int whole_cluster_size(Kern kern) {
     static thread_local int cached = 0;
     if (cached) return cached;
     int best = 8;
-    if (cudaFuncSetAttribute(meta_whole_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed,
                              1) == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr;
@@ -340,7 +412,7 @@ int whole_cluster_size() {
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, meta_whole_kernel, &cfg) == cudaSuccess &&
+        if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess &&
             clusters > 0)
             best = 16;
     }
@@ -357,7 +429,7 @@ cudaError_t launch_meta_quantize(const __half* x, int64_t n, int log2g, uint8_t*
     int lg = log2g;
     const int64_t ngroups = lg < 0 ? 1 : (n + ((int64_t)1 << lg) - 1) >> lg;
     if (ngroups == 1 && n > 4096) {
-        const int cl = whole_cluster_size();
+        const int cl = whole_cluster_size(meta_whole_kernel);
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr;
         attr.id = cudaLaunchAttributeClusterDimension;
@@ -390,6 +462,84 @@ cudaError_t launch_meta_quantize(const __half* x, int64_t n, int log2g, uint8_t*
         meta_group_kernel<<<(unsigned)blocks, kGroupThreads, 0, stream>>>(x, n, lg, ngroups,
                                                                           codes, scale, zero);
     return cudaGetLastError();
+}
+
+// Many meta tensors: whole-tensor jobs (one group) as one cluster each, grouped
+// jobs as block ranges of one grid, at most kMetaBatchMax jobs per launch.
+cudaError_t launch_meta_quantize_batch(const MetaJobIn* jobs, int64_t count,
+                                       cudaStream_t stream) {
+    const int64_t cap = (int64_t)sm_count() * 16;
+    MetaBatch whole, grouped;
+    whole.count = grouped.count = 0;
+    whole.first[0] = grouped.first[0] = 0;
+    auto flush_whole = [&]() -> cudaError_t {
+        if (whole.count == 0) return cudaSuccess;
+        const int cl = whole_cluster_size(meta_whole_batch_kernel);
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = cl;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)(whole.count * cl));
+        cfg.blockDim = dim3(kWholeThreads);
+        cfg.stream = stream;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, meta_whole_batch_kernel, whole);
+        whole.count = 0;
+        return e;
+    };
+    auto flush_grouped = [&]() -> cudaError_t {
+        if (grouped.count == 0) return cudaSuccess;
+        meta_group_batch_kernel<<<(unsigned)grouped.first[grouped.count], kGroupThreads, 0,
+                                  stream>>>(grouped);
+        grouped.count = 0;
+        grouped.first[0] = 0;
+        return cudaGetLastError();
+    };
+    for (int64_t i = 0; i < count; ++i) {
+        const MetaJobIn& in = jobs[i];
+        if (in.n == 0) continue;
+        int lg = in.log2g;
+        const int64_t ngroups = lg < 0 ? 1 : (in.n + ((int64_t)1 << lg) - 1) >> lg;
+        MetaJob j;
+        j.x = in.x;
+        j.n = in.n;
+        j.codes = in.codes;
+        j.scale = in.scale;
+        j.zero = in.zero;
+        j.ngroups = ngroups;
+        j.log2g = lg;
+        if (ngroups == 1) {
+            whole.job[whole.count++] = j;
+            if (whole.count == kMetaBatchMax) {
+                const cudaError_t e = flush_whole();
+                if (e != cudaSuccess) return e;
+            }
+            continue;
+        }
+        const bool vec = lg >= 3;
+        const int lanes_log = vec ? lg - 3 : lg;
+        const int lseg = lanes_log < 5 ? lanes_log : 5;
+        const int64_t warps = (ngroups + (32 >> lseg) - 1) / (32 >> lseg);
+        int64_t blocks = (warps + kGroupThreads / 32 - 1) / (kGroupThreads / 32);
+        if (blocks > cap) blocks = cap;
+        if ((int64_t)grouped.first[grouped.count] + blocks > ((int64_t)1 << 30)) {
+            const cudaError_t e = flush_grouped();
+            if (e != cudaSuccess) return e;
+        }
+        grouped.job[grouped.count] = j;
+        grouped.first[grouped.count + 1] = grouped.first[grouped.count] + (int)blocks;
+        ++grouped.count;
+        if (grouped.count == kMetaBatchMax) {
+            const cudaError_t e = flush_grouped();
+            if (e != cudaSuccess) return e;
+        }
+    }
+    cudaError_t e = flush_whole();
+    if (e != cudaSuccess) return e;
+    return flush_grouped();
 }
 
 cudaError_t launch_meta_dequantize(const uint8_t* codes, const __half* scale, const __half* zero,

@@ -33,6 +33,16 @@ struct LinearParams {
     Meta8 zq, sq;            // 8-bit zero points / scales (codes NULL: use zero / scale)
 };
 
+// One meta tensor of a batch (validated on the host): log2g < 0 for one group.
+struct MetaJobIn {
+    const __half* x;
+    int64_t n;
+    int log2g;
+    uint8_t* codes;
+    __half* scale;
+    __half* zero;
+};
+
 struct DequantParams {
     const uint8_t* packed;
     const __half* scale;   // fp16 scales, unless given in 8-bit form (sq)
