@@ -52,21 +52,35 @@ __device__ __forceinline__ MetaAffine meta_affine(float mn, float mx) {
     return a;
 }
 
+// clamp(round(x (1/s) + z), 0, 255), half to even: clamping to the integers 0
+// and 255 first gives the same code, and adding 1.5 * 2^23 then rounds to an
+// integer held in the low mantissa bits (no conversion instructions).
+constexpr float kMetaShift = 12582912.0f;   // 1.5 * 2^23
+
 __device__ __forceinline__ uint32_t meta_code(float x, const MetaAffine& a) {
-    return (uint32_t)fminf(fmaxf(rintf(__fmaf_rn(x, a.inv, a.z)), 0.0f), kMetaL);
+    const float v = fminf(fmaxf(__fmaf_rn(x, a.inv, a.z), 0.0f), kMetaL);
+    return __float_as_uint(__fadd_rn(v, kMetaShift)) & 0xFFu;
 }
 
 // Eight consecutive values -> eight codes, first code in the low byte.
 __device__ __forceinline__ uint2 meta_codes8(uint4 v, const MetaAffine& a) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t c[2] = {0u, 0u};
+    const float2 inv2 = make_float2(a.inv, a.inv), z2 = make_float2(a.z, a.z);
+    const float2 sh2 = make_float2(kMetaShift, kMetaShift);
+    uint32_t t[8];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const __half2 h = *reinterpret_cast<const __half2*>(&w[j]);
-        const float2 f = __half22float2(h);
-        c[j >> 1] |= (meta_code(f.x, a) | (meta_code(f.y, a) << 8)) << (16 * (j & 1));
+        float2 f = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&w[j])), inv2, z2);
+        f.x = fminf(fmaxf(f.x, 0.0f), kMetaL);
+        f.y = fminf(fmaxf(f.y, 0.0f), kMetaL);
+        f = __fadd2_rn(f, sh2);
+        t[2 * j] = __float_as_uint(f.x);
+        t[2 * j + 1] = __float_as_uint(f.y);
     }
-    return make_uint2(c[0], c[1]);
+    // the low byte of each sum, in order
+    return make_uint2(
+        __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410),
+        __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410));
 }
 
 __device__ __forceinline__ void minmax8(uint4 v, __half2& mn, __half2& mx) {
@@ -200,7 +214,7 @@ meta_group_vec_kernel(const __half* __restrict__ x, int64_t n, int log2g, int64_
     meta_group_vec_body(x, n, log2g, ngroups, codes, scale, zero, blockIdx.x, gridDim.x);
 }
 
-constexpr int kWholeThreads = 1024;
+constexpr int kWholeThreads = 512;
 constexpr int kWholeBatch = 8;                        // 16-byte loads in flight per thread
 
 // One tensor reduced and quantized by the calling thread-block cluster.
@@ -251,8 +265,9 @@ __device__ __forceinline__ void meta_whole_body(const __half* __restrict__ x, in
     }
     __syncthreads();
     if (warp == 0) {
-        mn = warp_mn[lane];
-        mx = warp_mx[lane];
+        constexpr int kWarps = kWholeThreads / 32;
+        mn = lane < kWarps ? warp_mn[lane] : INFINITY;
+        mx = lane < kWarps ? warp_mx[lane] : -INFINITY;
         for (int o = 16; o > 0; o >>= 1) {
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -297,7 +312,7 @@ __device__ __forceinline__ void meta_whole_body(const __half* __restrict__ x, in
     }
 }
 
-__global__ void __launch_bounds__(kWholeThreads)
+__global__ void __launch_bounds__(kWholeThreads, 2)
 meta_whole_kernel(const __half* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
                   __half* __restrict__ scale, __half* __restrict__ zero) {
     meta_whole_body(x, n, codes, scale, zero);
@@ -322,7 +337,7 @@ struct MetaBatch {
     MetaJob job[kMetaBatchMax];
 };
 
-__global__ void __launch_bounds__(kWholeThreads)
+__global__ void __launch_bounds__(kWholeThreads, 2)
 meta_whole_batch_kernel(const __grid_constant__ MetaBatch b) {
     const MetaJob& j = b.job[blockIdx.x / cg::this_cluster().num_blocks()];
     meta_whole_body(j.x, j.n, j.codes, j.scale, j.zero);
