@@ -19,7 +19,7 @@
  *         implementation holding 1/s rather than s;
  *   - section 4.1: p = 0.7, beta = 1, kappa = 1.01, 20 iterations, stop early
  *         once the error stops improving.
- * Readings taken where the page is silent (all listed in the design notes):
+ * Readings taken where the page is silent:
  *   - min-max initialisation s = (max-min)/(2^b-1), z = -min * (1/s);
  *   - codes are clamped to [0, 2^b-1]; rounding is round-half-to-even;
  *   - early stopping is decided per group on the sum of |W - W_hat|^p (equal to
