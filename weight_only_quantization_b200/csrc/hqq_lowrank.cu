@@ -80,116 +80,189 @@ __device__ __forceinline__ void unit_delta(const UnitLoad& u, float (&d)[8]) {
     }
 }
 
+// Both products run on the tensor cores: mma.sync m16n8k8 with tf32 operands
+// and fp32 accumulation, each fp32 operand split into a tf32 high part and a
+// tf32 remainder, a b ~ ah bh + ah bl + al bh (the dropped al bl is below
+// 2^-22 of the product), so the products keep fp32 accuracy.  A CTA's 8 warps
+// take a 16-row block each and half of the L columns (L/16 blocks of 8).
+// Fragments of m16n8k8 (g = lane / 4, q = lane % 4): A (row-major 16 x 8)
+// a0 = (g, q), a1 = (g + 8, q), a2 = (g, q + 4), a3 = (g + 8, q + 4);
+// B (8 x 8) b0 = (k q, column g), b1 = (k q + 4, column g); D c0 = (g, 2q),
+// c1 = (g, 2q + 1), c2 = (g + 8, 2q), c3 = (g + 8, 2q + 1).
+__device__ __forceinline__ uint32_t tf32_of(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = tf32_of(x);
+    lo = tf32_of(__fsub_rn(x, __uint_as_float(hi)));
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// d += A B in split tf32 for one 16 x 8 block: A given as its four fp32
+// fragment values, B as the high and low tf32 parts of its two.
+__device__ __forceinline__ void mma3(float (&d)[4], const uint32_t (&ah)[4],
+                                     const uint32_t (&al)[4], uint32_t bh0, uint32_t bh1,
+                                     uint32_t bl0, uint32_t bl1) {
+    mma_tf32(d, al, bh0, bh1);
+    mma_tf32(d, ah, bl0, bl1);
+    mma_tf32(d, ah, bh0, bh1);
+}
+
+// Store 4 consecutive values of an operand tile as high and low tf32 parts.
+__device__ __forceinline__ void store_split4(uint32_t* hi, uint32_t* lo, float4 v) {
+    uint4 h, l;
+    split_tf32(v.x, h.x, l.x);
+    split_tf32(v.y, h.y, l.y);
+    split_tf32(v.z, h.z, l.z);
+    split_tf32(v.w, h.w, l.w);
+    *reinterpret_cast<uint4*>(hi) = h;
+    *reinterpret_cast<uint4*>(lo) = l;
+}
+
+// Shared memory of one product CTA: the dW tile (64 x 64, row stride AS) and
+// the other operand's tile split into high and low tf32 parts (64 x L, row
+// stride L + 8).
+constexpr int kLrTile = 64;                               // k (right) or rows (left) per step
+template <int L, int AS>
+constexpr int prod_smem() {
+    return (64 * AS + 2 * kLrTile * (L + 8)) * 4;
+}
+
 // Y[N, L] = dW[N, K] M[K, L] over the k-tiles of split blockIdx.y (out: Y, or
 // the split's partial block when gridDim.y > 1).  CTA: 64 rows x L, k-tiles
-// of 32; the dW tile is stored k-major with its rows rotated by 8 (k / 8)
-// (conflict-free stores of the four units of a row); thread t forms one unit
-// of the dW tile (row t/4, k 8(t%4)) and owns
-// RPT = L/16 consecutive rows x 4 columns of the result (two vector shared
-// loads per k for 4 RPT FMAs).  The next tile's loads are issued before the
-// current tile's FMAs.
+// of 64.  Thread t forms units u = t and t + 256 (row u/8, k 8(u%8)) into
+// As[row][k] (row stride 68 words: the fragment loads of a warp hit 32
+// distinct banks; lanes 4..7 of each 8 store their upper half first, so each
+// quarter-warp store covers 8 distinct 16-byte bank groups); the M tile is
+// stored split, [k][column].  Warp w: rows 16 (w / 2) .. +15, column blocks
+// (w % 2) L/16 .. +L/16 - 1.  The next tile's loads are issued before the
+// current tile's MMAs.
 template <int NBITS, int L>
 __global__ void __launch_bounds__(kLrThreads)
 lr_right_kernel(const __grid_constant__ LrParams p, const float* __restrict__ M,
                 float* __restrict__ out, int64_t tiles_per_split) {
-    constexpr int RPT = L / 16, CG = L / 4, MV = 32 * L / 4;       // float4s of an M tile
-    __shared__ __align__(16) float As[32][64 + 4];                 // [k][row]
-    __shared__ __align__(16) float Bs[32][L];                      // [k][column]
-    const int t = threadIdx.x;
+    constexpr int NBW = L / 16, LP = L + 8, CG = L / 4, AS = 68;
+    constexpr int MV = kLrTile * L / 4, MVT = (MV + kLrThreads - 1) / kLrThreads;
+    extern __shared__ __align__(16) float lr_psm[];
+    auto As = reinterpret_cast<float(*)[AS]>(lr_psm);
+    auto Bh = reinterpret_cast<uint32_t(*)[LP]>(lr_psm + 64 * AS);
+    auto Bl = reinterpret_cast<uint32_t(*)[LP]>(lr_psm + 64 * AS + kLrTile * LP);
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, q = lane & 3;
+    const int rb = 16 * (warp >> 1), cb = (warp & 1) * NBW;
     const int64_t n0 = (int64_t)blockIdx.x * 64;
     const int64_t kt0 = (int64_t)blockIdx.y * tiles_per_split;
-    const int64_t ktiles = (p.K + 31) / 32;
+    const int64_t ktiles = (p.K + kLrTile - 1) / kLrTile;
     const int64_t kt1 = kt0 + tiles_per_split < ktiles ? kt0 + tiles_per_split : ktiles;
-    const int ur = t >> 2, uk = 8 * (t & 3);                       // this thread's unit
-    const int tr = (t / CG) * RPT, tc = 4 * (t % CG);              // this thread's outputs
-    const bool row_ok = n0 + ur < p.N;
-    float acc[RPT][4];
+    const int ur[2] = {t >> 3, (t >> 3) + 32}, uk = 8 * (t & 7);
+    const int hs = (t & 4) ? 4 : 0;                         // half stored first
+    float acc[NBW][4];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
-    auto load = [&](int64_t kt, UnitLoad& u, float4 (&mv)[(MV + kLrThreads - 1) / kLrThreads]) {
-        const int64_t k = kt * 32 + uk;
-        u = unit_load<NBITS>(p, (n0 + ur) * p.K + k, row_ok && k < p.K);
+    for (int i = 0; i < NBW; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+    auto load = [&](int64_t kt, UnitLoad (&u)[2], float4 (&mv)[MVT]) {
+        const int64_t k = kt * kLrTile + uk;
 #pragma unroll
-        for (int v = 0; v < (MV + kLrThreads - 1) / kLrThreads; ++v) {
+        for (int h = 0; h < 2; ++h)
+            u[h] = unit_load<NBITS>(p, (n0 + ur[h]) * p.K + k, n0 + ur[h] < p.N && k < p.K);
+#pragma unroll
+        for (int v = 0; v < MVT; ++v) {
             const int idx = t + v * kLrThreads;
             const int kk = idx / CG, c4 = idx % CG;
             mv[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (idx < MV && kt * 32 + kk < p.K)
-                mv[v] = __ldg(reinterpret_cast<const float4*>(M + (kt * 32 + kk) * L) + c4);
+            if (idx < MV && kt * kLrTile + kk < p.K)
+                mv[v] = __ldg(reinterpret_cast<const float4*>(M + (kt * kLrTile + kk) * L) + c4);
         }
     };
-    UnitLoad u;
-    float4 mv[(MV + kLrThreads - 1) / kLrThreads];
+    UnitLoad u[2];
+    float4 mv[MVT];
     if (kt0 < kt1) load(kt0, u, mv);
     for (int64_t kt = kt0; kt < kt1; ++kt) {
-        float d[8];
-        unit_delta<NBITS>(u, d);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) As[uk + i][(ur + uk) & 63] = d[i];   // rows rotated by 8 (k / 8)
+        for (int h = 0; h < 2; ++h) {
+            float d[8];
+            unit_delta<NBITS>(u[h], d);
+            const float4 lo = make_float4(d[0], d[1], d[2], d[3]), hi = make_float4(d[4], d[5], d[6], d[7]);
+            *reinterpret_cast<float4*>(&As[ur[h]][uk + hs]) = hs ? hi : lo;
+            *reinterpret_cast<float4*>(&As[ur[h]][uk + 4 - hs]) = hs ? lo : hi;
+        }
 #pragma unroll
-        for (int v = 0; v < (MV + kLrThreads - 1) / kLrThreads; ++v) {
+        for (int v = 0; v < MVT; ++v) {
             const int idx = t + v * kLrThreads;
-            if (idx < MV) *reinterpret_cast<float4*>(&Bs[idx / CG][4 * (idx % CG)]) = mv[v];
+            if (idx < MV) store_split4(&Bh[idx / CG][4 * (idx % CG)], &Bl[idx / CG][4 * (idx % CG)], mv[v]);
         }
         __syncthreads();
         if (kt + 1 < kt1) load(kt + 1, u, mv);
-#pragma unroll 8
-        for (int kk = 0; kk < 32; ++kk) {
-            const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tc]);
-            const int ar = (tr + (kk & ~7)) & 63;    // same rotation; RPT-groups stay whole
-            float a[RPT];
-            if constexpr (RPT == 4) {
-                const float4 a4 = *reinterpret_cast<const float4*>(&As[kk][ar]);
-                a[0] = a4.x; a[1] = a4.y; a[2] = a4.z; a[3] = a4.w;
-            } else if constexpr (RPT == 2) {
-                const float2 a2 = *reinterpret_cast<const float2*>(&As[kk][ar]);
-                a[0] = a2.x; a[1] = a2.y;
-            } else {
-                a[0] = As[kk][ar];
-            }
+#pragma unroll 4
+        for (int k8 = 0; k8 < kLrTile; k8 += 8) {
+            uint32_t ah[4], al[4];
+            split_tf32(As[rb + g][k8 + q], ah[0], al[0]);
+            split_tf32(As[rb + g + 8][k8 + q], ah[1], al[1]);
+            split_tf32(As[rb + g][k8 + q + 4], ah[2], al[2]);
+            split_tf32(As[rb + g + 8][k8 + q + 4], ah[3], al[3]);
 #pragma unroll
-            for (int i = 0; i < RPT; ++i) {
-                acc[i][0] = __fmaf_rn(a[i], b.x, acc[i][0]);
-                acc[i][1] = __fmaf_rn(a[i], b.y, acc[i][1]);
-                acc[i][2] = __fmaf_rn(a[i], b.z, acc[i][2]);
-                acc[i][3] = __fmaf_rn(a[i], b.w, acc[i][3]);
+            for (int i = 0; i < NBW; ++i) {
+                const int c = 8 * (cb + i) + g;
+                mma3(acc[i], ah, al, Bh[k8 + q][c], Bh[k8 + q + 4][c], Bl[k8 + q][c],
+                     Bl[k8 + q + 4][c]);
             }
         }
         __syncthreads();
     }
     float* o = out + (int64_t)blockIdx.y * p.N * L;
 #pragma unroll
-    for (int i = 0; i < RPT; ++i)
-        if (n0 + tr + i < p.N)
-            *reinterpret_cast<float4*>(o + (n0 + tr + i) * L + tc) =
-                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    for (int i = 0; i < NBW; ++i) {
+        const int c = 8 * (cb + i) + 2 * q;
+        const int64_t r0 = n0 + rb + g, r1 = r0 + 8;
+        if (r0 < p.N) *reinterpret_cast<float2*>(o + r0 * L + c) = make_float2(acc[i][0], acc[i][1]);
+        if (r1 < p.N) *reinterpret_cast<float2*>(o + r1 * L + c) = make_float2(acc[i][2], acc[i][3]);
+    }
 }
 
 // Z[K, L] = dW^T Y over the rows of split blockIdx.y (out: Z, or the split's
-// partial block).  CTA: 64 columns k x L, rows in tiles of 32; thread t forms
-// one unit (row t/8, k 8(t%8)) and owns RPT = L/16 consecutive k x 4 columns.
+// partial block).  CTA: 64 columns k x L, rows in tiles of 64.  Thread t forms
+// units u = t and t + 256 (row u/8, k 8(u%8)) into As[row][k] (stride 72
+// words, upper half first on lanes 4..7 as above); the Y tile is stored split,
+// [row][column].  Warp w: k 16 (w / 2) .. +15 (the rows of dW^T), column
+// blocks as above.
 template <int NBITS, int L>
 __global__ void __launch_bounds__(kLrThreads)
 lr_left_kernel(const __grid_constant__ LrParams p, const float* __restrict__ Y,
                float* __restrict__ out, int64_t rows_per_split) {
-    constexpr int RPT = L / 16, CG = L / 4, YV = 32 * L / 4;
-    __shared__ __align__(16) float As[32][64 + 4];                 // [row][k]
-    __shared__ __align__(16) float Bs[32][L];                      // [row][column]
-    const int t = threadIdx.x;
+    constexpr int NBW = L / 16, LP = L + 8, CG = L / 4, AS = 72;
+    constexpr int YV = kLrTile * L / 4, YVT = (YV + kLrThreads - 1) / kLrThreads;
+    extern __shared__ __align__(16) float lr_psm[];
+    auto As = reinterpret_cast<float(*)[AS]>(lr_psm);
+    auto Bh = reinterpret_cast<uint32_t(*)[LP]>(lr_psm + 64 * AS);
+    auto Bl = reinterpret_cast<uint32_t(*)[LP]>(lr_psm + 64 * AS + kLrTile * LP);
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, q = lane & 3;
+    const int kb = 16 * (warp >> 1), cb = (warp & 1) * NBW;
     const int64_t k0 = (int64_t)blockIdx.x * 64;
     const int64_t rb = (int64_t)blockIdx.y * rows_per_split;
     const int64_t re = rb + rows_per_split < p.N ? rb + rows_per_split : p.N;
-    const int ur = t >> 3, uk = 8 * (t & 7);
-    const int tk = (t / CG) * RPT, tc = 4 * (t % CG);
+    const int ur[2] = {t >> 3, (t >> 3) + 32}, uk = 8 * (t & 7);
+    const int hs = (t & 4) ? 4 : 0;
     const bool col_ok = k0 + uk < p.K;
-    float acc[RPT][4];
+    float acc[NBW][4];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
-    auto load = [&](int64_t r0, UnitLoad& u, float4 (&yv)[(YV + kLrThreads - 1) / kLrThreads]) {
-        const int64_t n = r0 + ur;
-        u = unit_load<NBITS>(p, n * p.K + k0 + uk, col_ok && n < re);
+    for (int i = 0; i < NBW; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+    auto load = [&](int64_t r0, UnitLoad (&u)[2], float4 (&yv)[YVT]) {
 #pragma unroll
-        for (int v = 0; v < (YV + kLrThreads - 1) / kLrThreads; ++v) {
+        for (int h = 0; h < 2; ++h) {
+            const int64_t n = r0 + ur[h];
+            u[h] = unit_load<NBITS>(p, n * p.K + k0 + uk, col_ok && n < re);
+        }
+#pragma unroll
+        for (int v = 0; v < YVT; ++v) {
             const int idx = t + v * kLrThreads;
             const int r = idx / CG, c4 = idx % CG;
             yv[v] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -197,56 +270,49 @@ lr_left_kernel(const __grid_constant__ LrParams p, const float* __restrict__ Y,
                 yv[v] = __ldg(reinterpret_cast<const float4*>(Y + (r0 + r) * L) + c4);
         }
     };
-    UnitLoad u;
-    float4 yv[(YV + kLrThreads - 1) / kLrThreads];
+    UnitLoad u[2];
+    float4 yv[YVT];
     if (rb < re) load(rb, u, yv);
-    for (int64_t r0 = rb; r0 < re; r0 += 32) {
-        float d[8];
-        unit_delta<NBITS>(u, d);
-        {   // lanes 4..7 of each group of 8 write their upper half first: the 8
-            // lanes of a quarter-warp then cover all 32 banks in each store
-            const int h = (t & 4) ? 4 : 0;
-            *reinterpret_cast<float4*>(&As[ur][uk + h]) =
-                h ? make_float4(d[4], d[5], d[6], d[7]) : make_float4(d[0], d[1], d[2], d[3]);
-            *reinterpret_cast<float4*>(&As[ur][uk + 4 - h]) =
-                h ? make_float4(d[0], d[1], d[2], d[3]) : make_float4(d[4], d[5], d[6], d[7]);
+    for (int64_t r0 = rb; r0 < re; r0 += kLrTile) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float d[8];
+            unit_delta<NBITS>(u[h], d);
+            const float4 lo = make_float4(d[0], d[1], d[2], d[3]), hi = make_float4(d[4], d[5], d[6], d[7]);
+            *reinterpret_cast<float4*>(&As[ur[h]][uk + hs]) = hs ? hi : lo;
+            *reinterpret_cast<float4*>(&As[ur[h]][uk + 4 - hs]) = hs ? lo : hi;
         }
 #pragma unroll
-        for (int v = 0; v < (YV + kLrThreads - 1) / kLrThreads; ++v) {
+        for (int v = 0; v < YVT; ++v) {
             const int idx = t + v * kLrThreads;
-            if (idx < YV) *reinterpret_cast<float4*>(&Bs[idx / CG][4 * (idx % CG)]) = yv[v];
+            if (idx < YV) store_split4(&Bh[idx / CG][4 * (idx % CG)], &Bl[idx / CG][4 * (idx % CG)], yv[v]);
         }
         __syncthreads();
-        if (r0 + 32 < re) load(r0 + 32, u, yv);
-#pragma unroll 8
-        for (int r = 0; r < 32; ++r) {
-            const float4 b = *reinterpret_cast<const float4*>(&Bs[r][tc]);
-            float a[RPT];
-            if constexpr (RPT == 4) {
-                const float4 a4 = *reinterpret_cast<const float4*>(&As[r][tk]);
-                a[0] = a4.x; a[1] = a4.y; a[2] = a4.z; a[3] = a4.w;
-            } else if constexpr (RPT == 2) {
-                const float2 a2 = *reinterpret_cast<const float2*>(&As[r][tk]);
-                a[0] = a2.x; a[1] = a2.y;
-            } else {
-                a[0] = As[r][tk];
-            }
+        if (r0 + kLrTile < re) load(r0 + kLrTile, u, yv);
+#pragma unroll 4
+        for (int n8 = 0; n8 < kLrTile; n8 += 8) {
+            uint32_t ah[4], al[4];                 // dW^T fragment: (k, n) = As[n][k]
+            split_tf32(As[n8 + q][kb + g], ah[0], al[0]);
+            split_tf32(As[n8 + q][kb + g + 8], ah[1], al[1]);
+            split_tf32(As[n8 + q + 4][kb + g], ah[2], al[2]);
+            split_tf32(As[n8 + q + 4][kb + g + 8], ah[3], al[3]);
 #pragma unroll
-            for (int i = 0; i < RPT; ++i) {
-                acc[i][0] = __fmaf_rn(a[i], b.x, acc[i][0]);
-                acc[i][1] = __fmaf_rn(a[i], b.y, acc[i][1]);
-                acc[i][2] = __fmaf_rn(a[i], b.z, acc[i][2]);
-                acc[i][3] = __fmaf_rn(a[i], b.w, acc[i][3]);
+            for (int i = 0; i < NBW; ++i) {
+                const int c = 8 * (cb + i) + g;
+                mma3(acc[i], ah, al, Bh[n8 + q][c], Bh[n8 + q + 4][c], Bl[n8 + q][c],
+                     Bl[n8 + q + 4][c]);
             }
         }
         __syncthreads();
     }
     float* o = out + (int64_t)blockIdx.y * p.K * L;
 #pragma unroll
-    for (int i = 0; i < RPT; ++i)
-        if (k0 + tk + i < p.K)
-            *reinterpret_cast<float4*>(o + (k0 + tk + i) * L + tc) =
-                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    for (int i = 0; i < NBW; ++i) {
+        const int c = 8 * (cb + i) + 2 * q;
+        const int64_t r0 = k0 + kb + g, r1 = r0 + 8;
+        if (r0 < p.K) *reinterpret_cast<float2*>(o + r0 * L + c) = make_float2(acc[i][0], acc[i][1]);
+        if (r1 < p.K) *reinterpret_cast<float2*>(o + r1 * L + c) = make_float2(acc[i][2], acc[i][3]);
+    }
 }
 
 // Z[i] = sum_s Zp[s * n + i].
@@ -290,6 +356,19 @@ lr_gram_kernel(const float* __restrict__ X, int64_t n, int64_t rpb, double* __re
     for (int e = 0; e < EPT; ++e) GP[(int64_t)blockIdx.x * L * L + e0 + e] = acc[e];
 }
 
+// Sum over the nparts Gram blocks of element e: eight independent partial
+// sums (loads in flight), then added in a fixed order.
+template <int L>
+__device__ __forceinline__ double sum_parts(const double* __restrict__ GP, int nparts, int e) {
+    double a[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    int q = 0;
+    for (; q + 8 <= nparts; q += 8)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] += __ldg(GP + (int64_t)(q + i) * L * L + e);
+    for (; q < nparts; ++q) a[q & 7] += __ldg(GP + (int64_t)q * L * L + e);
+    return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+}
+
 // One CTA: G = sum of the nparts Gram blocks (+ shift * trace / L on the
 // diagonal when shift > 0), G = R^T R (upper R), Rinv = R^-1 (fp32 out).  A
 // pivot at most 1e-20 of G's largest diagonal (a column with no norm left)
@@ -305,7 +384,7 @@ lr_chol_kernel(const double* __restrict__ GP, int nparts, double shift, float* _
     const int t = threadIdx.x;
     for (int e = t; e < L * L; e += kLrThreads) {
         double s = 0.0;
-        for (int q = 0; q < nparts; ++q) s += GP[(int64_t)q * L * L + e];
+        s = sum_parts<L>(GP, nparts, e);
         G[e / L][e % L] = s;
         R[e / L][e % L] = 0.0;
     }
@@ -412,7 +491,7 @@ lr_jacobi_kernel(const double* __restrict__ GP, int nparts, int rank, float* __r
     const int t = threadIdx.x;
     for (int e = t; e < L * L; e += kLrThreads) {
         double s = 0.0;
-        for (int q = 0; q < nparts; ++q) s += GP[(int64_t)q * L * L + e];
+        s = sum_parts<L>(GP, nparts, e);
         A[e / L][e % L] = s;
         V[e / L][e % L] = (e / L == e % L) ? 1.0 : 0.0;
     }
@@ -550,18 +629,25 @@ cudaError_t run(const LrParams& p, int rank, int power_iters, const float* omega
         e = cudaFuncSetAttribute(lr_jacobi_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kJacobiSmem);
     if (e != cudaSuccess) return e;
+    constexpr int kRightSmem = prod_smem<L, 68>(), kLeftSmem = prod_smem<L, 72>();
+    e = cudaFuncSetAttribute(lr_right_kernel<NBITS, L>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kRightSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(lr_left_kernel<NBITS, L>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kLeftSmem);
+    if (e != cudaSuccess) return e;
     const int64_t SR = right_splits(p.N), SL = left_splits(p.K);
-    const int64_t ktiles = (p.K + 31) / 32;
+    const int64_t ktiles = (p.K + kLrTile - 1) / kLrTile;
     const int64_t tps = (ktiles + SR - 1) / SR;                 // k-tiles per right split
-    const int64_t rps = ((p.N + SL - 1) / SL + 31) / 32 * 32;   // rows per left split
+    const int64_t rps = ((p.N + SL - 1) / SL + kLrTile - 1) / kLrTile * kLrTile;   // rows per left split
     auto right = [&](const float* M) {
-        lr_right_kernel<NBITS, L><<<dim3((unsigned)((p.N + 63) / 64), (unsigned)SR), kLrThreads, 0,
-                                    st>>>(p, M, SR > 1 ? w.P : w.Y, tps);
+        lr_right_kernel<NBITS, L><<<dim3((unsigned)((p.N + 63) / 64), (unsigned)SR), kLrThreads,
+                                    kRightSmem, st>>>(p, M, SR > 1 ? w.P : w.Y, tps);
         if (SR > 1) lr_reduce_kernel<<<592, kLrThreads, 0, st>>>(w.P, (int)SR, p.N * L, w.Y);
     };
     auto left = [&]() {
-        lr_left_kernel<NBITS, L><<<dim3((unsigned)((p.K + 63) / 64), (unsigned)SL), kLrThreads, 0,
-                                   st>>>(p, w.Y, SL > 1 ? w.P : w.Z, rps);
+        lr_left_kernel<NBITS, L><<<dim3((unsigned)((p.K + 63) / 64), (unsigned)SL), kLrThreads,
+                                   kLeftSmem, st>>>(p, w.Y, SL > 1 ? w.P : w.Z, rps);
         if (SL > 1) lr_reduce_kernel<<<592, kLrThreads, 0, st>>>(w.P, (int)SL, p.K * L, w.Z);
     };
     auto gram = [&](const float* X, int64_t n) {
