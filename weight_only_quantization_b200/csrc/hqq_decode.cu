@@ -85,9 +85,34 @@ struct Run<3, S, VEC> {
 #pragma unroll
         for (int i = 0; i < NR; ++i) r[i] = __funnelshift_r(p[i] << 2, p[i + 1], 2u + 3u * o);
     }
+    // Constants the caller sets once per kernel, opaque to the compiler so that
+    // they stay in registers: the bits of 2^23 (one logic operation per code,
+    // (field & mask) | magic, with the mask as the immediate) and the
+    // multipliers 2^20 and 2^8 (a right shift by 12 or 24 as a multiply-high,
+    // kept off the logic pipe).
+    uint32_t mg, k20, k8;
+    // codes at bits b, b + 3 of x (b = 0, or 6 when B6) as exact floats
+    template <int B6>
+    __device__ __forceinline__ float2 pair3(uint32_t x) const {
+        constexpr uint32_t m0 = 7u << (B6 ? 6 : 0), m1 = m0 << 3;
+        uint32_t f0, f1;
+        asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(f0) : "r"(x), "n"(m0), "r"(mg));
+        asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(f1) : "r"(x), "n"(m1), "r"(mg));
+        constexpr float i0 = B6 ? 1.0f / 64 : 1.0f, i1 = B6 ? 1.0f / 512 : 1.0f / 8;
+        constexpr float o0 = B6 ? -131072.0f : -8388608.0f, o1 = B6 ? -16384.0f : -1048576.0f;
+        return __ffma2_rn(make_float2(__uint_as_float(f0), __uint_as_float(f1)), make_float2(i0, i1),
+                          make_float2(o0, o1));
+    }
+    // slots 0-1, 2-3 from x; 4-5, 6-7 from x >> 12; 8-9 from x >> 24: two
+    // constant sets for the five pairs of a word
     __device__ __forceinline__ float2 pair(int pp) const {
         const int m = 2 * pp, sl = m % 10;
-        return sl < 6 ? field_pair<3>(r[m / 10], 3 * sl) : field_pair<3>(r[m / 10] >> 12, 3 * sl - 12);
+        const uint32_t x = r[m / 10];
+        if (sl == 0) return pair3<0>(x);
+        if (sl == 2) return pair3<1>(x);
+        if (sl == 4) return pair3<0>(__umulhi(x, k20));
+        if (sl == 6) return pair3<1>(__umulhi(x, k20));
+        return pair3<0>(__umulhi(x, k8));
     }
     __device__ __forceinline__ uint32_t dq(int pp, float z, float s) const { return dq2(pair(pp), z, s); }
 };
@@ -331,7 +356,7 @@ __device__ __forceinline__ void chunk_mma(float (&acc)[NT][4], const Run<NBITS, 
 // the copy is zero-filled), so two chunks are in flight while one is decoded;
 // otherwise the lanes load their runs from global memory directly.
 template <int NBITS, int S, bool VEC, bool STAGED, int NT, bool MX>
-__global__ void __launch_bounds__(kDcThreads, NT == 1 ? 3 : 2)
+__global__ void __launch_bounds__(kDcThreads, NT == 2 ? 2 : NBITS == 3 ? 4 : 3)
 decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams p, int split,
               int64_t packed_bytes) {
     extern __shared__ __align__(16) uint32_t dc_smem[];
@@ -341,6 +366,8 @@ decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams
     const int rank = (int)(blockIdx.x % (unsigned)split);
     const int64_t tile = blockIdx.x / (unsigned)split;
 
+    uint32_t mg = 0x4B000000u, k20 = 1u << 20, k8 = 1u << 8;
+    asm volatile("" : "+r"(mg), "+r"(k20), "+r"(k8));
     const int64_t n0 = tile * 16 + r, n1 = n0 + 8;
     const bool ok0 = n0 < p.N, ok1 = n1 < p.N;
     const int64_t runs = p.K / S;                         // runs per feature
@@ -432,6 +459,11 @@ decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams
             const uint32_t* s0 = ring + stage * G::STAGE + r * G::RS;
             const uint32_t* s1 = s0 + 8 * G::RS;
             Run<NBITS, S, VEC> a, b;
+            if constexpr (NBITS == 3) {
+                a.mg = b.mg = mg;
+                a.k20 = b.k20 = k20;
+                a.k8 = b.k8 = k8;
+            }
             if constexpr (NBITS == 1) {
                 a.read(reinterpret_cast<const uint16_t*>(s0) + l0.off, 0u);
                 b.read(reinterpret_cast<const uint16_t*>(s1) + l1.off, 0u);
@@ -453,6 +485,11 @@ decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams
             const bool v0 = ok0 && qok, v1 = ok1 && qok;
             const int64_t f0 = n0 * p.K + k, f1 = f0 + 8 * p.K;
             Run<NBITS, S, VEC> a, b;
+            if constexpr (NBITS == 3) {
+                a.mg = b.mg = mg;
+                a.k20 = b.k20 = k20;
+                a.k8 = b.k8 = k8;
+            }
             a.load(p.packed, f0, v0);
             b.load(p.packed, f1, v1);
             chunk_mma<NBITS, S, VEC, NT, MX>(acc, a, b, group_of(ch, g0, ok0), group_of(ch, g1, ok1),

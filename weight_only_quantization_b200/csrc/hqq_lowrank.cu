@@ -339,12 +339,24 @@ lr_gram_kernel(const float* __restrict__ X, int64_t n, int64_t rpb, double* __re
     for (int e = 0; e < EPT; ++e) acc[e] = 0.0;
     const int64_t rb = (int64_t)blockIdx.x * rpb;
     const int64_t re = rb + rpb < n ? rb + rpb : n;
+    constexpr int LPT = 32 * L / kLrThreads;              // tile values per thread
+    float nx[LPT];                                        // the next tile, loaded ahead
+    auto fetch = [&](int64_t r0) {
+#pragma unroll
+        for (int u = 0; u < LPT; ++u) {
+            const int idx = t + u * kLrThreads, r = idx / L, c = idx % L;
+            nx[u] = r0 + r < re ? __ldg(X + (r0 + r) * L + c) : 0.0f;
+        }
+    };
+    if (rb < re) fetch(rb);
     for (int64_t r0 = rb; r0 < re; r0 += 32) {
-        for (int idx = t; idx < 32 * L; idx += kLrThreads) {
-            const int r = idx / L, c = idx % L;
-            Xs[r][c] = r0 + r < re ? X[(r0 + r) * L + c] : 0.0f;
+#pragma unroll
+        for (int u = 0; u < LPT; ++u) {
+            const int idx = t + u * kLrThreads;
+            Xs[idx / L][idx % L] = nx[u];
         }
         __syncthreads();
+        if (r0 + 32 < re) fetch(r0 + 32);
         for (int r = 0; r < 32; ++r) {
             const double a = (double)Xs[r][i];
 #pragma unroll
@@ -354,6 +366,37 @@ lr_gram_kernel(const float* __restrict__ X, int64_t n, int64_t rpb, double* __re
     }
 #pragma unroll
     for (int e = 0; e < EPT; ++e) GP[(int64_t)blockIdx.x * L * L + e0 + e] = acc[e];
+}
+
+// Block 0 of GP <- the sum of the nparts Gram blocks (L x L doubles each), in a
+// fixed order: CTA b owns elements 32b .. 32b + 31 (L * L is a multiple of 32);
+// warp s of 8 sums blocks s, s + 8, .. (four running sums), then the eight
+// warp sums are added in order.  Each element is read and written by its own
+// CTA only, and block 0's element is written after every read of it.
+template <int L>
+__global__ void __launch_bounds__(kLrThreads)
+lr_gsum_kernel(double* GP, int nparts) {
+    __shared__ double red[8][32];
+    constexpr int64_t LL = (int64_t)L * L;
+    const int el = threadIdx.x & 31, s = threadIdx.x >> 5;
+    const int64_t e = (int64_t)blockIdx.x * 32 + el;
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    int q = s;
+    for (; q + 24 < nparts; q += 32) {
+        a0 += __ldg(GP + q * LL + e);
+        a1 += __ldg(GP + (q + 8) * LL + e);
+        a2 += __ldg(GP + (q + 16) * LL + e);
+        a3 += __ldg(GP + (q + 24) * LL + e);
+    }
+    for (; q < nparts; q += 8) a0 += __ldg(GP + q * LL + e);
+    red[s][el] = (a0 + a1) + (a2 + a3);
+    __syncthreads();
+    if (s == 0) {
+        double t = red[0][el];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) t += red[i][el];
+        GP[e] = t;
+    }
 }
 
 // Sum over the nparts Gram blocks of element e: eight independent partial
@@ -369,64 +412,95 @@ __device__ __forceinline__ double sum_parts(const double* __restrict__ GP, int n
     return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
-// One CTA: G = sum of the nparts Gram blocks (+ shift * trace / L on the
-// diagonal when shift > 0), G = R^T R (upper R), Rinv = R^-1 (fp32 out).  A
-// pivot at most 1e-20 of G's largest diagonal (a column with no norm left)
-// becomes 1 with a zero row of R: that column of X R^-1 stays as it is (near
-// zero) instead of being blown up.
+// One warp: G = the Gram matrix in block 0 of GP (+ shift * trace / L on the
+// diagonal when shift > 0), G = R^T R (upper R, row by row: R[k][j] = (G[k][j]
+// - sum_{i<k} R[i][k] R[i][j]) / R[k][k]), Rinv = R^-1 (fp32 out).  Lane l
+// owns columns l, l + 32, ..  A pivot at most 1e-20 of G's largest diagonal (a
+// column with no norm left) becomes 1 with a zero row of R: that column of
+// X R^-1 stays as it is (near zero) instead of being blown up.
 template <int L>
-__global__ void __launch_bounds__(kLrThreads)
-lr_chol_kernel(const double* __restrict__ GP, int nparts, double shift, float* __restrict__ Rinv) {
+__global__ void __launch_bounds__(32)
+lr_chol_kernel(const double* __restrict__ GP, double shift, float* __restrict__ Rinv) {
+    constexpr int CPL = (L + 31) / 32;                    // columns per lane
     extern __shared__ double lr_dsm[];                    // G, R, Ri: L x (L + 1) each
     auto G = reinterpret_cast<double(*)[L + 1]>(lr_dsm);
     auto R = reinterpret_cast<double(*)[L + 1]>(lr_dsm + L * (L + 1));
     auto Ri = reinterpret_cast<double(*)[L + 1]>(lr_dsm + 2 * L * (L + 1));
-    const int t = threadIdx.x;
-    for (int e = t; e < L * L; e += kLrThreads) {
-        double s = 0.0;
-        s = sum_parts<L>(GP, nparts, e);
-        G[e / L][e % L] = s;
+    __shared__ double ir[L];                              // 1 / R[k][k]
+    const int lane = threadIdx.x;
+#pragma unroll 16
+    for (int e = lane; e < L * L; e += 32) {              // loads kept in flight
+        G[e / L][e % L] = __ldg(GP + e);
         R[e / L][e % L] = 0.0;
     }
-    __syncthreads();
-    __shared__ double thr;
-    __shared__ int live;
-    if (t == 0) {
-        double tr = 0.0, dmax = 0.0;
-        for (int i = 0; i < L; ++i) {
-            tr += G[i][i];
-            dmax = G[i][i] > dmax ? G[i][i] : dmax;
-        }
-        const double sh = shift * tr / L;
-        for (int i = 0; i < L; ++i) G[i][i] += sh;
-        thr = 1e-20 * dmax + 1e-300;
+    __syncwarp();
+    double tr = 0.0, dmax = 0.0;
+    for (int i = lane; i < L; i += 32) {
+        tr += G[i][i];
+        dmax = G[i][i] > dmax ? G[i][i] : dmax;
     }
-    __syncthreads();
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tr += __shfl_xor_sync(0xffffffffu, tr, o);
+        dmax = fmax(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+    }
+    const double sh = shift * tr / L, thr = 1e-20 * dmax + 1e-300;
     for (int k = 0; k < L; ++k) {
-        if (t == 0) {
-            const double d = G[k][k];
-            live = d > thr;
-            R[k][k] = live ? sqrt(d) : 1.0;
+        double sv[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int j = lane + 32 * c;
+            double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+            if (j < L && j >= k) {
+                int i = 0;
+                for (; i + 4 <= k; i += 4) {
+                    s0 = fma(R[i][k], R[i][j], s0);
+                    s1 = fma(R[i + 1][k], R[i + 1][j], s1);
+                    s2 = fma(R[i + 2][k], R[i + 2][j], s2);
+                    s3 = fma(R[i + 3][k], R[i + 3][j], s3);
+                }
+                for (; i < k; ++i) s0 = fma(R[i][k], R[i][j], s0);
+            }
+            sv[c] = (j < L ? G[k][j] + (j == k ? sh : 0.0) : 0.0) - ((s0 + s1) + (s2 + s3));
         }
-        __syncthreads();
-        for (int j = k + 1 + t; j < L; j += kLrThreads) R[k][j] = live ? G[k][j] / R[k][k] : 0.0;
-        __syncthreads();
-        for (int e = t; e < L * L; e += kLrThreads) {
-            const int i = e / L, j = e % L;
-            if (i > k && j >= i) G[i][j] -= R[k][i] * R[k][j];
+        double d = sv[0];
+#pragma unroll
+        for (int c = 1; c < CPL; ++c)
+            if ((k >> 5) == c) d = sv[c];
+        d = __shfl_sync(0xffffffffu, d, k & 31);
+        const bool live = d > thr;
+        const double inv = live ? rsqrt(d) : 1.0, rkk = live ? d * inv : 1.0;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int j = lane + 32 * c;
+            if (j < L && j > k) R[k][j] = live ? sv[c] * inv : 0.0;
         }
-        __syncthreads();
+        if (lane == 0) {
+            R[k][k] = rkk;
+            ir[k] = inv;
+        }
+        __syncwarp();
     }
-    for (int j = t; j < L; j += kLrThreads) {      // column j of the upper inverse
-        for (int i = L - 1; i > j; --i) Ri[i][j] = 0.0;
-        for (int i = j; i >= 0; --i) {
-            double s = i == j ? 1.0 : 0.0;
-            for (int k = i + 1; k <= j; ++k) s -= R[i][k] * Ri[k][j];
-            Ri[i][j] = s / R[i][i];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {                       // column j of the upper inverse
+        const int j = lane + 32 * c;
+        if (j < L) {
+            for (int i = L - 1; i > j; --i) Ri[i][j] = 0.0;
+            Ri[j][j] = ir[j];
+            for (int i = j - 1; i >= 0; --i) {
+                double s0 = 0.0, s1 = 0.0;
+                int k = i + 1;
+                for (; k + 2 <= j + 1; k += 2) {
+                    s0 = fma(R[i][k], Ri[k][j], s0);
+                    s1 = fma(R[i][k + 1], Ri[k + 1][j], s1);
+                }
+                if (k <= j) s0 = fma(R[i][k], Ri[k][j], s0);
+                Ri[i][j] = -(s0 + s1) * ir[i];
+            }
         }
     }
-    __syncthreads();
-    for (int e = t; e < L * L; e += kLrThreads) Rinv[e] = (float)Ri[e / L][e % L];
+    __syncwarp();
+    for (int e = lane; e < L * L; e += 32) Rinv[e] = (float)Ri[e / L][e % L];
 }
 
 // out = X[n, L] Rm[L, L] restricted to the first ncols columns; one row per
@@ -451,21 +525,30 @@ lr_apply_kernel(const float* X, int64_t n, const float* __restrict__ Rm, int nco
         x[c + 3] = v.w;
     }
     constexpr int JB = L < 16 ? L : 16;
+    // row-major output in whole 16-byte pieces when the rows allow it
+    const bool vec = !trans && (ostride & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
     for (int j0 = 0; j0 < ncols; j0 += JB) {
         float o[JB];
 #pragma unroll
         for (int jj = 0; jj < JB; ++jj) o[jj] = 0.0f;
-#pragma unroll 8
+#pragma unroll
         for (int c = 0; c < L; ++c)
 #pragma unroll
             for (int jj = 0; jj < JB; ++jj)
                 if (j0 + jj < L) o[jj] = __fmaf_rn(x[c], Rs[c][j0 + jj], o[jj]);
+        if (vec && j0 + JB <= ncols) {
 #pragma unroll
-        for (int jj = 0; jj < JB; ++jj) {
-            const int j = j0 + jj;
-            if (j < ncols) {
-                if (trans) out[(int64_t)j * ostride + row] = o[jj];
-                else out[row * ostride + j] = o[jj];
+            for (int jj = 0; jj < JB; jj += 4)
+                *reinterpret_cast<float4*>(out + row * ostride + j0 + jj) =
+                    make_float4(o[jj], o[jj + 1], o[jj + 2], o[jj + 3]);
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < JB; ++jj) {
+                const int j = j0 + jj;
+                if (j < ncols) {
+                    if (trans) out[(int64_t)j * ostride + row] = o[jj];
+                    else out[row * ostride + j] = o[jj];
+                }
             }
         }
     }
@@ -486,6 +569,7 @@ lr_jacobi_kernel(const double* __restrict__ GP, int nparts, int rank, float* __r
     __shared__ double rc[L / 2], rs[L / 2];
     __shared__ int rp[L / 2], rq[L / 2];
     __shared__ double off_rel;
+    __shared__ double wsum[kLrThreads / 32][2];
     __shared__ int perm[L];
     __shared__ double sg[L];
     const int t = threadIdx.x;
@@ -497,15 +581,32 @@ lr_jacobi_kernel(const double* __restrict__ GP, int nparts, int rank, float* __r
     }
     __syncthreads();
     for (int sweep = 0; sweep < 40; ++sweep) {
-        if (t == 0) {
+        {
             double off = 0.0, tot = 0.0;
-            for (int i = 0; i < L; ++i)
-                for (int j = 0; j < L; ++j) {
-                    const double a2 = A[i][j] * A[i][j];
-                    tot += a2;
-                    if (i != j) off += a2;
+            for (int e = t; e < L * L; e += kLrThreads) {
+                const int i = e / L, j = e % L;
+                const double a2 = A[i][j] * A[i][j];
+                tot += a2;
+                if (i != j) off += a2;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                off += __shfl_xor_sync(0xffffffffu, off, o);
+                tot += __shfl_xor_sync(0xffffffffu, tot, o);
+            }
+            if ((t & 31) == 0) {
+                wsum[t >> 5][0] = off;
+                wsum[t >> 5][1] = tot;
+            }
+            __syncthreads();
+            if (t == 0) {
+                double fo = 0.0, ft = 0.0;
+                for (int w = 0; w < kLrThreads / 32; ++w) {
+                    fo += wsum[w][0];
+                    ft += wsum[w][1];
                 }
-            off_rel = tot > 0.0 ? off / tot : 0.0;
+                off_rel = ft > 0.0 ? fo / ft : 0.0;
+            }
         }
         __syncthreads();
         if (off_rel < 1e-28) break;
@@ -516,9 +617,13 @@ lr_jacobi_kernel(const double* __restrict__ GP, int nparts, int rank, float* __r
                 const double apq = A[p][q];
                 double c = 1.0, s = 0.0;
                 if (fabs(apq) > 1e-300) {
-                    const double tau = (A[q][q] - A[p][p]) / (2.0 * apq);
-                    const double tt = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
-                    c = 1.0 / sqrt(1.0 + tt * tt);
+                    // t = tan of the rotation angle, the smaller root of
+                    // t^2 + 2 tau t - 1 = 0 with tau = (a_qq - a_pp) / (2 a_pq),
+                    // written as 2 a_pq sign(dq) / (|dq| + sqrt(dq^2 + 4 a_pq^2))
+                    const double dq = A[q][q] - A[p][p];
+                    const double tt = (dq >= 0.0 ? 2.0 * apq : -2.0 * apq) /
+                                      (fabs(dq) + sqrt(dq * dq + 4.0 * apq * apq));
+                    c = rsqrt(1.0 + tt * tt);
                     s = tt * c;
                 }
                 rp[t] = p;
@@ -650,15 +755,20 @@ cudaError_t run(const LrParams& p, int rank, int power_iters, const float* omega
                                    kLeftSmem, st>>>(p, w.Y, SL > 1 ? w.P : w.Z, rps);
         if (SL > 1) lr_reduce_kernel<<<592, kLrThreads, 0, st>>>(w.P, (int)SL, p.K * L, w.Z);
     };
+    // X^T X into block 0 of w.GP: Gram blocks of at least kGramRows rows, about
+    // one per SM of a 148-SM part (never more blocks than the workspace holds),
+    // then their fixed-order sum
     auto gram = [&](const float* X, int64_t n) {
-        const int64_t parts = (n + kGramRows - 1) / kGramRows;
-        lr_gram_kernel<L><<<(unsigned)parts, kLrThreads, 0, st>>>(X, n, kGramRows, w.GP);
-        return (int)parts;
+        int64_t rpb = ((n + 147) / 148 + 31) / 32 * 32;
+        rpb = rpb < kGramRows ? kGramRows : rpb;
+        const int64_t parts = (n + rpb - 1) / rpb;
+        lr_gram_kernel<L><<<(unsigned)parts, kLrThreads, 0, st>>>(X, n, rpb, w.GP);
+        if (parts > 1) lr_gsum_kernel<L><<<L * L / 32, kLrThreads, 0, st>>>(w.GP, (int)parts);
     };
     auto orth = [&](float* X, int64_t n) {
         for (int pass = 0; pass < 3; ++pass) {
-            const int parts = gram(X, n);
-            lr_chol_kernel<L><<<1, kLrThreads, kCholSmem, st>>>(w.GP, parts, pass == 0 ? 1e-9 : 0.0, w.R);
+            gram(X, n);
+            lr_chol_kernel<L><<<1, 32, kCholSmem, st>>>(w.GP, pass == 0 ? 1e-9 : 0.0, w.R);
             lr_apply_kernel<L><<<(unsigned)((n + kLrThreads - 1) / kLrThreads), kLrThreads, 0, st>>>(
                 X, n, w.R, L, X, L, 0);
         }
@@ -672,8 +782,8 @@ cudaError_t run(const LrParams& p, int rank, int power_iters, const float* omega
         orth(w.Y, p.N);
     }
     left();
-    const int parts = gram(w.Z, p.K);
-    lr_jacobi_kernel<L><<<1, kLrThreads, kJacobiSmem, st>>>(w.GP, parts, rank, w.Mr, w.Mi, sigma);
+    gram(w.Z, p.K);
+    lr_jacobi_kernel<L><<<1, kLrThreads, kJacobiSmem, st>>>(w.GP, 1, rank, w.Mr, w.Mi, sigma);
     lr_apply_kernel<L><<<(unsigned)((p.N + kLrThreads - 1) / kLrThreads), kLrThreads, 0, st>>>(
         w.Y, p.N, w.Mr, rank, B, rank, 0);
     lr_apply_kernel<L><<<(unsigned)((p.K + kLrThreads - 1) / kLrThreads), kLrThreads, 0, st>>>(
