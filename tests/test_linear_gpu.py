@@ -180,11 +180,13 @@ def test_linear_exact_full_size_k(hqq, rows, cols, nbits, M):
     assert not bad.any(), (int(bad.sum()), np.argwhere(bad)[:5].tolist())
 
 
-@pytest.mark.parametrize("nbits,group", [(3, 64), (4, 64), (2, 16), (8, 32), (1, 128)])
-@pytest.mark.parametrize("M", [4, 8, 9, 15, 24, 32, 33])
+@pytest.mark.parametrize("nbits,group", [(3, 64), (3, 32), (3, 16), (4, 64), (2, 16), (8, 32), (1, 128)])
+@pytest.mark.parametrize("M", [4, 8, 9, 15, 16, 24, 32, 33])
 def test_linear_decode_token_blocks(hqq, nbits, group, M):
     """Token counts inside and at the edges of the few-token kernel's 8-token
-    MMA column blocks (1, 2 and 4 blocks) and the first count past them."""
+    MMA column blocks (1, 2 and 4 blocks) and the first count past them; at 3
+    bits, 9 to 16 tokens take the kernel whose CTAs share one staged copy of X
+    (200 features: a partly empty 128-feature CTA tile)."""
     rows, cols = 200, 1024
     W = synth.student_t_host((rows, cols), seed=53, stream=nbits * 1000 + M).astype(np.float16)
     q, Wh, _ = _quantized(hqq, W, nbits, group)

@@ -320,11 +320,10 @@ __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0
 // S/4 MMAs per 8-token block of one chunk: codes 4i..4i+3 of the lane's runs of
 // features r and r + 8 against X[m, k + 4i .. k + 4i + 3]; xo[c] = row offset
 // of token 8c + r in X (the last token for rows past M).
-template <int NBITS, int S, bool VEC, int NT, bool MX>
-__device__ __forceinline__ void chunk_mma(float (&acc)[NT][4], const Run<NBITS, S, VEC>& a,
-                                          const Run<NBITS, S, VEC>& b, __half2 sz0, __half2 sz1,
-                                          const __half* __restrict__ X, const int64_t (&xo)[NT],
-                                          int64_t k) {
+template <int NBITS, int S, bool VEC, int NT, bool MX, typename XF>
+__device__ __forceinline__ void chunk_mma_x(float (&acc)[NT][4], const Run<NBITS, S, VEC>& a,
+                                            const Run<NBITS, S, VEC>& b, __half2 sz0, __half2 sz1,
+                                            XF xfrag) {
     const float s0 = __low2float(sz0), z0 = __high2float(sz0);
     const float s1 = __low2float(sz1), z1 = __high2float(sz1);
     auto dq = [&](const Run<NBITS, S, VEC>& run, int pp, float z, float s) {
@@ -339,11 +338,23 @@ __device__ __forceinline__ void chunk_mma(float (&acc)[NT][4], const Run<NBITS, 
         const uint32_t a6 = dq(a, 2 * i + 3, z0, s0), a7 = dq(b, 2 * i + 3, z1, s1);
 #pragma unroll
         for (int c = 0; c < NT; ++c) {
-            const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + xo[c] + k) + i / 2);
+            const uint4 x = xfrag(c, i / 2);
             mma16816(acc[c], a0, a1, a2, a3, x.x, x.y);
             mma16816(acc[c], a4, a5, a6, a7, x.z, x.w);
         }
     }
+}
+
+// X fragments straight from global memory: eight halves of token row xo[c]
+// from k + 8 u.
+template <int NBITS, int S, bool VEC, int NT, bool MX>
+__device__ __forceinline__ void chunk_mma(float (&acc)[NT][4], const Run<NBITS, S, VEC>& a,
+                                          const Run<NBITS, S, VEC>& b, __half2 sz0, __half2 sz1,
+                                          const __half* __restrict__ X, const int64_t (&xo)[NT],
+                                          int64_t k) {
+    chunk_mma_x<NBITS, S, VEC, NT, MX>(acc, a, b, sz0, sz1, [&](int c, int u) {
+        return __ldg(reinterpret_cast<const uint4*>(X + xo[c] + k) + u);
+    });
 }
 
 // Grid: ceil(N / 16) feature tiles x `split` CTAs (a (split, 1, 1) cluster when
@@ -550,6 +561,206 @@ decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams
     }
 }
 
+// Halves per run row of the shared X stage (a run's S values + 8 of padding,
+// so that the eight lanes of each quarter-warp read distinct banks) and per
+// stage (16 token rows x 4 runs).
+template <int S>
+struct XGeo {
+    static constexpr int XR = S + 8;
+    static constexpr int STAGE = 16 * 4 * XR;
+};
+
+template <int NBITS, int S>
+constexpr size_t decode_sx_smem() {
+    const size_t ring = (size_t)kDcWarps * kDcStages * Geo<NBITS, S>::STAGE * 4 +
+                        (size_t)kDcStages * XGeo<S>::STAGE * 2;
+    const size_t red = (size_t)(kDcMaxSplit - 1) * kDcWarps * 4 * 2 * 32 * 4;
+    return ring > red ? ring : red;
+}
+
+// 9 to 16 tokens (two 8-token blocks): the 8 warps of a CTA own 8 consecutive
+// 16-feature tiles and walk the same chunks, so one copy of X per chunk (16
+// token rows x 4S columns, zero past M and past K) serves them all: the CTA's
+// threads stage it with cp.async next to each warp's code ring, and a CTA
+// barrier per chunk publishes it.  Grid: ceil(N / 128) CTA tiles x `split`
+// (a (split, 1, 1) cluster when split > 1; rank = blockIdx.x % split takes
+// chunks rank, rank + split, ..); partial tiles meet in rank 0's shared memory.
+// Needs packed and X 16-byte aligned and K < 2^30.
+template <int NBITS, int S>
+__global__ void __launch_bounds__(kDcThreads, 2)
+decode_sx_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams p, int split,
+                 int64_t packed_bytes) {
+    constexpr int NT = 2;
+    extern __shared__ __align__(16) uint32_t dc_smem[];
+    using G = Geo<NBITS, S>;
+    using XG = XGeo<S>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 2, j = lane & 3;
+    const int rank = (int)(blockIdx.x % (unsigned)split);
+    const int64_t tile = (int64_t)(blockIdx.x / (unsigned)split) * kDcWarps + warp;
+    uint32_t mg = 0x4B000000u, k20 = 1u << 20, k8 = 1u << 8;
+    asm volatile("" : "+r"(mg), "+r"(k20), "+r"(k8));
+
+    const int64_t n0 = tile * 16 + r, n1 = n0 + 8;
+    const bool ok0 = n0 < p.N, ok1 = n1 < p.N;
+    const int64_t runs = p.K / S;
+    const int64_t nchunk = (runs + 3) >> 2;
+    float acc[NT][4];
+#pragma unroll
+    for (int c = 0; c < NT; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
+    int64_t ch = rank;
+    const int64_t gstep = (4 * S * (int64_t)split) >> p.log2_group;
+    int64_t g0 = (n0 * p.K + (4 * ch + j) * S) >> p.log2_group;
+    int64_t g1 = g0 + ((8 * p.K) >> p.log2_group);
+    auto group_of = [&](int64_t c, int64_t g, bool ok) {
+        return (ok && c < nchunk && 4 * c + j < runs) ? group_sz(p, g) : __float2half2_rn(0.0f);
+    };
+
+    uint32_t* ring = dc_smem + (size_t)warp * kDcStages * G::STAGE;
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    const __half* xring = reinterpret_cast<const __half*>(dc_smem + (size_t)kDcWarps * kDcStages * G::STAGE);
+    const uint32_t xring_s = (uint32_t)__cvta_generic_to_shared(xring);
+    const int64_t b00 = NBITS == 3 ? n0 * p.K / 10 : n0 * p.K * NBITS >> 5;
+    const int64_t b10 = NBITS == 3 ? n1 * p.K / 10 : n1 * p.K * NBITS >> 5;
+    const uint32_t b01 = NBITS == 3 ? (uint32_t)(n0 * p.K - 10 * b00) : 0u;
+    const uint32_t b11 = NBITS == 3 ? (uint32_t)(n1 * p.K - 10 * b10) : 0u;
+    // this warp's code granules of chunk c (as in decode_kernel), and this
+    // thread's share of the chunk's X granules: granule q of the stage is
+    // token m = q / (S / 2), run jj, 16-byte piece u of that run
+    auto fill = [&](int64_t c, int stage) {
+        if (c < nchunk) {
+            const uint32_t kc = (uint32_t)(4 * S * c);
+            const Loc<NBITS, S> l0(b00, b01, kc, 0), l1(b10, b11, kc, 0);
+            const uint32_t d0 = ring_s + 4u * (uint32_t)(stage * G::STAGE + r * G::RS) + 16u * j;
+            const uint32_t d1 = d0 + 4u * 8u * G::RS;
+#pragma unroll
+            for (int t = 0; t < G::GPL; ++t) {
+                const int gi = j + 4 * t;
+                if (gi < G::GR) {
+                    const int64_t s0 = 16 * (l0.g + gi), s1 = 16 * (l1.g + gi);
+                    const int64_t r0 = ok0 ? packed_bytes - s0 : 0, r1 = ok1 ? packed_bytes - s1 : 0;
+                    const uint32_t c0 = r0 <= 0 ? 0u : r0 >= 16 ? 16u : (uint32_t)r0;
+                    const uint32_t c1 = r1 <= 0 ? 0u : r1 >= 16 ? 16u : (uint32_t)r1;
+                    cp_async16(d0 + 64u * t, p.packed + (c0 ? s0 : 0), c0);
+                    cp_async16(d1 + 64u * t, p.packed + (c1 ? s1 : 0), c1);
+                }
+            }
+            constexpr int XQ = 16 * 4 * S / 8;               // 16-byte granules per X stage
+            for (int q = threadIdx.x; q < XQ; q += kDcThreads) {
+                const int m = q / (S / 2), o = q % (S / 2), jj = o / (S / 8), u = o % (S / 8);
+                const int64_t k = 4 * S * c + (int64_t)jj * S + 8 * u;
+                const bool in = m < p.M && k < p.K;
+                cp_async16(xring_s + 2u * (uint32_t)(stage * XG::STAGE + (m * 4 + jj) * XG::XR + 8 * u),
+                           in ? X + m * p.K + k : X, in ? 16u : 0u);
+            }
+        }
+        cp_commit();
+    };
+#pragma unroll
+    for (int st = 0; st < kDcStages - 1; ++st) fill(ch + st * (int64_t)split, st);
+    __half2 sz0 = group_of(ch, g0, ok0), sz1 = group_of(ch, g1, ok1);
+    for (int it = 0; ch < nchunk; ++it, ch += split) {
+        g0 += gstep;
+        g1 += gstep;
+        const __half2 nz0 = group_of(ch + split, g0, ok0), nz1 = group_of(ch + split, g1, ok1);
+        cp_wait<kDcStages - 2>();
+        __syncthreads();                       // every thread's copies of this chunk landed
+        fill(ch + (kDcStages - 1) * (int64_t)split, (it + kDcStages - 1) % kDcStages);
+        const int stage = it % kDcStages;
+        const uint32_t kc = (uint32_t)(4 * S * ch);
+        const Loc<NBITS, S> l0(b00, b01, kc, j), l1(b10, b11, kc, j);
+        const uint32_t* s0 = ring + stage * G::STAGE + r * G::RS;
+        const uint32_t* s1 = s0 + 8 * G::RS;
+        Run<NBITS, S, false> a, b;
+        if constexpr (NBITS == 3) {
+            a.mg = b.mg = mg;
+            a.k20 = b.k20 = k20;
+            a.k8 = b.k8 = k8;
+        }
+        a.read(s0 + l0.off, l0.o);
+        b.read(s1 + l1.off, l1.o);
+        const __half* xs = xring + stage * XG::STAGE + j * XG::XR;
+        chunk_mma_x<NBITS, S, false, NT, false>(acc, a, b, sz0, sz1, [&](int c, int u) {
+            return *reinterpret_cast<const uint4*>(xs + (8 * c + r) * 4 * XG::XR + 8 * u);
+        });
+        sz0 = nz0;
+        sz1 = nz1;
+    }
+    cp_wait<0>();
+    __syncthreads();
+
+    // element e of block c in lane l: feature tile*16 + l/4 + 8*(e/2), token
+    // 8c + 2*(l%4) + e%2
+    constexpr int TW = 4 * NT * 32;                       // floats per warp
+    float* cred = reinterpret_cast<float*>(dc_smem);
+    if (split > 1) {
+        // every CTA of the cluster is past its main loop: rank 0's memory is free
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                     "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+        if (rank != 0) {
+            float* dst = cg::this_cluster().map_shared_rank(cred, 0) + ((rank - 1) * kDcWarps + warp) * TW;
+#pragma unroll
+            for (int c = 0; c < NT; ++c)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dst[(4 * c + e) * 32 + lane] = acc[c][e];
+        }
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                     "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+        if (rank == 0)
+            for (int q = 1; q < split; ++q)
+#pragma unroll
+                for (int c = 0; c < NT; ++c)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        acc[c][e] += cred[((q - 1) * kDcWarps + warp) * TW + (4 * c + e) * 32 + lane];
+    }
+    if (rank == 0) {
+#pragma unroll
+        for (int c = 0; c < NT; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int64_t n = tile * 16 + r + 8 * (e >> 1);
+                const int64_t m = 8 * c + 2 * j + (e & 1);
+                if (n < p.N && m < p.M) p.Y[m * p.N + n] = __float2half_rn(acc[c][e]);
+            }
+    }
+}
+
+template <int NBITS, int S>
+cudaError_t launch_sx(const LinearParams& p, const void* X, int64_t packed_bytes, cudaStream_t stream) {
+    auto kern = decode_sx_kernel<NBITS, S>;
+    constexpr size_t smem = decode_sx_smem<NBITS, S>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // split the chunks over a cluster while the grid is short of two CTAs per
+    // SM and every CTA keeps at least two chunks
+    const int64_t ctiles = (p.N + 16 * kDcWarps - 1) / (16 * kDcWarps);
+    const int64_t nchunk = (p.K / S + 3) / 4;
+    int split = 1;
+    while (split < kDcMaxSplit && ctiles * split < 2 * sms && nchunk >= 4 * split) split *= 2;
+    const __half* xp = static_cast<const __half*>(X);
+    if (split == 1) {
+        kern<<<(unsigned)ctiles, kDcThreads, smem, stream>>>(xp, p, 1, packed_bytes);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = (unsigned)split;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(ctiles * split));
+    cfg.blockDim = dim3(kDcThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, xp, p, split, packed_bytes);
+}
+
 template <int NBITS, int S, bool VEC, bool STAGED, int NT, bool MX>
 cudaError_t launch_s(const LinearParams& p, const void* X, int64_t packed_bytes,
                      cudaStream_t stream) {
@@ -612,6 +823,13 @@ cudaError_t launch_g(const LinearParams& p, const void* X, int64_t pb, cudaStrea
 template <int NBITS, bool VEC, int NT, bool MX>
 cudaError_t launch_st(const LinearParams& p, const void* X, int64_t pb, cudaStream_t stream) {
     const bool staged = (reinterpret_cast<uintptr_t>(p.packed) & 15u) == 0 && p.K < ((int64_t)1 << 30);
+    if constexpr (NBITS == 3 && NT == 2) {
+        if (staged && (reinterpret_cast<uintptr_t>(X) & 15u) == 0) {
+            if (p.log2_group == 4) return launch_sx<3, 16>(p, X, pb, stream);
+            if (p.log2_group == 5) return launch_sx<3, 32>(p, X, pb, stream);
+            return launch_sx<3, 64>(p, X, pb, stream);
+        }
+    }
     return staged ? launch_g<NBITS, VEC, true, NT, MX>(p, X, pb, stream)
                   : launch_g<NBITS, VEC, false, NT, MX>(p, X, pb, stream);
 }
