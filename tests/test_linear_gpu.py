@@ -198,11 +198,13 @@ def test_linear_decode_token_blocks(hqq, nbits, group, M):
 
 @pytest.mark.parametrize("nbits,group,rows,cols", [(3, 64, 130, 1088), (4, 16, 48, 16384),
                                                    (1, 32, 77, 96), (8, 64, 33, 512)])
-@pytest.mark.parametrize("M", [1, 5])
+@pytest.mark.parametrize("M", [1, 5, 8, 12])
 def test_linear_decode_packed_alignment(hqq, nbits, group, rows, cols, M):
     """A packed buffer that is 4-byte but not 16-byte aligned takes the
-    few-token kernel's direct-load form; it must give the same bits as the
-    staged form on an aligned copy (same products, same summation order)."""
+    few-token kernels' direct-load form; it must give the same bits as the
+    staged form on an aligned copy (same products, same summation order).  At
+    3 bits, 8 and 12 tokens take the kernel whose CTAs share a staged X; past
+    8 tokens the other widths take the many-token kernel for both copies."""
     W = synth.student_t_host((rows, cols), seed=54, stream=rows + nbits).astype(np.float16)
     q, Wh, r = _quantized(hqq, W, nbits, group)
     shift = 8 if nbits == 8 else 4

@@ -564,36 +564,37 @@ decode_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams
 // Halves per run row of the shared X stage (a run's S values + 8 of padding,
 // so that the eight lanes of each quarter-warp read distinct banks) and per
 // stage (16 token rows x 4 runs).
-template <int S>
+template <int S, int NT>
 struct XGeo {
     static constexpr int XR = S + 8;
-    static constexpr int STAGE = 16 * 4 * XR;
+    static constexpr int STAGE = 8 * NT * 4 * XR;
 };
 
-template <int NBITS, int S>
+template <int NBITS, int S, int NT>
 constexpr size_t decode_sx_smem() {
     const size_t ring = (size_t)kDcWarps * kDcStages * Geo<NBITS, S>::STAGE * 4 +
-                        (size_t)kDcStages * XGeo<S>::STAGE * 2;
-    const size_t red = (size_t)(kDcMaxSplit - 1) * kDcWarps * 4 * 2 * 32 * 4;
+                        (size_t)kDcStages * XGeo<S, NT>::STAGE * 2;
+    const size_t red = (size_t)(kDcMaxSplit - 1) * kDcWarps * 4 * NT * 32 * 4;
     return ring > red ? ring : red;
 }
 
-// 9 to 16 tokens (two 8-token blocks): the 8 warps of a CTA own 8 consecutive
-// 16-feature tiles and walk the same chunks, so one copy of X per chunk (16
+// NT 8-token blocks (2 to 16 tokens): the 8 warps of a CTA own 8 consecutive
+// 16-feature tiles and walk the same chunks, so one copy of X per chunk (8 NT
 // token rows x 4S columns, zero past M and past K) serves them all: the CTA's
 // threads stage it with cp.async next to each warp's code ring, and a CTA
 // barrier per chunk publishes it.  Grid: ceil(N / 128) CTA tiles x `split`
 // (a (split, 1, 1) cluster when split > 1; rank = blockIdx.x % split takes
 // chunks rank, rank + split, ..); partial tiles meet in rank 0's shared memory.
-// Needs packed and X 16-byte aligned and K < 2^30.
-template <int NBITS, int S>
-__global__ void __launch_bounds__(kDcThreads, 2)
+// Needs X 16-byte aligned and K < 2^30.  STAGED (packed 16-byte aligned): each
+// warp's codes come through its cp.async ring as in decode_kernel; otherwise
+// the lanes load their runs from global memory (same products, same order).
+template <int NBITS, int S, int NT, bool STAGED>
+__global__ void __launch_bounds__(kDcThreads, NT == 2 ? 2 : 3)
 decode_sx_kernel(const __half* __restrict__ X, const __grid_constant__ LinearParams p, int split,
                  int64_t packed_bytes) {
-    constexpr int NT = 2;
     extern __shared__ __align__(16) uint32_t dc_smem[];
     using G = Geo<NBITS, S>;
-    using XG = XGeo<S>;
+    using XG = XGeo<S, NT>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, j = lane & 3;
     const int rank = (int)(blockIdx.x % (unsigned)split);
@@ -631,6 +632,7 @@ decode_sx_kernel(const __half* __restrict__ X, const __grid_constant__ LinearPar
         if (c < nchunk) {
             const uint32_t kc = (uint32_t)(4 * S * c);
             const Loc<NBITS, S> l0(b00, b01, kc, 0), l1(b10, b11, kc, 0);
+            if constexpr (STAGED) {
             const uint32_t d0 = ring_s + 4u * (uint32_t)(stage * G::STAGE + r * G::RS) + 16u * j;
             const uint32_t d1 = d0 + 4u * 8u * G::RS;
 #pragma unroll
@@ -645,7 +647,8 @@ decode_sx_kernel(const __half* __restrict__ X, const __grid_constant__ LinearPar
                     cp_async16(d1 + 64u * t, p.packed + (c1 ? s1 : 0), c1);
                 }
             }
-            constexpr int XQ = 16 * 4 * S / 8;               // 16-byte granules per X stage
+            }
+            constexpr int XQ = 8 * NT * 4 * S / 8;           // 16-byte granules per X stage
             for (int q = threadIdx.x; q < XQ; q += kDcThreads) {
                 const int m = q / (S / 2), o = q % (S / 2), jj = o / (S / 8), u = o % (S / 8);
                 const int64_t k = 4 * S * c + (int64_t)jj * S + 8 * u;
@@ -667,18 +670,26 @@ decode_sx_kernel(const __half* __restrict__ X, const __grid_constant__ LinearPar
         __syncthreads();                       // every thread's copies of this chunk landed
         fill(ch + (kDcStages - 1) * (int64_t)split, (it + kDcStages - 1) % kDcStages);
         const int stage = it % kDcStages;
-        const uint32_t kc = (uint32_t)(4 * S * ch);
-        const Loc<NBITS, S> l0(b00, b01, kc, j), l1(b10, b11, kc, j);
-        const uint32_t* s0 = ring + stage * G::STAGE + r * G::RS;
-        const uint32_t* s1 = s0 + 8 * G::RS;
         Run<NBITS, S, false> a, b;
         if constexpr (NBITS == 3) {
             a.mg = b.mg = mg;
             a.k20 = b.k20 = k20;
             a.k8 = b.k8 = k8;
         }
-        a.read(s0 + l0.off, l0.o);
-        b.read(s1 + l1.off, l1.o);
+        if constexpr (STAGED) {
+            const uint32_t kc = (uint32_t)(4 * S * ch);
+            const Loc<NBITS, S> l0(b00, b01, kc, j), l1(b10, b11, kc, j);
+            const uint32_t* s0 = ring + stage * G::STAGE + r * G::RS;
+            const uint32_t* s1 = s0 + 8 * G::RS;
+            a.read(s0 + l0.off, l0.o);
+            b.read(s1 + l1.off, l1.o);
+        } else {
+            const int64_t q = 4 * ch + j;
+            const bool qok = q < runs;
+            const int64_t f0 = n0 * p.K + (qok ? q * S : 0), f1 = f0 + 8 * p.K;
+            a.load(p.packed, f0, ok0 && qok);
+            b.load(p.packed, f1, ok1 && qok);
+        }
         const __half* xs = xring + stage * XG::STAGE + j * XG::XR;
         chunk_mma_x<NBITS, S, false, NT, false>(acc, a, b, sz0, sz1, [&](int c, int u) {
             return *reinterpret_cast<const uint4*>(xs + (8 * c + r) * 4 * XG::XR + 8 * u);
@@ -726,10 +737,10 @@ decode_sx_kernel(const __half* __restrict__ X, const __grid_constant__ LinearPar
     }
 }
 
-template <int NBITS, int S>
+template <int NBITS, int S, int NT, bool STAGED>
 cudaError_t launch_sx(const LinearParams& p, const void* X, int64_t packed_bytes, cudaStream_t stream) {
-    auto kern = decode_sx_kernel<NBITS, S>;
-    constexpr size_t smem = decode_sx_smem<NBITS, S>();
+    auto kern = decode_sx_kernel<NBITS, S, NT, STAGED>;
+    constexpr size_t smem = decode_sx_smem<NBITS, S, NT>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -823,11 +834,20 @@ cudaError_t launch_g(const LinearParams& p, const void* X, int64_t pb, cudaStrea
 template <int NBITS, bool VEC, int NT, bool MX>
 cudaError_t launch_st(const LinearParams& p, const void* X, int64_t pb, cudaStream_t stream) {
     const bool staged = (reinterpret_cast<uintptr_t>(p.packed) & 15u) == 0 && p.K < ((int64_t)1 << 30);
-    if constexpr (NBITS == 3 && NT == 2) {
-        if (staged && (reinterpret_cast<uintptr_t>(X) & 15u) == 0) {
-            if (p.log2_group == 4) return launch_sx<3, 16>(p, X, pb, stream);
-            if (p.log2_group == 5) return launch_sx<3, 32>(p, X, pb, stream);
-            return launch_sx<3, 64>(p, X, pb, stream);
+    // 3 bits, 6 to 16 tokens: CTAs that share one staged copy of X (measured
+    // on the 70B gate and down shapes: 102-111 -> 103 us at 6 tokens, 123-144
+    // -> 103-105 us at 8, 168 -> 114-120 us at 16; slower than the per-warp
+    // form below 6)
+    if constexpr (NBITS == 3) {
+        if (p.M >= 6 && p.K < ((int64_t)1 << 30) && (reinterpret_cast<uintptr_t>(X) & 15u) == 0) {
+            if (staged) {
+                if (p.log2_group == 4) return launch_sx<3, 16, NT, true>(p, X, pb, stream);
+                if (p.log2_group == 5) return launch_sx<3, 32, NT, true>(p, X, pb, stream);
+                return launch_sx<3, 64, NT, true>(p, X, pb, stream);
+            }
+            if (p.log2_group == 4) return launch_sx<3, 16, NT, false>(p, X, pb, stream);
+            if (p.log2_group == 5) return launch_sx<3, 32, NT, false>(p, X, pb, stream);
+            return launch_sx<3, 64, NT, false>(p, X, pb, stream);
         }
     }
     return staged ? launch_g<NBITS, VEC, true, NT, MX>(p, X, pb, stream)
