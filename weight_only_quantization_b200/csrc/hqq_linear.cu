@@ -192,6 +192,54 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 // an SM to itself and takes a deeper ring.
 __host__ __device__ constexpr int prefetch_of(int bn) { return bn >= 256 ? 4 : 2; }
 
+// The 32 codes of a 3-bit quad as four re-based words: word i holds codes
+// 10i .. 10i + 9 in bits 0..29 (one funnel shift of the 60-bit payload of the
+// stored words i and i + 1 from the quad's first slot, which is even).
+__device__ __forceinline__ void rebase3(const QuadCodes<3>& c, uint32_t (&r)[4]) {
+    const uint32_t sh = 2u + 3u * c.off;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = __funnelshift_r(c.w[i] << 2, i < 3 ? c.w[i + 1] : 0u, sh);
+}
+
+// Codes at bits b, b + 3 of x (b = 0, or 6 when B6) as exact floats: one
+// logic operation per code, (x & mask) | magic with the mask as the immediate
+// and the bits of 2^23 in a register (mg), then one fma pair.
+template <int B6>
+__device__ __forceinline__ float2 pair3_at(uint32_t x, uint32_t mg) {
+    constexpr uint32_t m0 = 7u << (B6 ? 6 : 0), m1 = m0 << 3;
+    uint32_t f0, f1;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(f0) : "r"(x), "n"(m0), "r"(mg));
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(f1) : "r"(x), "n"(m1), "r"(mg));
+    constexpr float i0 = B6 ? 1.0f / 64 : 1.0f, i1 = B6 ? 1.0f / 512 : 1.0f / 8;
+    constexpr float o0 = B6 ? -131072.0f : -8388608.0f, o1 = B6 ? -16384.0f : -1048576.0f;
+    return __ffma2_rn(make_float2(__uint_as_float(f0), __uint_as_float(f1)), make_float2(i0, i1),
+                      make_float2(o0, o1));
+}
+
+// Unit t (codes 8t .. 8t + 7) of a re-based 3-bit quad as fp16 weights: pair
+// (2m, 2m + 1) sits at slot 2m % 10 of word 2m / 10; slots 0-3 are read from
+// the word, 4-7 from the word shifted right by 12 and 8-9 by 24 (multiply-high
+// by the opaque k20 = 2^20 and k8 = 2^8), so two constant sets serve all.
+__device__ __forceinline__ uint4 quad_unit3(const QuadCodes<3>& c, const uint32_t (&r)[4], int t,
+                                            uint32_t mg, uint32_t k20, uint32_t k8) {
+    const __half2 sz = c.sz[t >> 1];
+    const float s = __low2float(sz), z = __high2float(sz);
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int m = 2 * (4 * t + q), sl = m % 10;
+        const uint32_t x = r[m / 10];
+        float2 cc;
+        if (sl == 0) cc = pair3_at<0>(x, mg);
+        else if (sl == 2) cc = pair3_at<1>(x, mg);
+        else if (sl == 4) cc = pair3_at<0>(__umulhi(x, k20), mg);
+        else if (sl == 6) cc = pair3_at<1>(__umulhi(x, k20), mg);
+        else cc = pair3_at<0>(__umulhi(x, k8), mg);
+        o[q] = dq2(cc, z, s);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // gridDim.z > 1: the CTAs of a (1, 1, gridDim.z) cluster split the k-tiles of
 // one output tile; each keeps its partial sums in its own tensor memory, the
 // others write theirs into rank 0's (then idle) stage buffers through
@@ -296,6 +344,8 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
     } else {
         // ---- producers of W_hat: quads of 4 units, a ring of kPrefetch k-tiles
         constexpr int kPrefetch = prefetch_of(BN);
+        uint32_t mg = 0x4B000000u, k20 = 1u << 20, k8 = 1u << 8;
+        asm volatile("" : "+r"(mg), "+r"(k20), "+r"(k8));
         // of codes in registers (indices fixed by unrolling)
         const int pw = warp - 2, j4 = lane & 1;
         const int r = pw * 16 + (lane >> 1);
@@ -323,12 +373,24 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
                     mbar_wait(empty(s), ph ^ 1u, abrt, prm.status, false);
                     uint8_t* arow = a_st + s * kABytes + r * 128;
                     const QuadCodes<NBITS>& cur = ring[u];
+                    if constexpr (NBITS == 3) {
+                        uint32_t rb[4];
+                        rebase3(cur, rb);
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const int j = 4 * j4 + t;
-                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                        if (cur.present & (1u << t)) v = quad_unit<NBITS>(cur, t);
-                        *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = v;
+                        for (int t = 0; t < 4; ++t) {
+                            const int j = 4 * j4 + t;
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                            if (cur.present & (1u << t)) v = quad_unit3(cur, rb, t, mg, k20, k8);
+                            *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = v;
+                        }
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const int j = 4 * j4 + t;
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                            if (cur.present & (1u << t)) v = quad_unit<NBITS>(cur, t);
+                            *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = v;
+                        }
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     mbar_arrive(full_a(s));
