@@ -65,14 +65,17 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
+// One test of the phase; the waiting thread may be suspended in hardware for
+// up to about 0.1 ms (the suspend-time hint) before the test fails, so that
+// waiting warps take no issue slots from the warps doing work.
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "n"(100000)
         : "memory");
     return ok != 0;
 }
@@ -204,16 +207,53 @@ __device__ __forceinline__ void rebase3(const QuadCodes<3>& c, uint32_t (&r)[4])
 // Codes at bits b, b + 3 of x (b = 0, or 6 when B6) as exact floats: one
 // logic operation per code, (x & mask) | magic with the mask as the immediate
 // and the bits of 2^23 in a register (mg), then one fma pair.
+// Constants of the 3-bit decode, made opaque once per thread so that they
+// stay in registers (packed f32x2 operations take register pairs only):
+// mg = the bits of 2^23, k20 = 2^20, k8 = 2^8, and per field pair (b, b + 3)
+// with b = 0 or 6 the multipliers (2^-b, 2^-(b+3)) and offsets
+// (-2^(23-b), -2^(20-b)) that turn 2^23 + c 2^b into c.
+struct Dec3 {
+    uint32_t mg, k20, k8;
+    float2 i0, o0, i6, o6;
+    __device__ __forceinline__ void init() {
+        mg = 0x4B000000u;
+        k20 = 1u << 20;
+        k8 = 1u << 8;
+        i0 = make_float2(1.0f, 0.125f);
+        o0 = make_float2(-8388608.0f, -1048576.0f);
+        i6 = make_float2(0.015625f, 0.001953125f);
+        o6 = make_float2(-131072.0f, -16384.0f);
+        asm volatile("" : "+r"(mg), "+r"(k20), "+r"(k8));
+        asm volatile("" : "+f"(i0.x), "+f"(i0.y), "+f"(o0.x), "+f"(o0.y));
+        asm volatile("" : "+f"(i6.x), "+f"(i6.y), "+f"(o6.x), "+f"(o6.y));
+    }
+};
+
+// fp16((c - z) s) of the codes at bits b, b + 3 of x (b = 0, or 6 when B6),
+// packed in one word, as one block: the two fields into the mantissa of 2^23
+// (one logic operation each), the exact codes (one f32x2 fma), fl32(c - z) and
+// fl32(. s) (one f32x2 add and multiply, nz = (-z, -z), ss = (s, s)), the fp16
+// pair.
 template <int B6>
-__device__ __forceinline__ float2 pair3_at(uint32_t x, uint32_t mg) {
+__device__ __forceinline__ uint32_t pair3_dq(uint32_t x, const Dec3& d, uint64_t nz, uint64_t ss) {
     constexpr uint32_t m0 = 7u << (B6 ? 6 : 0), m1 = m0 << 3;
-    uint32_t f0, f1;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(f0) : "r"(x), "n"(m0), "r"(mg));
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(f1) : "r"(x), "n"(m1), "r"(mg));
-    constexpr float i0 = B6 ? 1.0f / 64 : 1.0f, i1 = B6 ? 1.0f / 512 : 1.0f / 8;
-    constexpr float o0 = B6 ? -131072.0f : -8388608.0f, o1 = B6 ? -16384.0f : -1048576.0f;
-    return __ffma2_rn(make_float2(__uint_as_float(f0), __uint_as_float(f1)), make_float2(i0, i1),
-                      make_float2(o0, o1));
+    const float2 iv = B6 ? d.i6 : d.i0, of = B6 ? d.o6 : d.o0;
+    uint32_t h;
+    asm("{\n\t.reg .b32 a, b, lo, hi;\n\t.reg .b64 ab, iv, of, c;\n\t"
+        "lop3.b32 a, %1, %2, %4, 0xEA;\n\t"
+        "lop3.b32 b, %1, %3, %4, 0xEA;\n\t"
+        "mov.b64 ab, {a, b};\n\t"
+        "mov.b64 iv, {%5, %6};\n\t"
+        "mov.b64 of, {%7, %8};\n\t"
+        "fma.rn.f32x2 c, ab, iv, of;\n\t"
+        "add.rn.f32x2 c, c, %9;\n\t"
+        "mul.rn.f32x2 c, c, %10;\n\t"
+        "mov.b64 {lo, hi}, c;\n\t"
+        "cvt.rn.f16x2.f32 %0, hi, lo;\n\t}"
+        : "=r"(h)
+        : "r"(x), "n"(m0), "n"(m1), "r"(d.mg), "f"(iv.x), "f"(iv.y), "f"(of.x), "f"(of.y),
+          "l"(nz), "l"(ss));
+    return h;
 }
 
 // Unit t (codes 8t .. 8t + 7) of a re-based 3-bit quad as fp16 weights: pair
@@ -221,21 +261,22 @@ __device__ __forceinline__ float2 pair3_at(uint32_t x, uint32_t mg) {
 // the word, 4-7 from the word shifted right by 12 and 8-9 by 24 (multiply-high
 // by the opaque k20 = 2^20 and k8 = 2^8), so two constant sets serve all.
 __device__ __forceinline__ uint4 quad_unit3(const QuadCodes<3>& c, const uint32_t (&r)[4], int t,
-                                            uint32_t mg, uint32_t k20, uint32_t k8) {
+                                            const Dec3& d) {
     const __half2 sz = c.sz[t >> 1];
     const float s = __low2float(sz), z = __high2float(sz);
+    uint64_t ss, nz;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(nz) : "f"(-z));
     uint32_t o[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int m = 2 * (4 * t + q), sl = m % 10;
         const uint32_t x = r[m / 10];
-        float2 cc;
-        if (sl == 0) cc = pair3_at<0>(x, mg);
-        else if (sl == 2) cc = pair3_at<1>(x, mg);
-        else if (sl == 4) cc = pair3_at<0>(__umulhi(x, k20), mg);
-        else if (sl == 6) cc = pair3_at<1>(__umulhi(x, k20), mg);
-        else cc = pair3_at<0>(__umulhi(x, k8), mg);
-        o[q] = dq2(cc, z, s);
+        if (sl == 0) o[q] = pair3_dq<0>(x, d, nz, ss);
+        else if (sl == 2) o[q] = pair3_dq<1>(x, d, nz, ss);
+        else if (sl == 4) o[q] = pair3_dq<0>(__umulhi(x, d.k20), d, nz, ss);
+        else if (sl == 6) o[q] = pair3_dq<1>(__umulhi(x, d.k20), d, nz, ss);
+        else o[q] = pair3_dq<0>(__umulhi(x, d.k8), d, nz, ss);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -344,8 +385,8 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
     } else {
         // ---- producers of W_hat: quads of 4 units, a ring of kPrefetch k-tiles
         constexpr int kPrefetch = prefetch_of(BN);
-        uint32_t mg = 0x4B000000u, k20 = 1u << 20, k8 = 1u << 8;
-        asm volatile("" : "+r"(mg), "+r"(k20), "+r"(k8));
+        Dec3 dec;
+        if constexpr (NBITS == 3) dec.init();
         // of codes in registers (indices fixed by unrolling)
         const int pw = warp - 2, j4 = lane & 1;
         const int r = pw * 16 + (lane >> 1);
@@ -377,19 +418,17 @@ linear_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ 
                         uint32_t rb[4];
                         rebase3(cur, rb);
 #pragma unroll
-                        for (int t = 0; t < 4; ++t) {
+                        for (int t = 0; t < 4; ++t) {                // absent units: s = z = 0
                             const int j = 4 * j4 + t;
-                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                            if (cur.present & (1u << t)) v = quad_unit3(cur, rb, t, mg, k20, k8);
-                            *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = v;
+                            *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) =
+                                quad_unit3(cur, rb, t, dec);
                         }
                     } else {
 #pragma unroll
-                        for (int t = 0; t < 4; ++t) {
+                        for (int t = 0; t < 4; ++t) {                // absent units: s = z = 0
                             const int j = 4 * j4 + t;
-                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                            if (cur.present & (1u << t)) v = quad_unit<NBITS>(cur, t);
-                            *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = v;
+                            *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) =
+                                quad_unit<NBITS>(cur, t);
                         }
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -188,6 +188,7 @@ struct QuadCodes {
     __half2 sz[2];                                     // (s, z) of units 0-1 and 2-3
     uint32_t off;                                      // 3 bits: slot of code 0 in w[0]
     uint32_t present;                                  // bit t: unit t inside the matrix
+                                                       // (absent units decode to 0)
 };
 
 // (s, z) of group g: the stored fp16 values, or restored from their 8-bit
@@ -267,6 +268,9 @@ __device__ __forceinline__ void load_quad(const LinearParams& p, int64_t fbase, 
     c.sz[0] = group_sz(p, g);
     c.sz[1] = c.sz[0];
     if (p.log2_group == 4 && (c.present & 4u)) c.sz[1] = group_sz(p, g + 1);
+    // K is a multiple of 16: units 0-1 are both present, and so are 2-3 or
+    // neither; absent units get s = z = 0, so their weights are exactly 0
+    if (!(c.present & 4u)) c.sz[1] = __float2half2_rn(0.0f);
 }
 
 // Weights of unit t (0..3) of a loaded quad.
