@@ -214,18 +214,20 @@ __device__ __forceinline__ void rebase3(const QuadCodes<3>& c, uint32_t (&r)[4])
 // (-2^(23-b), -2^(20-b)) that turn 2^23 + c 2^b into c.
 struct Dec3 {
     uint32_t mg, k20, k8;
-    float2 i0, o0, i6, o6;
+    uint64_t i0, o0, i6, o6;                  // f32x2 pairs, low word first
     __device__ __forceinline__ void init() {
         mg = 0x4B000000u;
         k20 = 1u << 20;
         k8 = 1u << 8;
-        i0 = make_float2(1.0f, 0.125f);
-        o0 = make_float2(-8388608.0f, -1048576.0f);
-        i6 = make_float2(0.015625f, 0.001953125f);
-        o6 = make_float2(-131072.0f, -16384.0f);
+        auto pack = [](float lo, float hi) {
+            return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+        };
+        i0 = pack(1.0f, 0.125f);
+        o0 = pack(-8388608.0f, -1048576.0f);
+        i6 = pack(0.015625f, 0.001953125f);
+        o6 = pack(-131072.0f, -16384.0f);
         asm volatile("" : "+r"(mg), "+r"(k20), "+r"(k8));
-        asm volatile("" : "+f"(i0.x), "+f"(i0.y), "+f"(o0.x), "+f"(o0.y));
-        asm volatile("" : "+f"(i6.x), "+f"(i6.y), "+f"(o6.x), "+f"(o6.y));
+        asm volatile("" : "+l"(i0), "+l"(o0), "+l"(i6), "+l"(o6));
     }
 };
 
@@ -237,21 +239,18 @@ struct Dec3 {
 template <int B6>
 __device__ __forceinline__ uint32_t pair3_dq(uint32_t x, const Dec3& d, uint64_t nz, uint64_t ss) {
     constexpr uint32_t m0 = 7u << (B6 ? 6 : 0), m1 = m0 << 3;
-    const float2 iv = B6 ? d.i6 : d.i0, of = B6 ? d.o6 : d.o0;
     uint32_t h;
-    asm("{\n\t.reg .b32 a, b, lo, hi;\n\t.reg .b64 ab, iv, of, c;\n\t"
+    asm("{\n\t.reg .b32 a, b, lo, hi;\n\t.reg .b64 ab, c;\n\t"
         "lop3.b32 a, %1, %2, %4, 0xEA;\n\t"
         "lop3.b32 b, %1, %3, %4, 0xEA;\n\t"
         "mov.b64 ab, {a, b};\n\t"
-        "mov.b64 iv, {%5, %6};\n\t"
-        "mov.b64 of, {%7, %8};\n\t"
-        "fma.rn.f32x2 c, ab, iv, of;\n\t"
-        "add.rn.f32x2 c, c, %9;\n\t"
-        "mul.rn.f32x2 c, c, %10;\n\t"
+        "fma.rn.f32x2 c, ab, %5, %6;\n\t"
+        "add.rn.f32x2 c, c, %7;\n\t"
+        "mul.rn.f32x2 c, c, %8;\n\t"
         "mov.b64 {lo, hi}, c;\n\t"
         "cvt.rn.f16x2.f32 %0, hi, lo;\n\t}"
         : "=r"(h)
-        : "r"(x), "n"(m0), "n"(m1), "r"(d.mg), "f"(iv.x), "f"(iv.y), "f"(of.x), "f"(of.y),
+        : "r"(x), "n"(m0), "n"(m1), "r"(d.mg), "l"(B6 ? d.i6 : d.i0), "l"(B6 ? d.o6 : d.o0),
           "l"(nz), "l"(ss));
     return h;
 }
