@@ -935,8 +935,9 @@ def run_lowrank(views, hqq, dev, fma_peak, pg):
     """Times the low-rank residual B A of the quantization error W - W_hat
     (rank 16 from a 32-column Gaussian sketch, 2 power iterations) on the first
     seven matrices (one layer of the model-shaped sets).  The products with
-    Delta W, (2 * iters + 2) * rows * cols * sketch fp32 FMAs per matrix, are
-    reported against the fp32 FMA lane peak."""
+    Delta W, (2 * iters + 2) * rows * cols * sketch multiply-adds per matrix
+    (each as three split-tf32 tensor-core products, fp32 accurate), are
+    reported over the whole call's time against the fp32 FMA lane peak."""
     import torch
     sub = views[:7]
     rank, sketch, iters = 16, 32, 2
@@ -961,7 +962,8 @@ def run_lowrank(views, hqq, dev, fma_peak, pg):
     ms = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps], pg, dev)[0]
     fmas = sum((2 * iters + 2) * q.rows * q.cols * sketch for _, q, _ in sub)
     return {"what": "rank-16 residual of W - W_hat by randomized subspace iteration (32-column "
-                    "sketch, 2 power iterations), Delta W formed inside the fp32 products",
+                    "sketch, 2 power iterations), Delta W formed in fp32 inside the products "
+                    "(split-tf32 tensor-core MMAs); rate over the whole call",
             "matrices": len(sub), "ms_per_pass": ms,
             "products_tfma_s": fmas / (ms / 1e3) / 1e12,
             "fma_frac": fmas / (ms / 1e3) / 1e12 / fma_peak,
