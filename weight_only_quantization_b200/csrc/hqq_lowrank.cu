@@ -89,12 +89,14 @@ __device__ __forceinline__ void unit_delta(const UnitLoad& u, float (&d)[8]) {
 // a0 = (g, q), a1 = (g + 8, q), a2 = (g, q + 4), a3 = (g + 8, q + 4);
 // B (8 x 8) b0 = (k q, column g), b1 = (k q + 4, column g); D c0 = (g, 2q),
 // c1 = (g, 2q + 1), c2 = (g + 8, 2q), c3 = (g + 8, 2q + 1).
+// x rounded to tf32 (10 mantissa bits), half-way cases away from zero, as bit
+// operations on the magnitude: a carry out of the mantissa moves to the next
+// binade, as it should (finite inputs only; the products' operands are).
 __device__ __forceinline__ uint32_t tf32_of(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
 }
 
+// x = hi + lo with hi = tf32(x) and lo = tf32(x - hi) (x - hi is exact in fp32).
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
     hi = tf32_of(x);
     lo = tf32_of(__fsub_rn(x, __uint_as_float(hi)));
