@@ -28,13 +28,20 @@
 //    bound on |W - Q^-1(Q(W))| lies below the shrink threshold, W_e is exactly
 //    zero, so sp1 reduces to W - W_e = W.
 #pragma once
+#include <cmath>
 #include <type_traits>
 
 #include "hqq_common.cuh"
 
 namespace hqq {
 
-constexpr int kQWarps = 8;                 // warps per CTA (share the 32 KiB table)
+// Warps per CTA (they share the power tables): 8 in each of two CTAs per SM
+// (up to 128 registers per thread), or 20 in one CTA per SM, whose 96
+// registers hold the single-precision solver without spills; the half-
+// precision solver (its fp16 steps need more registers) keeps 8.  (Single
+// precision, 3-bit 28672 x 8192: 20 warps 0.90 ms, 2 x 8 warps 0.98 ms,
+// 1 x 16 warps 0.94 ms, 2 x 10 warps 0.94 ms.)
+constexpr int kWideWarps = 20;
 constexpr int kChunk = 2560;               // weights per warp chunk
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -670,8 +677,9 @@ __device__ __forceinline__ void final_pass(const QuantParams& prm, __half* s_w, 
 // once at most PARK/4 of the phase-B slots are busy.  TAB2: combined power
 // table (off for G = 16, whose per-group state already fills the shared memory
 // that two resident CTAs per SM can have).
-template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK, bool TAB2, bool HALF>
-__global__ void __launch_bounds__(kQWarps * 32, 2)
+template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK, bool TAB2, bool HALF,
+          int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, WARPS > 8 ? 1 : 2)
 quantize_kernel(const __grid_constant__ QuantParams prm) {
     using C = QCfg<NBITS, G, NB>;      // phase A layout (and the chunk's shared memory)
     using CB = QCfg<NBITS, G, NBB>;    // phase B layout
@@ -718,8 +726,8 @@ quantize_kernel(const __grid_constant__ QuantParams prm) {
     int np = 0;                        // groups parked in the pool by the last yield
 
     const int64_t n_chunks = (prm.n_elems + kChunk - 1) / kChunk;
-    for (int64_t chunk = (int64_t)blockIdx.x * kQWarps + warp; chunk < n_chunks;
-         chunk += (int64_t)gridDim.x * kQWarps) {
+    for (int64_t chunk = (int64_t)blockIdx.x * WARPS + warp; chunk < n_chunks;
+         chunk += (int64_t)gridDim.x * WARPS) {
         const int64_t e0 = chunk * kChunk;
         const int64_t left = prm.n_elems - e0;
         const int n_here = left < kChunk ? (int)left : kChunk;
@@ -779,7 +787,7 @@ quantize_kernel(const __grid_constant__ QuantParams prm) {
             const int subb = lane / CB::K;
             const int klb = lane % CB::K;
             const bool leadb = klb == 0;
-            const bool more = CARRY && chunk + (int64_t)gridDim.x * kQWarps < n_chunks;
+            const bool more = CARRY && chunk + (int64_t)gridDim.x * WARPS < n_chunks;
             const int nq = np + qn;
             int head = 0;
             bool live = false;
@@ -875,27 +883,70 @@ quantize_kernel(const __grid_constant__ QuantParams prm) {
     }
 }
 
+// A kernel instance with its dynamic shared memory set, and the warps it keeps
+// resident per SM.
+template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK, bool HALF, bool TAB2,
+          int WARPS>
+struct QuantLaunch {
+    using C = QCfg<NBITS, G, NB>;
+    using CB = QCfg<NBITS, G, NBB>;
+    static constexpr int SMEM = WARPS * (C::CHUNK_BYTES + (CARRY ? CB::POOL_BYTES : 0));
+    static_assert(SMEM + sizeof(QuantSmem<TAB2, HALF>) <= 227 * 1024, "shared memory per CTA");
+    static constexpr auto kern = quantize_kernel<NBITS, G, NB, NBB, CARRY, PARK, TAB2, HALF, WARPS>;
+    int per_sm = 1;
+    cudaError_t prepare() {
+        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               SMEM);
+        if (err != cudaSuccess) return err;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WARPS * 32, SMEM);
+        if (per_sm < 1) per_sm = 1;
+        return err;
+    }
+    // resident warps per SM x (chunks per warp / rounds of chunks): the share
+    // of the warp-slots that the chunks fill
+    double fill(int64_t n_chunks, int sms) const {
+        const double rounds = (double)n_chunks / ((double)sms * per_sm * WARPS);
+        return rounds / std::ceil(rounds);
+    }
+    cudaError_t launch(const QuantParams& prm, int64_t n_chunks, int sms, cudaStream_t stream) {
+        const int64_t want = (n_chunks + WARPS - 1) / WARPS;
+        const int64_t cap = (int64_t)sms * per_sm;
+        const unsigned grid = (unsigned)(want < cap ? want : cap);
+        kern<<<grid, WARPS * 32, SMEM, stream>>>(prm);
+        return cudaGetLastError();
+    }
+};
+
+// The single-precision kernels come in two shapes where the shared memory
+// allows: 20 warps in one CTA per SM (more warps to hide latency: 9% faster
+// per SM on large matrices) and 8 warps in each of two CTAs per SM.  Chunks are dealt to
+// warps round-robin, so a matrix of few chunks leaves part of its last round
+// of warps idle; the launch takes the shape whose filled share of warp-slots,
+// weighted by that per-SM speed, is larger (the 70B q/o/gate/up/down shapes
+// take 20 warps, 4096 x 4096 and the 1024-row k/v take 8).
 template <int NBITS, int G, int NB, int NBB, bool CARRY, int PARK, bool HALF,
           bool TAB2 = (G > 16)>
 static cudaError_t launch_quantize_g(const QuantParams& prm, cudaStream_t stream) {
-    using C = QCfg<NBITS, G, NB>;
-    using CB = QCfg<NBITS, G, NBB>;
-    constexpr int SMEM = kQWarps * (C::CHUNK_BYTES + (CARRY ? CB::POOL_BYTES : 0));
-    auto kern = quantize_kernel<NBITS, G, NB, NBB, CARRY, PARK, TAB2, HALF>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    if (err != cudaSuccess) return err;
-    int dev = 0, sms = 148, per_sm = 1;
+    int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQWarps * 32, SMEM);
-    if (err != cudaSuccess) return err;
-    if (per_sm < 1) per_sm = 1;
     const int64_t n_chunks = (prm.n_elems + kChunk - 1) / kChunk;
-    const int64_t want = (n_chunks + kQWarps - 1) / kQWarps;
-    const int64_t cap = (int64_t)sms * per_sm;
-    const unsigned grid = (unsigned)(want < cap ? want : cap);
-    kern<<<grid, kQWarps * 32, SMEM, stream>>>(prm);
-    return cudaGetLastError();
+    QuantLaunch<NBITS, G, NB, NBB, CARRY, PARK, HALF, TAB2, 8> l8;
+    cudaError_t err = l8.prepare();
+    if (err != cudaSuccess) return err;
+    using C = QCfg<NBITS, G, NB>;
+    using CB = QCfg<NBITS, G, NBB>;
+    constexpr int kWarpBytes = C::CHUNK_BYTES + (CARRY ? CB::POOL_BYTES : 0);
+    constexpr bool kWide = !HALF && kWideWarps * kWarpBytes +
+                                        (int)sizeof(QuantSmem<TAB2, HALF>) <= 227 * 1024;
+    if constexpr (kWide) {
+        QuantLaunch<NBITS, G, NB, NBB, CARRY, PARK, HALF, TAB2, kWideWarps> lw;
+        err = lw.prepare();
+        if (err != cudaSuccess) return err;
+        if (1.09 * lw.fill(n_chunks, sms) > l8.fill(n_chunks, sms))
+            return lw.launch(prm, n_chunks, sms, stream);
+    }
+    return l8.launch(prm, n_chunks, sms, stream);
 }
 
 // 16 weights per lane in both phases.  4 bit: park the last busy groups of a
