@@ -36,11 +36,12 @@
 namespace hqq {
 
 // Warps per CTA (they share the power tables): 8 in each of two CTAs per SM
-// (up to 128 registers per thread), or 20 in one CTA per SM, whose 96
-// registers hold the single-precision solver without spills; the half-
-// precision solver (its fp16 steps need more registers) keeps 8.  (Single
-// precision, 3-bit 28672 x 8192: 20 warps 0.90 ms, 2 x 8 warps 0.98 ms,
-// 1 x 16 warps 0.94 ms, 2 x 10 warps 0.94 ms.)
+// (up to 128 registers per thread), or 20 in one CTA per SM at 96 registers
+// (no spills in single precision, a few bytes in half precision).  3-bit
+// 28672 x 8192, single precision: 20 warps 0.90 ms, 2 x 8 warps 0.98 ms,
+// 1 x 16 warps 0.94 ms, 2 x 10 warps 0.94 ms, 22 warps (88 registers)
+// 1.01 ms, 24 warps (80 registers) 0.92 ms; half precision: 20 warps
+// 1.21 ms, 2 x 8 warps 1.42 ms.
 constexpr int kWideWarps = 20;
 constexpr int kChunk = 2560;               // weights per warp chunk
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -917,9 +918,10 @@ struct QuantLaunch {
     }
 };
 
-// The single-precision kernels come in two shapes where the shared memory
-// allows: 20 warps in one CTA per SM (more warps to hide latency: 9% faster
-// per SM on large matrices) and 8 warps in each of two CTAs per SM.  Chunks are dealt to
+// The kernels come in two shapes where the shared memory allows: 20 warps in
+// one CTA per SM (more warps to hide latency: 9% faster per SM on large
+// matrices in single precision, 15% in half precision) and 8 warps in each
+// of two CTAs per SM.  Chunks are dealt to
 // warps round-robin, so a matrix of few chunks leaves part of its last round
 // of warps idle; the launch takes the shape whose filled share of warp-slots,
 // weighted by that per-SM speed, is larger (the 70B q/o/gate/up/down shapes
@@ -937,8 +939,8 @@ static cudaError_t launch_quantize_g(const QuantParams& prm, cudaStream_t stream
     using C = QCfg<NBITS, G, NB>;
     using CB = QCfg<NBITS, G, NBB>;
     constexpr int kWarpBytes = C::CHUNK_BYTES + (CARRY ? CB::POOL_BYTES : 0);
-    constexpr bool kWide = !HALF && kWideWarps * kWarpBytes +
-                                        (int)sizeof(QuantSmem<TAB2, HALF>) <= 227 * 1024;
+    constexpr bool kWide =
+        kWideWarps * kWarpBytes + (int)sizeof(QuantSmem<TAB2, HALF>) <= 227 * 1024;
     if constexpr (kWide) {
         QuantLaunch<NBITS, G, NB, NBB, CARRY, PARK, HALF, TAB2, kWideWarps> lw;
         err = lw.prepare();
