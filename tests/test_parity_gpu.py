@@ -111,6 +111,20 @@ def test_shrink_active(hqq, nbits, group, std):
     assert st["code_match"] == 1.0 and st["iters_equal"] == 1.0
 
 
+# ------------------------- the 20-warp CTA shape, every group compared in full
+@pytest.mark.parametrize("nbits,group", [(3, 64), (2, 32), (4, 64)])
+@pytest.mark.parametrize("std", [0.02, 3.0])
+def test_wide_ctas_full(hqq, nbits, group, std):
+    """4096 x 8192 (13108 chunks of 2560 weights): enough chunks that the
+    launch takes one 20-warp CTA per SM on a 148-SM B200 rather than two
+    8-warp CTAs.  Every group against the oracle, with the shrink inactive
+    (std 0.02) and active (std 3), so the clamp and exact-shrink paths of that
+    kernel shape run on full-size data."""
+    W, Wn = _dev_weights((4096, 8192), seed=25, stream=nbits, std=std)
+    _, _, st = _check(hqq, W, Wn, nbits, group, f"wide std {std} {nbits}b g{group}")
+    assert st["code_match"] == 1.0 and st["iters_equal"] == 1.0
+
+
 # ---------------------------------------------------------- solver parameters
 @pytest.mark.parametrize("kw", [
     dict(iters=0), dict(iters=1), dict(iters=255), dict(p=1.0), dict(p=0.5),

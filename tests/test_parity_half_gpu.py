@@ -118,6 +118,17 @@ def test_shrink_active(hqq, nbits, group, std):
     assert st["code_match"] == 1.0 and st["iters_equal"] == 1.0
 
 
+@pytest.mark.parametrize("nbits,group", [(3, 64), (4, 64)])
+@pytest.mark.parametrize("std", [0.02, 3.0])
+def test_wide_ctas_full(hqq, nbits, group, std):
+    """4096 x 8192: enough chunks for one 20-warp CTA per SM on a 148-SM B200;
+    every group against the oracle's half-precision solver, shrink inactive
+    and active."""
+    W, Wn = _dev_weights((4096, 8192), seed=25, stream=nbits, std=std)
+    _, _, st = _check(W, Wn, nbits, group, f"fp16 wide std {std} {nbits}b g{group}")
+    assert st["code_match"] == 1.0 and st["iters_equal"] == 1.0
+
+
 @pytest.mark.parametrize("kw", [
     dict(iters=0), dict(iters=1), dict(iters=255), dict(p=1.0), dict(p=0.5),
     dict(p=0.05), dict(beta=0.1), dict(beta=50.0), dict(kappa=1.5), dict(kappa=0.9),
